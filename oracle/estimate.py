@@ -1,0 +1,132 @@
+"""Estimators on the codes: attention logits, MSE dequantisation, decode
+attention and top-k search (TEST INFRASTRUCTURE).
+
+* Inner-product estimate ("TurboQuant explainer" (m.163.com), "第二步：QJL"
+  and its identity E[<y, Q^-1(Q(x))>] = <y, x>).  For a query q and a key
+  stored as (n, idx, gamma, s):
+
+      q_rot = H D q / sqrt(d_pad)            (the rotated query)
+      u     = S q_rot                        (the projected query)
+      l     = n * ( sum_j q_rot_j c[idx_j]
+                    + gamma * sqrt(pi/2) / m * sum_i u_i (2 s_i - 1) )
+
+  The first term is <q, k_mse> because the rotation is orthogonal; the second
+  is the QJL correction.  Logits are raw inner products (no 1/sqrt(d) scale).
+  GQA: query head h reads KV head h // group.
+* MSE-only values ("TurboQuant explainer", "速度" - logits from compressed KV;
+  zhidx turboquant_plus article - asymmetric K/V):
+      v_hat = n * D o (H c[idx]) / sqrt(d_pad), first d coordinates.
+* Decode attention: o = sum_j softmax_j(scale * l_j) v_hat_j with the
+  maximum subtracted; scale defaults to 1/sqrt(d).  Plain token-by-token
+  fp64; the GPU's chunked online softmax is a reassociation of this sum.
+* Search ("TurboQuant explainer", "向量搜索"): the k database ids with the
+  largest estimate, ties to the lower id.
+
+All arithmetic in fp64; the stored fp16 norms are used as stored.
+"""
+import numpy as np
+
+from .codec import rotate, unrotate, pad
+
+
+def prep_queries(q, D, S):
+    """Rotated queries q_rot [n_q, d_pad] and projections u [n_q, m] (fp64)."""
+    d_pad = D.shape[0]
+    q_rot = rotate(pad(np.asarray(q, dtype=np.float64), d_pad), D)
+    u = q_rot @ np.asarray(S, dtype=np.float64).T if S is not None else None
+    return q_rot, u
+
+
+def logits_from_codes(q_rot, u, idx, signs, norm_f16, rnorm_f16, centroids, m):
+    """Estimates for every (query, key) pair: [n_q, n_keys] fp64.
+
+    q_rot [n_q, d_pad], u [n_q, m] (None for MSE-only codes), idx [n_keys, d_pad],
+    signs [n_keys, m] 0/1 (None for MSE-only), norms fp16 [n_keys].
+    """
+    c = np.asarray(centroids, dtype=np.float64)
+    k_mse = c[idx]                                           # [n_keys, d_pad]
+    base = q_rot @ k_mse.T
+    if signs is not None:
+        pm = 2.0 * signs.astype(np.float64) - 1.0            # [n_keys, m]
+        corr = (u @ pm.T) * (np.sqrt(np.pi / 2.0) / m) * rnorm_f16.astype(np.float64)[None, :]
+        base = base + corr
+    return base * norm_f16.astype(np.float64)[None, :]
+
+
+def logits_gqa(q, D, S, idx, signs, norm_f16, rnorm_f16, centroids, m, n_kv_heads, group, n_keys):
+    """tq_logits semantics: q [n_kv_heads*group, d]; keys of head g are rows
+    g*n_keys .. (g+1)*n_keys-1 of idx/signs/norms.  Returns [n_q, n_keys]."""
+    q_rot, u = prep_queries(q, D, S)
+    out = np.zeros((q.shape[0], n_keys), dtype=np.float64)
+    for h in range(q.shape[0]):
+        g = h // group
+        sl = slice(g * n_keys, (g + 1) * n_keys)
+        out[h] = logits_from_codes(q_rot[h:h + 1], None if u is None else u[h:h + 1],
+                                   idx[sl], None if signs is None else signs[sl],
+                                   norm_f16[sl], None if rnorm_f16 is None else rnorm_f16[sl],
+                                   centroids, m)[0]
+    return out
+
+
+def dequant_mse(idx, norm_f16, centroids, D, d):
+    """v_hat rows [n, d] (fp64) from MSE-only codes."""
+    y = np.asarray(centroids, dtype=np.float64)[idx]
+    return unrotate(y, D)[:, :d] * norm_f16.astype(np.float64)[:, None]
+
+
+def softmax_attend(logit_row, values, scale):
+    """o = sum_j p_j values_j with p = softmax(scale * logit_row), max subtracted."""
+    s = scale * np.asarray(logit_row, dtype=np.float64)
+    s = s - np.max(s)
+    p = np.exp(s)
+    p = p / np.sum(p)
+    return p @ values
+
+
+def decode_attention(q, kD, kS, k_idx, k_signs, k_norm, k_rnorm, k_cent, km,
+                     vD, v_idx, v_norm, v_cent, d, seq_lens, Hq, Hkv, max_tokens,
+                     scale=0.0, pairs=None):
+    """tq_decode_attn semantics.
+
+    q [B, Hq, d]; key/value vector index = (b*Hkv + g)*max_tokens + t.
+    Returns out [B, Hq, d] (fp64); rows not in `pairs` (list of (b, h)) are NaN
+    when `pairs` is given.
+    """
+    B = q.shape[0]
+    group = Hq // Hkv
+    if scale == 0.0:
+        scale = 1.0 / np.sqrt(d)
+    out = np.full((B, Hq, d), np.nan)
+    todo = pairs if pairs is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    cache = {}
+    for (b, h) in todo:
+        g = h // group
+        L = int(seq_lens[b])
+        if L == 0:
+            out[b, h] = 0.0
+            continue
+        base = (b * Hkv + g) * max_tokens
+        sl = slice(base, base + L)
+        q_rot, u = prep_queries(q[b, h][None, :], kD, kS)
+        lg = logits_from_codes(q_rot, u, k_idx[sl], k_signs[sl], k_norm[sl], k_rnorm[sl], k_cent, km)[0]
+        key = (b, g)
+        if key not in cache:
+            cache[key] = dequant_mse(v_idx[sl], v_norm[sl], v_cent, vD, d)
+        out[b, h] = softmax_attend(lg, cache[key], scale)
+    return out
+
+
+def topk(scores, k):
+    """Top-k column ids per row by descending score, ties to the lower id."""
+    scores = np.asarray(scores, dtype=np.float64)
+    n = scores.shape[1]
+    ids = np.broadcast_to(np.arange(n), scores.shape)
+    order = np.lexsort((ids, -scores), axis=1)   # primary: -score, secondary: id
+    top = order[:, :k]
+    return top.astype(np.int64), np.take_along_axis(scores, top, axis=1)
+
+
+def recall_at_k(found, truth):
+    """Mean over rows of |found_row ∩ truth_row| / k."""
+    k = truth.shape[1]
+    return float(np.mean([len(set(f) & set(t)) / k for f, t in zip(found, truth)]))
