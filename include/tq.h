@@ -1,0 +1,197 @@
+/*
+ * tq.h - C ABI of the TurboQuant codec library for NVIDIA B200 (sm_100a).
+ *
+ * The library quantizes key/value vectors with a random rotation (sign flips
+ * then a Walsh-Hadamard transform), a per-vector norm, a Lloyd-Max scalar
+ * code and a 1-bit QJL sketch of the residual, and computes attention logits,
+ * decode attention and top-k inner-product search directly from the packed
+ * codes.
+ *
+ * Sources (web articles about Google's TurboQuant; they print no code):
+ *  [E1] "TurboQuant explainer" (m.163.com), section "TurboQuant 怎么做的",
+ *       "第一步：PolarQuant": random rotation, then one precomputed Max-Lloyd
+ *       table for every coordinate, b-1 bits, no per-block normalisation.
+ *  [E2] same page, "第二步：QJL": JL transform of the residual kept as sign
+ *       bits, estimator with E[<y, Q^-1(Q(x))>] = <y, x>.
+ *  [E3] same page, "合起来": b-1 + 1 = b bits per value.
+ *  [E4] same page, "速度": attention logits computed from 4-bit codes.
+ *  [E5] same page, "向量搜索": inner-product nearest-neighbour search.
+ *  [Z1] zhidx turboquant_plus article, "01 turboquant_plus：介绍与详解": WHT
+ *       rotation; turbo4 = 4.25 bit/value; asymmetric K/V; block layout.
+ *
+ * Conventions (all entry points):
+ *  - The caller owns every buffer; the library allocates no memory.  Device
+ *    pointers must be device (or managed) memory of the current CUDA device.
+ *  - Kernels are launched asynchronously on `stream` (NULL = legacy default
+ *    stream).  The return value reports host-side validation and launch
+ *    errors only.
+ *  - Return value: TQ_OK or a negative TQ_E* status.  On error nothing is
+ *    launched and no output is written; tq_last_error() gives a message
+ *    (thread-local, valid until the next call on that thread).
+ *  - Code buffers must be 16-byte aligned; float/fp16 arrays 4-byte/2-byte.
+ *
+ * Code layout (canonical; produced by tq_quantize, consumed by every reader):
+ *   Vectors are grouped in tiles of 32 consecutive vectors; the last tile is
+ *   zero-filled.  A tile holds kb bit-planes (plane p = bit p of each index),
+ *   each 32 x d_pad/8 bytes with vector t at byte offset t*d_pad/8 and
+ *   coordinate j at bit j%32 of little-endian 32-bit word j/32; then (product
+ *   mode) the QJL signs, 32 x m/8 bytes, sign i at bit i%32 of word i/32.
+ *   kb = bits-1 (TQ_MODE_PROD) or bits (TQ_MODE_MSE).  Norms ||x|| and
+ *   residual norms ||r|| are separate fp16 arrays (IEEE half bit patterns),
+ *   one per vector.  For multi-head data, vector index =
+ *   (sequence*H_kv + head)*n_tokens + token.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* tq_stream_t; /* same type as cudaStream_t */
+
+/* status codes */
+#define TQ_OK 0
+#define TQ_EINVAL (-1)        /* invalid argument (null, size, alignment) */
+#define TQ_EUNSUPPORTED (-2)  /* valid but not implemented for this shape */
+#define TQ_ECUDA (-3)         /* CUDA launch/runtime error; see tq_last_error */
+
+/* code modes */
+#define TQ_MODE_PROD 0 /* (bits-1)-bit Lloyd-Max code + m QJL sign bits [E1][E2][E3] */
+#define TQ_MODE_MSE 1  /* bits-bit Lloyd-Max code only (values; 2/pi-biased inner products) */
+
+/* input element types */
+#define TQ_F32 0
+#define TQ_F16 1
+#define TQ_BF16 2
+
+/*
+ * Quantizer description.  d: input dimension (1..d_pad); d_pad: rotation
+ * size, 128 or 256; bits: total bits b (PROD: 2..4, MSE: 1..4); m: QJL rows
+ * (PROD: a multiple of 32, 32..256; MSE: 0).  The four device arrays are
+ * produced once by tq_make_codebook / tq_make_params and copied to the device
+ * by the caller:
+ *   centroids  [2^kb]   fp32, ascending, odd-symmetric
+ *   thresholds [2^kb-1] fp32, midpoints of neighbouring centroids
+ *   signs_D    [d_pad]  int8, +1 / -1
+ *   S          [m*d_pad] fp16 bit patterns, row-major (NULL in MSE mode)
+ */
+typedef struct tq_params {
+  int32_t d;
+  int32_t d_pad;
+  int32_t bits;
+  int32_t mode;
+  int32_t m;
+  int32_t reserved;
+  const float* centroids;
+  const float* thresholds;
+  const int8_t* signs_D;
+  const uint16_t* S;
+} tq_params;
+
+/*
+ * tq_make_codebook - Lloyd-Max codebook for the rotated-coordinate law [E1].
+ * Host memory only; no device.  The law is that of one coordinate of a
+ * uniform random unit vector in R^d_pad, density proportional to
+ * (1-t^2)^((d_pad-3)/2) on (-1,1) (the "Beta" law of [E1]).  Writes 2^kb
+ * centroids (fp64 Lloyd-Max fixed point rounded to fp32) and 2^kb-1
+ * thresholds (fp32 rounding of the exact midpoints of the fp32 centroids).
+ * d_pad: 4..4096 power of two; kb: 1..4.  Returns TQ_EINVAL on bad arguments.
+ */
+int tq_make_codebook(int d_pad, int kb, float* centroids, float* thresholds);
+
+/*
+ * tq_make_params - random sign flips D and QJL matrix S [E1][E2][Z1].
+ * Host memory only.  Generator: Philox4x32-10 keyed by seed (low 32 bits,
+ * high 32 bits); block i of stream s uses counter (i, s, 0, 0) and its four
+ * words are words 4i..4i+3 of the stream.  D[j] = -1 if bit 0 of word j of
+ * stream 0 is set, else +1.  S (m x d_pad, row-major) entries 2p, 2p+1 are
+ * the Box-Muller pair of words 2p, 2p+1 of stream 1, u = (w + 0.5)/2^32,
+ * (sqrt(-2 ln u_a) cos(2 pi u_b), sqrt(-2 ln u_a) sin(2 pi u_b)), rounded to
+ * fp16 (nearest even).  S may be NULL when m == 0.
+ */
+int tq_make_params(int d_pad, int m, uint64_t seed, int8_t* D, uint16_t* S);
+
+/* Bytes of a code buffer holding n_vec vectors (whole 32-vector tiles). */
+int64_t tq_code_bytes(int d_pad, int kb, int m, int64_t n_vec);
+
+/*
+ * tq_quantize - encode n_vec vectors [E1][E2].
+ *   x: device, n_vec rows of d elements of `dtype`, row stride ld elements
+ *      (ld >= d; x and ld*elem_size must be 16-byte aligned, d*elem_size a
+ *      multiple of 16).
+ *   codes: device, tq_code_bytes(d_pad, kb, m, n_vec) bytes (tail zeroed).
+ *   norms, rnorms: device fp16 [n_vec]; rnorms ignored (may be NULL) in MSE mode.
+ * Per vector: n = ||x||, x_hat = x/n (0 for n = 0), zero-pad to d_pad,
+ * y = H D x_hat / sqrt(d_pad), idx_j = #{l : y_j > t_l}, r = y - c[idx],
+ * gamma = ||r||, sign_i = [(S r)_i >= 0].  Norms are stored as fp16 (nearest
+ * even; values above 65504 become +inf).
+ */
+int tq_quantize(const tq_params* p, const void* x, int dtype, int64_t n_vec, int64_t ld,
+                void* codes, uint16_t* norms, uint16_t* rnorms, tq_stream_t stream);
+
+/*
+ * tq_logits - attention logits straight from the codes [E2][E4].
+ *   q: device fp32 [n_q][d], n_q = n_kv_heads*group; query head h reads KV
+ *      head h/group (GQA).
+ *   codes/norms/rnorms: n_kv_heads*n_keys vectors; keys of head g are
+ *      vectors g*n_keys .. g*n_keys+n_keys-1.
+ *   logits: device fp32 [n_q][n_keys], raw inner-product estimates (no 1/sqrt(d)):
+ *      l = n*( <q_rot, c[idx]> + gamma*sqrt(pi/2)/m*<S q_rot, 2s-1> ),
+ *      q_rot = H D q / sqrt(d_pad).  MSE-mode codes give n*<q_rot, c[idx]>.
+ *   workspace: device, >= tq_logits_workspace(p, n_q) bytes, 16-byte aligned.
+ * Supported: d_pad 128 with kb <= 3, d_pad 256 with kb <= 2.
+ */
+int64_t tq_logits_workspace(const tq_params* p, int n_q);
+int tq_logits(const tq_params* p, const float* q, int n_q, int group, const void* codes,
+              const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys, int n_kv_heads,
+              float* logits, void* workspace, int64_t workspace_bytes, tq_stream_t stream);
+
+/*
+ * tq_decode_attn - one decode step of attention over compressed K (product
+ * code) and V (MSE code) [E4][Z1 asymmetric K/V].
+ *   q: device fp32 [batch][n_q_heads][d].  K/V vector index =
+ *      (b*n_kv_heads + g)*max_tokens + t.  seq_lens: device int32 [batch],
+ *      0 <= seq_lens[b] <= max_tokens.
+ *   out[b][h] = sum_t softmax_t(scale*l_t) v_hat_t, v_hat = n_v D H c_v[idx_v] / sqrt(d_pad)
+ *      (first d coordinates); scale 0 means 1/sqrt(d).  Rows with
+ *      seq_lens[b] == 0 are zero.  out: device fp32 [batch][n_q_heads][d].
+ *   workspace: device, >= tq_decode_attn_workspace(...) bytes, 16-byte aligned.
+ * Supported: kp PROD kb <= 3 and vp MSE, same d/d_pad (128), n_q_heads a
+ * multiple of n_kv_heads.
+ */
+int64_t tq_decode_attn_workspace(const tq_params* kp, int batch, int n_q_heads, int n_kv_heads,
+                                 int64_t max_tokens);
+int tq_decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int batch,
+                   int n_q_heads, int n_kv_heads, const void* kcodes, const uint16_t* knorms,
+                   const uint16_t* krnorms, const void* vcodes, const uint16_t* vnorms,
+                   const int32_t* seq_lens, int64_t max_tokens, float scale, float* out,
+                   void* workspace, int64_t workspace_bytes, tq_stream_t stream);
+
+/*
+ * tq_search_topk - top-k inner-product search over quantized vectors [E5].
+ *   q: device fp32 [n_q][d]; codes/norms/rnorms: n_db vectors.
+ *   ids: device int32 [n_q][k], scores: device fp32 [n_q][k]: the k largest
+ *   logit estimates (as tq_logits with group 1) per query, in descending
+ *   order, ties to the lower id.  1 <= k <= 32.
+ *   workspace: device, >= tq_search_workspace(...) bytes, 16-byte aligned.
+ */
+int64_t tq_search_workspace(const tq_params* p, int n_q, int64_t n_db, int k);
+int tq_search_topk(const tq_params* p, const float* q, int n_q, const void* codes,
+                   const uint16_t* norms, const uint16_t* rnorms, int64_t n_db, int k,
+                   int32_t* ids, float* scores, void* workspace, int64_t workspace_bytes,
+                   tq_stream_t stream);
+
+/* Message for the last failed call on this thread ("" if none). */
+const char* tq_last_error(void);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int tq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TQ_H_ */

@@ -1,0 +1,122 @@
+"""CPU checks of the C ABI library: it loads, exports every function that
+include/tq.h declares, its host-side functions agree with the oracle, and
+argument validation rejects bad calls before anything reaches the GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import vector_quantization_randomized_b200 as tq
+from oracle.codebook import stored_codebook
+from oracle.params import sign_flips, qjl_matrix
+from oracle import codec
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tq.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 12
+    out = subprocess.check_output(["nm", "-D", "--defined-only", tq.LIB_PATH]).decode()
+    exported = set(re.findall(r" T (tq_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(tq.LIB_PATH)
+    for n in names:
+        assert getattr(lib, n) is not None
+
+
+def test_version():
+    assert tq.tq_version() >= 100
+
+
+@pytest.mark.parametrize("d_pad", [16, 128, 256])
+@pytest.mark.parametrize("kb", [1, 2, 3, 4])
+def test_codebook_matches_independent_oracle_solver(d_pad, kb):
+    c, t = tq.tq_make_codebook(d_pad, kb)
+    co, to = stored_codebook(d_pad, kb)
+    np.testing.assert_array_equal(c, co)
+    np.testing.assert_array_equal(t, to)
+
+
+@pytest.mark.parametrize("d_pad,m,seed", [(128, 128, 42), (256, 256, 7), (128, 64, 2 ** 40 + 3), (128, 0, 1)])
+def test_params_match_oracle_generator(d_pad, m, seed):
+    D, S = tq.tq_make_params(d_pad, m, seed)
+    np.testing.assert_array_equal(D, sign_flips(seed, d_pad))
+    if m:
+        np.testing.assert_array_equal(S.view(np.float16), qjl_matrix(seed, m, d_pad))
+
+
+def test_code_bytes():
+    for (d_pad, kb, m, n) in [(128, 3, 128, 1), (128, 2, 128, 4097), (256, 1, 256, 10 ** 6), (128, 3, 0, 33)]:
+        assert tq.tq_code_bytes(d_pad, kb, m, n) == codec.code_bytes(d_pad, kb, m, n)
+
+
+def _fake_params(**kw):
+    p = dict(d=128, d_pad=128, bits=4, mode=tq.TQ_MODE_PROD, m=128)
+    p.update(kw)
+    buf = np.zeros(64, np.float32)
+    ptr = buf.ctypes.data
+    st = tq.tq_params(p["d"], p["d_pad"], p["bits"], p["mode"], p["m"], 0, ptr, ptr, ptr, ptr)
+    return st, buf
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d_pad=64), tq.TQ_EUNSUPPORTED),
+    (dict(d=0), tq.TQ_EINVAL),
+    (dict(d=129), tq.TQ_EINVAL),
+    (dict(bits=5), tq.TQ_EINVAL),
+    (dict(bits=1), tq.TQ_EINVAL),
+    (dict(m=48), tq.TQ_EINVAL),
+    (dict(mode=7), tq.TQ_EINVAL),
+    (dict(mode=tq.TQ_MODE_MSE, m=128), tq.TQ_EINVAL),
+])
+def test_validation_rejects_bad_params(kw, code):
+    st, keep = _fake_params(**kw)
+    lib = tq._lib
+    rc = lib.tq_quantize(ctypes.byref(st), None, tq.TQ_BF16, 10, 128, None, None, None, None)
+    assert rc == code
+    assert tq.tq_last_error()
+
+
+def test_validation_rejects_null_and_misaligned():
+    st, keep = _fake_params()
+    lib = tq._lib
+    buf = np.zeros(1024, np.uint8)
+    base = buf.ctypes.data
+    base16 = (base + 15) // 16 * 16
+    # NULL input
+    assert lib.tq_quantize(ctypes.byref(st), None, tq.TQ_BF16, 10, 128, base16, base16, base16, None) == tq.TQ_EINVAL
+    # misaligned x
+    assert lib.tq_quantize(ctypes.byref(st), base16 + 2, tq.TQ_BF16, 10, 128, base16, base16, base16,
+                           None) == tq.TQ_EINVAL
+    # ld < d
+    assert lib.tq_quantize(ctypes.byref(st), base16, tq.TQ_BF16, 10, 64, base16, base16, base16, None) == tq.TQ_EINVAL
+    # bad dtype
+    assert lib.tq_quantize(ctypes.byref(st), base16, 9, 10, 128, base16, base16, base16, None) == tq.TQ_EINVAL
+    # n_vec == 0 is a no-op that touches nothing
+    assert lib.tq_quantize(ctypes.byref(st), None, tq.TQ_BF16, 0, 128, None, None, None, None) == tq.TQ_OK
+    # logits: n_q != heads*group
+    assert lib.tq_logits(ctypes.byref(st), base16, 5, 4, base16, base16, base16, 100, 1, base16, base16, 1 << 20,
+                         None) == tq.TQ_EINVAL
+    # logits: workspace too small
+    assert lib.tq_logits(ctypes.byref(st), base16, 4, 4, base16, base16, base16, 100, 1, base16, base16, 16,
+                         None) == tq.TQ_EINVAL
+    # logits: unsupported shape (d_pad 256 with 3 index bits)
+    st2, keep2 = _fake_params(d=200, d_pad=256, m=256)
+    assert lib.tq_logits(ctypes.byref(st2), base16, 4, 4, base16, base16, base16, 100, 1, base16, base16,
+                         1 << 20, None) == tq.TQ_EUNSUPPORTED
+    # decode: value params must be MSE mode
+    assert lib.tq_decode_attn(ctypes.byref(st), ctypes.byref(st), base16, 1, 4, 1, base16, base16, base16, base16,
+                              base16, base16, 64, 0.0, base16, base16, 1 << 20, None) == tq.TQ_EUNSUPPORTED
+    assert lib.tq_code_bytes(-1, 1, 1, 1) == -1

@@ -1,0 +1,184 @@
+"""Python binding of the TurboQuant codec library (libtq.so, C ABI in include/tq.h).
+
+Argument marshalling only: every step of quantization and estimation runs in
+the library's CUDA kernels.  PyTorch supplies device memory and streams.
+The functions keep the C names; tensors are passed by device pointer.
+
+If libtq.so is missing this module raises at import: there is no fallback.
+Build it with ``python -m vector_quantization_randomized_b200.build``.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECUDA = 0, -1, -2, -3
+TQ_MODE_PROD, TQ_MODE_MSE = 0, 1
+TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} not found: build it with `python -m vector_quantization_randomized_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+
+class tq_params(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("d_pad", ctypes.c_int32), ("bits", ctypes.c_int32),
+                ("mode", ctypes.c_int32), ("m", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("centroids", ctypes.c_void_p), ("thresholds", ctypes.c_void_p),
+                ("signs_D", ctypes.c_void_p), ("S", ctypes.c_void_p)]
+
+
+_P = ctypes.POINTER(tq_params)
+_vp, _i32, _i64, _u64, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_float
+_SIGS = {
+    "tq_make_codebook": (_i32, [_i32, _i32, _vp, _vp]),
+    "tq_make_params": (_i32, [_i32, _i32, _u64, _vp, _vp]),
+    "tq_code_bytes": (_i64, [_i32, _i32, _i32, _i64]),
+    "tq_quantize": (_i32, [_P, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "tq_logits_workspace": (_i64, [_P, _i32]),
+    "tq_logits": (_i32, [_P, _vp, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _i64, _vp]),
+    "tq_decode_attn_workspace": (_i64, [_P, _i32, _i32, _i32, _i64]),
+    "tq_decode_attn": (_i32, [_P, _P, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _f32, _vp,
+                              _vp, _i64, _vp]),
+    "tq_search_workspace": (_i64, [_P, _i32, _i64, _i32]),
+    "tq_search_topk": (_i32, [_P, _vp, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _vp, _i64, _vp]),
+    "tq_last_error": (ctypes.c_char_p, []),
+    "tq_version": (_i32, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class TQError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"{msg} (status {code})")
+        self.code = code
+
+
+def _check(rc):
+    if rc != TQ_OK:
+        raise TQError(rc, tq_last_error())
+    return rc
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def tq_last_error():
+    return _lib.tq_last_error().decode()
+
+
+def tq_version():
+    return _lib.tq_version()
+
+
+def tq_make_codebook(d_pad, kb):
+    """Host: Lloyd-Max codebook for the rotated-coordinate law -> (centroids, thresholds) fp32."""
+    c = np.zeros(1 << kb, np.float32)
+    t = np.zeros((1 << kb) - 1, np.float32)
+    _check(_lib.tq_make_codebook(d_pad, kb, c.ctypes.data, t.ctypes.data))
+    return c, t
+
+
+def tq_make_params(d_pad, m, seed):
+    """Host: sign flips D (int8) and QJL matrix S (fp16 bit patterns as uint16, m x d_pad)."""
+    D = np.zeros(d_pad, np.int8)
+    S = np.zeros((max(m, 1), d_pad), np.uint16)
+    _check(_lib.tq_make_params(d_pad, m, seed, D.ctypes.data, S.ctypes.data if m else None))
+    return D, (S if m else None)
+
+
+def tq_code_bytes(d_pad, kb, m, n_vec):
+    return _lib.tq_code_bytes(d_pad, kb, m, n_vec)
+
+
+class Params:
+    """A quantizer: host-made codebook/D/S copied to the device, plus the C struct."""
+
+    def __init__(self, d, bits, mode=TQ_MODE_PROD, m=None, seed=42, d_pad=None, device="cuda"):
+        import torch
+        d_pad = d_pad or (128 if d <= 128 else 256)
+        if mode == TQ_MODE_PROD and m is None:
+            m = d_pad
+        m = m if mode == TQ_MODE_PROD else 0
+        self.d, self.d_pad, self.bits, self.mode, self.m, self.seed = d, d_pad, bits, mode, m, seed
+        self.kb = bits - 1 if mode == TQ_MODE_PROD else bits
+        c, t = tq_make_codebook(d_pad, self.kb)
+        D, S = tq_make_params(d_pad, m, seed)
+        self.host = dict(centroids=c, thresholds=t, D=D, S=S)
+        self.centroids = torch.from_numpy(c).to(device)
+        self.thresholds = torch.from_numpy(t).to(device)
+        self.D = torch.from_numpy(D).to(device)
+        self.S = torch.from_numpy(S.view(np.int16)).to(device) if m else None
+        self.struct = tq_params(d, d_pad, bits, mode, m, 0, _ptr(self.centroids), _ptr(self.thresholds),
+                                _ptr(self.D), _ptr(self.S))
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+    def code_bytes(self, n_vec):
+        return tq_code_bytes(self.d_pad, self.kb, self.m, n_vec)
+
+
+def _dtype_code(x):
+    import torch
+    return {torch.float32: TQ_F32, torch.float16: TQ_F16, torch.bfloat16: TQ_BF16}[x.dtype]
+
+
+def tq_quantize(p, x, codes, norms, rnorms=None, n_vec=None, ld=None, stream=None):
+    """Encode rows of x (device tensor [n, ld] fp32/fp16/bf16) into codes/norms/rnorms."""
+    n_vec = x.shape[0] if n_vec is None else n_vec
+    ld = x.stride(0) if ld is None else ld
+    return _check(_lib.tq_quantize(p.ref, _ptr(x), _dtype_code(x), n_vec, ld, _ptr(codes), _ptr(norms),
+                                   _ptr(rnorms), _stream(stream)))
+
+
+def tq_logits_workspace(p, n_q):
+    return _lib.tq_logits_workspace(p.ref, n_q)
+
+
+def tq_logits(p, q, group, codes, norms, rnorms, n_keys, n_kv_heads, logits, workspace, stream=None):
+    return _check(_lib.tq_logits(p.ref, _ptr(q), q.shape[0], group, _ptr(codes), _ptr(norms), _ptr(rnorms),
+                                 n_keys, n_kv_heads, _ptr(logits), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)))
+
+
+def tq_decode_attn_workspace(kp, batch, n_q_heads, n_kv_heads, max_tokens):
+    return _lib.tq_decode_attn_workspace(kp.ref, batch, n_q_heads, n_kv_heads, max_tokens)
+
+
+def tq_decode_attn(kp, vp, q, n_kv_heads, kcodes, knorms, krnorms, vcodes, vnorms, seq_lens, max_tokens, out,
+                   workspace, scale=0.0, stream=None):
+    batch, n_q_heads = q.shape[0], q.shape[1]
+    return _check(_lib.tq_decode_attn(kp.ref, vp.ref, _ptr(q), batch, n_q_heads, n_kv_heads, _ptr(kcodes),
+                                      _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), _ptr(seq_lens),
+                                      max_tokens, scale, _ptr(out), _ptr(workspace), workspace.numel(),
+                                      _stream(stream)))
+
+
+def tq_search_workspace(p, n_q, n_db, k):
+    return _lib.tq_search_workspace(p.ref, n_q, n_db, k)
+
+
+def tq_search_topk(p, q, codes, norms, rnorms, n_db, k, ids, scores, workspace, stream=None):
+    return _check(_lib.tq_search_topk(p.ref, _ptr(q), q.shape[0], _ptr(codes), _ptr(norms), _ptr(rnorms), n_db,
+                                      k, _ptr(ids), _ptr(scores), _ptr(workspace), workspace.numel(),
+                                      _stream(stream)))

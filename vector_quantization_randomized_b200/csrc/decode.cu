@@ -1,0 +1,363 @@
+// tq_decode_attn: one decode step of attention over compressed K and V
+// ("TurboQuant explainer" (m.163.com), "速度": attention from the codes;
+// zhidx turboquant_plus article: asymmetric K/V - keys in the product code,
+// values MSE-only).
+//
+//   out[b][h] = sum_t softmax_t(scale * l_t) * v_hat_t,
+//   v_hat_t = n_v D H c_v[idx_t] / sqrt(d_pad).
+//
+// Split-K over tokens ("flash-decoding"): CTA (b, kv head, query chunk,
+// token chunk of 512) computes the logits of its 4 query heads with the
+// tensor-core code scan (scan.cuh), the chunk's softmax statistics, and the
+// value sum in the *rotated* domain, o_rot = sum_t p_t n_v,t c_v[idx_t]
+// (the rotation is linear, so it is applied once per output row instead of
+// once per token).  A combine kernel merges the chunks (log-sum-exp) and
+// applies the inverse rotation D H / sqrt(d_pad).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "common.h"
+#include "prep.h"
+#include "scan.cuh"
+
+namespace {
+using namespace tqd;
+
+constexpr int CH = 512;  // tokens per split-K chunk
+
+struct DArgs {
+  const uint8_t* kcodes;
+  const uint16_t* knorms;
+  const uint16_t* krnorms;
+  const uint8_t* vcodes;
+  const uint16_t* vnorms;
+  const int32_t* seq_lens;
+  const float* vcent;
+  int64_t max_tokens;
+  int hkv, group, nqc, nch, km, ktb, vtb, vkb, dp;
+  const uint8_t* prep;
+  int64_t prep_bytes;
+  float* part;  // [b][h][chunk][dp + 2]
+  float kappa, sl2;  // sqrt(pi/2)/m, scale*log2(e)
+};
+
+template <int KB, int SI, int VKB>
+__global__ void __launch_bounds__(128) decode_kernel(const DArgs a) {
+  constexpr int DP = 128;
+  using SC = Scan<DP, KB, SI>;
+  constexpr int SW = SI > 0 ? SI : 1;
+  __shared__ float sl[QCHUNK][CH];
+  __shared__ float4 wv[CH];
+  __shared__ float stat[QCHUNK][2];
+  __shared__ float vc[16];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int chunk_id = blockIdx.x % a.nch;
+  const int rest = blockIdx.x / a.nch;
+  const int qc = rest % a.nqc;
+  const int bg = rest / a.nqc;  // b * hkv + g
+  const int b = bg / a.hkv;
+  const int L = (int)min((int64_t)a.seq_lens[b], a.max_tokens);
+  const int t0 = chunk_id * CH;
+  const int ntok = max(0, min(CH, L - t0));
+  if (threadIdx.x < (1 << VKB)) vc[threadIdx.x] = a.vcent[threadIdx.x];
+  const int64_t vbase = (int64_t)bg * a.max_tokens;
+
+  // 1) logits of the chunk's tokens for the 4 query heads
+  if (ntok > 0) {
+    const uint8_t* prep = a.prep + (int64_t)(bg * a.nqc + qc) * a.prep_bytes;
+    SC sc;
+    sc.load(prep, lane);
+    const int g = lane >> 2, t = lane & 3;
+    const float4 qs = reinterpret_cast<const float4*>(prep + SC::FR * 128)[g & 3];
+    const int nsub = (ntok + 7) / 8;
+    for (int s = warp; s < nsub; s += 4) {
+      uint32_t bw[KB][1], sw[SW];
+      const int tk = 8 * s + g;
+      load_words<DP, KB, SI>(a.kcodes, a.ktb, a.km, vbase + t0 + tk, tk < ntok, t, bw, sw);
+      int accC[4] = {0, 0, 0, 0}, accS[4] = {0, 0, 0, 0};
+      sc.run(accC, accS, bw, sw);
+      double c0, c1, z0 = 0.0, z1 = 0.0;
+      combine_digits(accC, lane, c0, c1);
+      if constexpr (SI > 0) combine_digits(accS, lane, z0, z1);
+      if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int tok = 8 * s + 2 * t + e;
+          float val = -INFINITY;
+          if (tok < ntok) {
+            const int64_t v = vbase + t0 + tok;
+            const float n = __half2float(__ushort_as_half(a.knorms[v]));
+            float l = (float)((e ? c1 : c0) * (double)qs.x) - qs.y;
+            if constexpr (SI > 0) {
+              const float gm = __half2float(__ushort_as_half(a.krnorms[v]));
+              l = fmaf(gm * a.kappa, (float)((e ? z1 : z0) * (double)qs.z) - qs.w, l);
+            }
+            val = n * l * a.sl2;
+          }
+          sl[g][tok] = val;
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // 2) softmax statistics per query (warp q), weights p * n_v
+  if (ntok > 0) {
+    const int qq = warp;
+    float mx = -INFINITY;
+    for (int j = lane; j < ntok; j += 32) mx = fmaxf(mx, sl[qq][j]);
+    mx = warp_max(mx);
+    float sum = 0.f;
+    for (int j = lane; j < ntok; j += 32) {
+      const float p = exp2f(sl[qq][j] - mx);
+      sl[qq][j] = p;
+      sum += p;
+    }
+    sum = warp_sum(sum);
+    if (lane == 0) {
+      stat[qq][0] = mx;
+      stat[qq][1] = sum;
+    }
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < ntok; j += 128) {
+    const float nv = __half2float(__ushort_as_half(a.vnorms[vbase + t0 + j]));
+    wv[j] = make_float4(sl[0][j] * nv, sl[1][j] * nv, sl[2][j] * nv, sl[3][j] * nv);
+  }
+  __syncthreads();
+
+  // 3) value sum in the rotated domain: thread = coordinate c
+  const int c = threadIdx.x;  // DP == blockDim.x
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+  const int w = c >> 5, bit = c & 31;
+  for (int j = 0; j < ntok; ++j) {
+    const int64_t v = vbase + t0 + j;
+    const uint8_t* tbase = a.vcodes + (v >> 5) * a.vtb + (int)(v & 31) * (DP / 8);
+    int idx = 0;
+#pragma unroll
+    for (int p = 0; p < VKB; ++p) {
+      const uint32_t word = __ldg(reinterpret_cast<const uint32_t*>(tbase + p * TILE * (DP / 8)) + w);
+      idx |= ((word >> bit) & 1u) << p;
+    }
+    const float cv = vc[idx];
+    const float4 ww = wv[j];
+    acc0 = fmaf(ww.x, cv, acc0);
+    acc1 = fmaf(ww.y, cv, acc1);
+    acc2 = fmaf(ww.z, cv, acc2);
+    acc3 = fmaf(ww.w, cv, acc3);
+  }
+
+  // 4) partials: [b][h][chunk][dp + 2] = (o_rot[0..dp), max (log2 units), sum)
+  const int hq0 = (bg % a.hkv) * a.group + QCHUNK * qc;
+  const int nq = min(QCHUNK, a.group - QCHUNK * qc);
+  const float accs[4] = {acc0, acc1, acc2, acc3};
+#pragma unroll
+  for (int qq = 0; qq < QCHUNK; ++qq) {
+    if (qq < nq) {
+      const int64_t h = (int64_t)b * (a.hkv * a.group) + hq0 + qq;
+      float* dst = a.part + (h * a.nch + chunk_id) * (DP + 2);
+      dst[c] = accs[qq];
+      if (c == 0) {
+        dst[DP] = ntok > 0 ? stat[qq][0] : -INFINITY;
+        dst[DP + 1] = ntok > 0 ? stat[qq][1] : 0.f;
+      }
+    }
+  }
+}
+
+struct CArgs {
+  const float* part;
+  const int8_t* vD;
+  const int32_t* seq_lens;
+  float* out;
+  int nch, d, dp, hq;
+};
+
+__global__ void __launch_bounds__(128) combine_kernel(const CArgs a) {
+  __shared__ float o[256];
+  __shared__ float wts[1024];
+  __shared__ float tot;
+  const int64_t h = blockIdx.x;  // b * hq + head
+  const int b = (int)(h / a.hq);
+  const float* src = a.part + h * a.nch * (a.dp + 2);
+  // chunk weights 2^(m_k - M)
+  float mx = -INFINITY;
+  for (int k = threadIdx.x; k < a.nch; k += blockDim.x) mx = fmaxf(mx, src[(int64_t)k * (a.dp + 2) + a.dp]);
+  mx = warp_max(mx);
+  __shared__ float red[4];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  float lsum = 0.f;
+  for (int k = threadIdx.x; k < a.nch; k += blockDim.x) {
+    const float mk = src[(int64_t)k * (a.dp + 2) + a.dp];
+    const float wk = (mk == -INFINITY) ? 0.f : exp2f(mk - mx);
+    wts[k] = wk;
+    lsum += wk * src[(int64_t)k * (a.dp + 2) + a.dp + 1];
+  }
+  lsum = warp_sum(lsum);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = lsum;
+  __syncthreads();
+  if (threadIdx.x == 0) tot = red[0] + red[1] + red[2] + red[3];
+  __syncthreads();
+  const bool empty = (a.seq_lens[b] <= 0) || !(tot > 0.f);
+  for (int c = threadIdx.x; c < a.dp; c += blockDim.x) {
+    float s = 0.f;
+    for (int k = 0; k < a.nch; ++k) s = fmaf(wts[k], src[(int64_t)k * (a.dp + 2) + c], s);
+    o[c] = empty ? 0.f : s / tot;
+  }
+  __syncthreads();
+  // inverse rotation: x_hat = D o (H o_rot) / sqrt(dp)
+  const float rs = rsqrtf((float)a.dp);
+  for (int c = threadIdx.x; c < a.d; c += blockDim.x) {
+    float s = 0.f;
+    for (int j = 0; j < a.dp; ++j) s += (__popc(c & j) & 1) ? -o[j] : o[j];
+    a.out[h * a.d + c] = s * rs * (float)a.vD[c];
+  }
+}
+
+template <int KB, int SI, int VKB>
+int launch_decode(const DArgs& a, int blocks, cudaStream_t st) {
+  decode_kernel<KB, SI, VKB><<<blocks, 128, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_decode_attn: launch failed: %s", cudaGetErrorString(e));
+  return TQ_OK;
+}
+
+template <int KB, int SI>
+int dispatch_vkb(int vkb, const DArgs& a, int blocks, cudaStream_t st) {
+  switch (vkb) {
+    case 1: return launch_decode<KB, SI, 1>(a, blocks, st);
+    case 2: return launch_decode<KB, SI, 2>(a, blocks, st);
+    case 3: return launch_decode<KB, SI, 3>(a, blocks, st);
+    default: return launch_decode<KB, SI, 4>(a, blocks, st);
+  }
+}
+
+int64_t decode_ws_parts(int batch, int hq, int64_t max_tokens) {
+  const int64_t nch = (max_tokens + CH - 1) / CH;
+  return (int64_t)batch * hq * std::max<int64_t>(nch, 1) * (128 + 2) * 4;
+}
+
+}  // namespace
+
+extern "C" int64_t tq_decode_attn_workspace(const tq_params* kp, int batch, int n_q_heads, int n_kv_heads,
+                                            int64_t max_tokens) {
+  if (!kp || batch < 0 || n_q_heads < 1 || n_kv_heads < 1 || max_tokens < 0) return -1;
+  const int kb = kp->mode == TQ_MODE_PROD ? kp->bits - 1 : kp->bits;
+  if (kb < 1 || kb > 4) return -1;
+  const tqd::ScanShape sh(kp->d_pad, kb, kp->mode == TQ_MODE_PROD ? kp->m : 0);
+  const int group = n_q_heads / n_kv_heads;
+  const int nqc = (group + tqd::QCHUNK - 1) / tqd::QCHUNK;
+  int64_t prep = (int64_t)batch * n_kv_heads * nqc * tqd::prep_chunk_bytes(sh.fr);
+  prep = (prep + 255) & ~(int64_t)255;
+  return prep + decode_ws_parts(batch, n_q_heads, max_tokens);
+}
+
+extern "C" int tq_decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int batch, int n_q_heads,
+                              int n_kv_heads, const void* kcodes, const uint16_t* knorms, const uint16_t* krnorms,
+                              const void* vcodes, const uint16_t* vnorms, const int32_t* seq_lens,
+                              int64_t max_tokens, float scale, float* out, void* workspace,
+                              int64_t workspace_bytes, tq_stream_t stream) {
+  using namespace tq;
+  int rc = check_params(kp, "tq_decode_attn(kp)");
+  if (rc) return rc;
+  rc = check_params(vp, "tq_decode_attn(vp)");
+  if (rc) return rc;
+  if (kp->mode != TQ_MODE_PROD || vp->mode != TQ_MODE_MSE)
+    return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: needs product-code keys and MSE-code values");
+  if (kp->d_pad != 128 || vp->d_pad != 128 || kp->d != vp->d)
+    return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: keys and values need d_pad = 128 and equal d");
+  const int kkb = index_bits(kp), vkb = index_bits(vp);
+  if (kkb > 3) return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: key codes need <= 3 index bits");
+  if (batch < 0 || n_kv_heads < 1 || n_q_heads < 1 || (n_q_heads % n_kv_heads) != 0)
+    return set_error(TQ_EINVAL, "tq_decode_attn: n_q_heads must be a positive multiple of n_kv_heads");
+  if (max_tokens < 0 || max_tokens > (int64_t)1 << 31) return set_error(TQ_EINVAL, "tq_decode_attn: bad max_tokens");
+  if (batch == 0) {
+    clear_error();
+    return TQ_OK;
+  }
+  if (!q || !kcodes || !knorms || !krnorms || !vcodes || !vnorms || !seq_lens || !out || !workspace)
+    return set_error(TQ_EINVAL, "tq_decode_attn: NULL pointer argument");
+  if (!aligned(kcodes, 16) || !aligned(vcodes, 16) || !aligned(workspace, 16))
+    return set_error(TQ_EINVAL, "tq_decode_attn: codes and workspace must be 16-byte aligned");
+  const int64_t need = tq_decode_attn_workspace(kp, batch, n_q_heads, n_kv_heads, max_tokens);
+  if (workspace_bytes < need)
+    return set_error(TQ_EINVAL, "tq_decode_attn: workspace too small (%lld < %lld)", (long long)workspace_bytes,
+                     (long long)need);
+  const int group = n_q_heads / n_kv_heads;
+  const int nqc = (group + tqd::QCHUNK - 1) / tqd::QCHUNK;
+  const tqd::ScanShape sh(128, kkb, kp->m);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  tqd::PrepArgs pa;
+  pa.q = q;
+  pa.d = kp->d;
+  pa.dp = 128;
+  pa.kb = kkb;
+  pa.m = kp->m;
+  pa.n_outer = batch * n_kv_heads;
+  pa.group = group;
+  pa.nqc = nqc;
+  pa.cent = kp->centroids;
+  pa.D = kp->signs_D;
+  pa.S = kp->S;
+  pa.out = static_cast<uint8_t*>(workspace);
+  pa.fr = sh.fr;
+  rc = launch_prep(pa, st);
+  if (rc) return rc;
+  int64_t prep_total = (int64_t)batch * n_kv_heads * nqc * tqd::prep_chunk_bytes(sh.fr);
+  prep_total = (prep_total + 255) & ~(int64_t)255;
+  const int nch = (int)std::max<int64_t>(1, (max_tokens + CH - 1) / CH);
+  if (nch > 1024) return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: max_tokens above 524288 is not supported");
+  DArgs a;
+  a.kcodes = static_cast<const uint8_t*>(kcodes);
+  a.knorms = knorms;
+  a.krnorms = krnorms;
+  a.vcodes = static_cast<const uint8_t*>(vcodes);
+  a.vnorms = vnorms;
+  a.seq_lens = seq_lens;
+  a.vcent = vp->centroids;
+  a.max_tokens = max_tokens;
+  a.hkv = n_kv_heads;
+  a.group = group;
+  a.nqc = nqc;
+  a.nch = nch;
+  a.km = kp->m;
+  a.ktb = tqd::tile_bytes(128, kkb, kp->m);
+  a.vtb = tqd::tile_bytes(128, vkb, 0);
+  a.vkb = vkb;
+  a.dp = 128;
+  a.prep = pa.out;
+  a.prep_bytes = tqd::prep_chunk_bytes(sh.fr);
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + prep_total);
+  a.kappa = (float)(std::sqrt(M_PI / 2.0) / kp->m);
+  const float sc = scale != 0.f ? scale : (float)(1.0 / std::sqrt((double)kp->d));
+  a.sl2 = sc * 1.4426950408889634f;
+  const int64_t blocks64 = (int64_t)batch * n_kv_heads * nqc * nch;
+  if (blocks64 > 0x7fffffff) return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: grid too large");
+  const int blocks = (int)blocks64;
+  const int si = sh.nsi;
+  switch (kkb) {
+    case 1: rc = si == 2 ? dispatch_vkb<1, 2>(vkb, a, blocks, st) : dispatch_vkb<1, 1>(vkb, a, blocks, st); break;
+    case 2: rc = si == 2 ? dispatch_vkb<2, 2>(vkb, a, blocks, st) : dispatch_vkb<2, 1>(vkb, a, blocks, st); break;
+    default: rc = si == 2 ? dispatch_vkb<3, 2>(vkb, a, blocks, st) : dispatch_vkb<3, 1>(vkb, a, blocks, st); break;
+  }
+  if (rc) return rc;
+  CArgs ca;
+  ca.part = a.part;
+  ca.vD = vp->signs_D;
+  ca.seq_lens = seq_lens;
+  ca.out = out;
+  ca.nch = nch;
+  ca.d = kp->d;
+  ca.dp = 128;
+  ca.hq = n_q_heads;
+  combine_kernel<<<batch * n_q_heads, 128, 0, st>>>(ca);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(TQ_ECUDA, "tq_decode_attn: combine launch failed: %s", cudaGetErrorString(e));
+  clear_error();
+  return TQ_OK;
+}

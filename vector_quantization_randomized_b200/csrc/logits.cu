@@ -1,0 +1,212 @@
+// tq_logits: attention logits straight from the packed codes
+// ("TurboQuant explainer" (m.163.com), "第二步：QJL" estimator; "速度":
+// logits from 4-bit codes).
+//
+// One CTA (4 warps) scans a contiguous key range for one KV head and one
+// chunk of 4 query heads; each warp takes 8-key subtiles.  Per subtile a lane
+// loads its key's plane words with plain coalesced 32-bit loads (a warp reads
+// 8 keys x 16 B per plane = 128 contiguous bytes), the next subtile's words
+// are prefetched while the current one runs on the tensor cores (int8
+// mma.sync, exact integer sums, see scan.cuh), and lanes 0..15 write the
+// logits of their (query, key pair).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "common.h"
+#include "prep.h"
+#include "scan.cuh"
+
+namespace {
+using namespace tqd;
+
+struct LArgs {
+  const uint8_t* codes;
+  const uint16_t* norms;
+  const uint16_t* rnorms;
+  int64_t n_keys;
+  int group, nqc, nsplit, m, tb;
+  const uint8_t* prep;
+  int64_t prep_bytes;
+  float* logits;
+  float kappa;
+};
+
+template <int DP, int KB, int SI>
+__global__ void __launch_bounds__(128) logits_kernel(const LArgs a) {
+  using SC = Scan<DP, KB, SI>;
+  constexpr int NH = DP / 128;
+  constexpr int SW = SI > 0 ? SI : 1;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int chunk = blockIdx.x / a.nsplit, split = blockIdx.x % a.nsplit;
+  const int head = chunk / a.nqc, qc = chunk % a.nqc;
+  const uint8_t* prep = a.prep + (int64_t)chunk * a.prep_bytes;
+  SC sc;
+  sc.load(prep, lane);
+  const int g = lane >> 2, t = lane & 3;
+  const float4 qs = reinterpret_cast<const float4*>(prep + SC::FR * 128)[g & 3];
+  const int qrow = QCHUNK * qc + (g & 3);
+  const bool qvalid = (lane < 16) && (qrow < a.group);
+  const int64_t n_sub = (a.n_keys + 7) / 8;
+  const int64_t per = (n_sub + a.nsplit - 1) / a.nsplit;
+  const int64_t s_begin = (int64_t)split * per;
+  const int64_t s_end = min(n_sub, s_begin + per);
+  const int64_t vbase = (int64_t)head * a.n_keys;
+  float* out = a.logits + ((int64_t)head * a.group + qrow) * a.n_keys;
+
+  uint32_t bw[KB][NH], sw[SW];
+  int64_t s = s_begin + warp;
+  if (s < s_end) {
+    const int64_t kk = 8 * s + g;
+    load_words<DP, KB, SI>(a.codes, a.tb, a.m, vbase + kk, kk < a.n_keys, t, bw, sw);
+  }
+  for (; s < s_end; s += 4) {
+    uint32_t cbw[KB][NH], csw[SW];
+#pragma unroll
+    for (int p = 0; p < KB; ++p)
+#pragma unroll
+      for (int h = 0; h < NH; ++h) cbw[p][h] = bw[p][h];
+#pragma unroll
+    for (int i = 0; i < SW; ++i) csw[i] = sw[i];
+    const int64_t sn = s + 4;
+    if (sn < s_end) {
+      const int64_t kk = 8 * sn + g;
+      load_words<DP, KB, SI>(a.codes, a.tb, a.m, vbase + kk, kk < a.n_keys, t, bw, sw);
+    }
+    int accC[4] = {0, 0, 0, 0}, accS[4] = {0, 0, 0, 0};
+    sc.run(accC, accS, cbw, csw);
+    double c0, c1, z0 = 0.0, z1 = 0.0;
+    combine_digits(accC, lane, c0, c1);
+    if constexpr (SI > 0) combine_digits(accS, lane, z0, z1);
+    if (qvalid) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int64_t key = 8 * s + 2 * t + e;
+        if (key < a.n_keys) {
+          const int64_t v = vbase + key;
+          const float n = __half2float(__ushort_as_half(a.norms[v]));
+          float l = (float)((e ? c1 : c0) * (double)qs.x) - qs.y;
+          if constexpr (SI > 0) {
+            const float gm = __half2float(__ushort_as_half(a.rnorms[v]));
+            l = fmaf(gm * a.kappa, (float)((e ? z1 : z0) * (double)qs.z) - qs.w, l);
+          }
+          out[key] = n * l;
+        }
+      }
+    }
+  }
+}
+
+template <int DP, int KB, int SI>
+int launch_logits(const LArgs& a, int chunks, cudaStream_t st) {
+  logits_kernel<DP, KB, SI><<<chunks * a.nsplit, 128, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_logits: launch failed: %s", cudaGetErrorString(e));
+  return TQ_OK;
+}
+
+template <int DP, int KB>
+int dispatch_si(int si, const LArgs& a, int chunks, cudaStream_t st) {
+  switch (si) {
+    case 0: return launch_logits<DP, KB, 0>(a, chunks, st);
+    case 1: return launch_logits<DP, KB, 1>(a, chunks, st);
+    default: return launch_logits<DP, KB, 2>(a, chunks, st);
+  }
+}
+
+}  // namespace
+
+namespace tq {
+// Whether the register-fed scan supports this (d_pad, kb).
+bool scan_supported(int dp, int kb) { return (dp == 128 && kb >= 1 && kb <= 3) || (dp == 256 && kb >= 1 && kb <= 2); }
+}  // namespace tq
+
+extern "C" int64_t tq_logits_workspace(const tq_params* p, int n_q) {
+  if (!p || n_q < 0) return -1;
+  const int kb = p->mode == TQ_MODE_PROD ? p->bits - 1 : p->bits;
+  if (kb < 1 || kb > 4 || (p->d_pad != 128 && p->d_pad != 256)) return -1;
+  const tqd::ScanShape sh(p->d_pad, kb, p->mode == TQ_MODE_PROD ? p->m : 0);
+  return (int64_t)n_q * tqd::prep_chunk_bytes(sh.fr);
+}
+
+extern "C" int tq_logits(const tq_params* p, const float* q, int n_q, int group, const void* codes,
+                         const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys, int n_kv_heads,
+                         float* logits, void* workspace, int64_t workspace_bytes, tq_stream_t stream) {
+  using namespace tq;
+  int rc = check_params(p, "tq_logits");
+  if (rc) return rc;
+  const int kb = index_bits(p);
+  const bool prod = p->mode == TQ_MODE_PROD;
+  if (!scan_supported(p->d_pad, kb))
+    return set_error(TQ_EUNSUPPORTED, "tq_logits: d_pad=%d with %d index bits is not supported", p->d_pad, kb);
+  if (group < 1 || n_kv_heads < 1 || (int64_t)n_kv_heads * group != n_q)
+    return set_error(TQ_EINVAL, "tq_logits: need n_q == n_kv_heads * group (n_q=%d, heads=%d, group=%d)", n_q,
+                     n_kv_heads, group);
+  if (n_keys < 0) return set_error(TQ_EINVAL, "tq_logits: n_keys < 0");
+  if (n_keys == 0) {
+    clear_error();
+    return TQ_OK;
+  }
+  if (!q || !codes || !norms || !logits || !workspace || (prod && !rnorms))
+    return set_error(TQ_EINVAL, "tq_logits: NULL pointer argument");
+  if (!aligned(codes, 16) || !aligned(workspace, 16) || !aligned(q, 4) || !aligned(logits, 4))
+    return set_error(TQ_EINVAL, "tq_logits: misaligned pointer (codes/workspace need 16 bytes)");
+  const int m = prod ? p->m : 0;
+  const tqd::ScanShape sh(p->d_pad, kb, m);
+  const int nqc = (group + tqd::QCHUNK - 1) / tqd::QCHUNK;
+  const int chunks = n_kv_heads * nqc;
+  const int64_t need = (int64_t)chunks * tqd::prep_chunk_bytes(sh.fr);
+  if (workspace_bytes < need)
+    return set_error(TQ_EINVAL, "tq_logits: workspace too small (%lld < %lld bytes)", (long long)workspace_bytes,
+                     (long long)need);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  tqd::PrepArgs pa;
+  pa.q = q;
+  pa.d = p->d;
+  pa.dp = p->d_pad;
+  pa.kb = kb;
+  pa.m = m;
+  pa.n_outer = n_kv_heads;
+  pa.group = group;
+  pa.nqc = nqc;
+  pa.cent = p->centroids;
+  pa.D = p->signs_D;
+  pa.S = p->S;
+  pa.out = static_cast<uint8_t*>(workspace);
+  pa.fr = sh.fr;
+  rc = launch_prep(pa, st);
+  if (rc) return rc;
+
+  LArgs a;
+  a.codes = static_cast<const uint8_t*>(codes);
+  a.norms = norms;
+  a.rnorms = rnorms;
+  a.n_keys = n_keys;
+  a.group = group;
+  a.nqc = nqc;
+  a.m = m;
+  a.tb = tqd::tile_bytes(p->d_pad, kb, m);
+  a.prep = pa.out;
+  a.prep_bytes = tqd::prep_chunk_bytes(sh.fr);
+  a.logits = logits;
+  a.kappa = (float)(std::sqrt(M_PI / 2.0) / (m > 0 ? m : 1));
+  const int64_t n_sub = (n_keys + 7) / 8;
+  const int64_t target = (int64_t)sm_count() * 8;
+  a.nsplit = (int)std::max<int64_t>(1, std::min<int64_t>((target + chunks - 1) / chunks, (n_sub + 3) / 4));
+  const int si = sh.nsi;
+  if (p->d_pad == 128) {
+    switch (kb) {
+      case 1: rc = dispatch_si<128, 1>(si, a, chunks, st); break;
+      case 2: rc = dispatch_si<128, 2>(si, a, chunks, st); break;
+      default: rc = dispatch_si<128, 3>(si, a, chunks, st); break;
+    }
+  } else {
+    switch (kb) {
+      case 1: rc = dispatch_si<256, 1>(si, a, chunks, st); break;
+      default: rc = dispatch_si<256, 2>(si, a, chunks, st); break;
+    }
+  }
+  if (rc == TQ_OK) clear_error();
+  return rc;
+}
