@@ -1,0 +1,491 @@
+#!/usr/bin/env python
+"""Benchmark of the TurboQuant codec on B200.
+
+Default workload: one Llama-3.1-8B-shaped attention layer - 8 KV heads x
+32768 tokens, d = 128, 32 query heads (GQA 4), bf16 K/V from the synthetic
+law (per-channel lognormal(0, 0.5) scales, 4 outlier channels x20, per-token
+lognormal(0, 0.3) norms).  One step = the whole hot path at b = 3 and b = 4:
+    tq_quantize(K, product code), tq_quantize(V, MSE code),
+    tq_logits(32 decode queries over the 262144 compressed keys).
+Metric: compressed-key logits, keys/s (keys scored per second over the whole
+step, both bit widths), with per-kernel HBM GB/s and fractions of 8 TB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload layer|decode|quantize|search]
+
+N > 1 runs under torchrun, one rank per GPU, each rank a full independent
+layer (weak scaling, no collective on the data path).  Rank 0 prints one JSON
+line.  --impl reference times the CPU oracle (fp64 numpy) on a bounded
+sample of the same workload on the host cores.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HBM_NOMINAL_GBS = 8000.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="layer", choices=["layer", "decode", "quantize", "search"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-kernels", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = str(gpu_index)
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(gpu_index).uuid)
+            self.idx = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            pass
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), hw=parts[5], hwt=parts[6],
+                                 swt=parts[7], swp=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                            ("swp", "sw_power_cap")):
+                if r[k].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def allmax(world, v):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- workloads
+class Layer:
+    """One attention layer: 8 KV heads x 32768 tokens, 32 query heads, b = 3 and 4."""
+    H_KV, T, D, GROUP = 8, 32768, 128, 4
+    BITS = (3, 4)
+
+    def __init__(self, tq, wl, torch):
+        self.tq, self.torch = tq, torch
+        n = self.H_KV * self.T
+        self.n = n
+        K = wl.kv_block(1, self.H_KV, self.T, self.D, seed=wl.SEED_KEYS).reshape(n, self.D)
+        V = wl.kv_block(1, self.H_KV, self.T, self.D, seed=wl.SEED_VALUES).reshape(n, self.D)
+        q = wl.queries(self.H_KV * self.GROUP, self.D, seed=wl.SEED_QUERIES)
+        self.K = torch.from_numpy(K).to(torch.bfloat16).cuda()
+        self.V = torch.from_numpy(V).to(torch.bfloat16).cuda()
+        self.q = torch.from_numpy(q).cuda()
+        self.kp, self.vp, self.bufs = {}, {}, {}
+        for b in self.BITS:
+            kp = tq.Params(self.D, b, tq.TQ_MODE_PROD, 128, wl.SEED_PARAMS)
+            vp = tq.Params(self.D, b, tq.TQ_MODE_MSE, 0, wl.SEED_PARAMS + 1)
+            self.kp[b], self.vp[b] = kp, vp
+            dev = "cuda"
+            self.bufs[b] = dict(
+                kc=torch.empty(kp.code_bytes(n), dtype=torch.uint8, device=dev),
+                kn=torch.empty(n, dtype=torch.int16, device=dev),
+                krn=torch.empty(n, dtype=torch.int16, device=dev),
+                vc=torch.empty(vp.code_bytes(n), dtype=torch.uint8, device=dev),
+                vn=torch.empty(n, dtype=torch.int16, device=dev),
+                lg=torch.empty((self.q.shape[0], self.T), dtype=torch.float32, device=dev),
+                ws=torch.empty(tq.tq_logits_workspace(kp, self.q.shape[0]), dtype=torch.uint8, device=dev))
+        self.launches_per_step = len(self.BITS) * 4   # quantize K, quantize V, logits prep + scan
+
+    def calls(self):
+        """The step as a list of (label, callable)."""
+        tq = self.tq
+        out = []
+        for b in self.BITS:
+            B = self.bufs[b]
+            kp, vp = self.kp[b], self.vp[b]
+            out.append((f"tq_quantize_K_b{b}", lambda kp=kp, B=B: tq.tq_quantize(kp, self.K, B["kc"], B["kn"], B["krn"])))
+            out.append((f"tq_quantize_V_b{b}", lambda vp=vp, B=B: tq.tq_quantize(vp, self.V, B["vc"], B["vn"])))
+            out.append((f"tq_logits_b{b}", lambda kp=kp, B=B: tq.tq_logits(kp, self.q, self.GROUP, B["kc"], B["kn"],
+                                                                           B["krn"], self.T, self.H_KV, B["lg"],
+                                                                           B["ws"])))
+        return out
+
+    def keys_per_step(self):
+        return len(self.BITS) * self.n
+
+    def bytes_of(self, label):
+        """Algorithmic bytes one call must move (inputs read + outputs written)."""
+        b = int(label[-1])
+        n, d = self.n, self.D
+        kc = self.kp[b].code_bytes(n)
+        if label.startswith("tq_quantize_K"):
+            return n * d * 2 + kc + 4 * n
+        if label.startswith("tq_quantize_V"):
+            return n * d * 2 + self.vp[b].code_bytes(n) + 2 * n
+        nq = self.q.shape[0]
+        return kc + 4 * n + nq * d * 4 + nq * self.T * 4
+
+    def metric_bytes(self, b):
+        """Bytes the logits metric counts: packed codes + norms + residual norms + queries."""
+        return self.kp[b].code_bytes(self.n) + 4 * self.n + self.q.numel() * 4
+
+    def host_inputs(self):
+        return [self.K, self.V, self.q]
+
+    def host_outputs(self):
+        return [self.bufs[b]["lg"] for b in self.BITS]
+
+
+# --------------------------------------------------------------------------- timing helpers
+def l2_flush(torch, buf):
+    buf.zero_()
+
+
+def time_steps(torch, wk, steps, warmup, world, flush):
+    """Device-timed steps: per-step and per-call CUDA events on the launching stream."""
+    calls = wk.calls()
+    for _ in range(warmup):
+        for _, f in calls:
+            f()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
+    for s in range(steps):
+        l2_flush(torch, flush)
+        ev[s][0].record()
+        for i, (_, f) in enumerate(calls):
+            f()
+            ev[s][i + 1].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    step_ms = [ev[s][0].elapsed_time(ev[s][-1]) for s in range(steps)]
+    per_call = {}
+    for i, (label, _) in enumerate(calls):
+        per_call[label] = [ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)]
+    return step_ms, per_call
+
+
+def time_e2e(torch, wk, steps, warmup):
+    """Same step through the public API with pinned host buffers: H2D inputs, step, D2H results."""
+    hin = [t.cpu().pin_memory() for t in wk.host_inputs()]
+    hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in wk.host_outputs()]
+    din, dout = wk.host_inputs(), wk.host_outputs()
+    calls = wk.calls()
+
+    def one():
+        for h, d in zip(hin, din):
+            d.copy_(h, non_blocking=True)
+        for _, f in calls:
+            f()
+        for h, d in zip(hout, dout):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    h2d = sum(t.numel() * t.element_size() for t in hin)
+    d2h = sum(t.numel() * t.element_size() for t in hout)
+    return ms, h2d, d2h
+
+
+def logits_isolated(torch, tq, wk, reps_min=8):
+    """tq_logits alone on L2-cold inputs: rotate over copies of the codes totalling > 4x L2,
+    launches captured in a CUDA graph; returns {bits: (us per call, metric bytes)}."""
+    res = {}
+    for b in wk.BITS:
+        B = wk.bufs[b]
+        per_copy = B["kc"].numel() + 2 * B["kn"].numel() * 2
+        ncopy = max(reps_min, int(4 * L2_BYTES // per_copy) + 1)
+        copies = [(B["kc"].clone(), B["kn"].clone(), B["krn"].clone()) for _ in range(ncopy)]
+        kp = wk.kp[b]
+
+        def run_all():
+            for kc, kn, krn in copies:
+                tq.tq_logits(kp, wk.q, wk.GROUP, kc, kn, krn, wk.T, wk.H_KV, B["lg"], B["ws"])
+
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            run_all()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                run_all()
+        torch.cuda.current_stream().wait_stream(s)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1000.0 / (reps * ncopy)
+        # single-call latency (stream launch, L2-cold copy)
+        e0.record()
+        tq.tq_logits(kp, wk.q, wk.GROUP, copies[0][0], copies[0][1], copies[0][2], wk.T, wk.H_KV, B["lg"], B["ws"])
+        e1.record()
+        torch.cuda.synchronize()
+        lat = e0.elapsed_time(e1) * 1000.0
+        res[b] = (us, wk.metric_bytes(b), lat)
+        del copies, g
+        torch.cuda.empty_cache()
+    return res
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def cpu_oracle_layer(sample_tokens=16384):
+    """The oracle (fp64 numpy, as it stands) on a bounded sample of the layer workload:
+    all 8 heads x `sample_tokens` tokens, b = 3 and 4, quantize K and V + logits."""
+    from vector_quantization_randomized_b200 import workloads as wl
+    from oracle import codec, estimate
+    from oracle.codebook import stored_codebook
+    from oracle.params import sign_flips, qjl_matrix
+    H, T, d, group = Layer.H_KV, sample_tokens, Layer.D, Layer.GROUP
+    K = wl.kv_block(1, H, T, d, seed=wl.SEED_KEYS).reshape(-1, d)
+    V = wl.kv_block(1, H, T, d, seed=wl.SEED_VALUES).reshape(-1, d)
+    q = wl.queries(H * group, d, seed=wl.SEED_QUERIES)
+    t0 = time.perf_counter()
+    for b in Layer.BITS:
+        c, t = stored_codebook(128, b - 1)
+        cv, tv = stored_codebook(128, b)
+        Dk, S = sign_flips(wl.SEED_PARAMS, 128), qjl_matrix(wl.SEED_PARAMS, 128, 128)
+        Dv = sign_flips(wl.SEED_PARAMS + 1, 128)
+        ke = codec.encode(K, Dk, c, t, S)
+        kbuf = codec.pack(ke["idx"], ke["signs"], b - 1, 128)
+        ve = codec.encode(V, Dv, cv, tv)
+        codec.pack(ve["idx"], None, b, 0)
+        idx, sg = codec.unpack(kbuf, K.shape[0], 128, b - 1, 128)
+        estimate.logits_gqa(q, Dk, S, idx, sg, ke["norm_f16"], ke["rnorm_f16"], c, 128, H, group, T)
+    dt = time.perf_counter() - t0
+    keys = len(Layer.BITS) * H * T
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    return keys / dt, cores, dt, f"8 heads x {T} tokens (of 32768), b=3 and b=4: quantize K and V + logits"
+
+
+# --------------------------------------------------------------------------- traffic record
+def traffic_record(kernel_file_label):
+    """ncu-derived DRAM bytes per launch from profiles/traffic.json, or None if the
+    kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(kernel_file_label)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "vector_quantization_randomized_b200", "csrc", rec["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["bytes_per_launch"] if h == rec["source_sha"] else None
+
+
+# --------------------------------------------------------------------------- secondary workloads
+def run_secondary(args, world, rank, local, torch, tq, wl):
+    raise SystemExit(f"workload {args.workload}: not available yet")
+
+
+# --------------------------------------------------------------------------- main
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    vals = []
+    for _ in range(args.warmup):
+        cpu_oracle_layer(sample_tokens=2048)
+    for _ in range(max(1, args.steps)):
+        v, cores, dt, sample = cpu_oracle_layer(sample_tokens=2048)
+        vals.append(v)
+    v = statistics.median(vals)
+    line = {"impl": "reference", "metric": "compressed-key logits keys/s (whole step, b=3 and b=4)",
+            "value": v, "unit": "keys/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "llama3.1-8b-layer-kv8x32768-gqa4-d128", "kv_heads": 8, "tokens": 32768,
+                       "q_heads": 32, "d": 128, "bits": [3, 4]},
+            "cpu_baseline": {"value": v, "unit": "keys/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    world, rank, local = dist_setup(args)
+    import vector_quantization_randomized_b200 as tq
+    from vector_quantization_randomized_b200 import workloads as wl
+    if args.workload != "layer":
+        return run_secondary(args, world, rank, local, torch, tq, wl)
+    peak, peak_kind = measured_peaks()
+    wk = Layer(tq, wl, torch)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    sampler = ClockSampler(local)
+    sampler.start()
+    step_ms, per_call = time_steps(torch, wk, args.steps, args.warmup, world, flush)
+    clocks = sampler.stop()
+    ms = statistics.mean(step_ms)
+    ms_max = allmax(world, sum(step_ms)) / args.steps
+    value = world * wk.keys_per_step() / (ms_max / 1e3)
+
+    # dominant API call in the step and its roofline
+    kinds = {}
+    for label, times in per_call.items():
+        kind = label.rsplit("_b", 1)[0]
+        k = kinds.setdefault(kind, [0.0, 0.0, 0])
+        k[0] += sum(times)
+        k[1] += wk.bytes_of(label) * len(times)
+        k[2] += len(times)
+    dom = max(kinds, key=lambda k: kinds[k][0])
+    t_ms, byts, nl = kinds[dom]
+    achieved = byts / (t_ms / 1e3) / 1e9
+    traffic = traffic_record(dom)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": dom,
+                "peak_kind": f"{peak_kind} (copy bandwidth)", "algorithmic_bytes_per_launch": int(byts / nl)}
+
+    kernels = {}
+    for label, times in per_call.items():
+        avg = statistics.mean(times)
+        gbs = wk.bytes_of(label) / (avg / 1e3) / 1e9
+        kernels[label] = {"us": round(avg * 1000, 2), "gbs": round(gbs, 1), "frac_measured": round(gbs / peak, 4)}
+    if not args.no_kernels:
+        iso = logits_isolated(torch, tq, wk)
+        for b, (us, mb, lat) in iso.items():
+            gbs = mb / (us / 1e6) / 1e9
+            kernels[f"tq_logits_b{b}_l2cold"] = {
+                "us": round(us, 2), "keys_per_s": round(wk.n / (us / 1e6)), "gbs": round(gbs, 1),
+                "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4), "frac_measured": round(gbs / peak, 4),
+                "single_launch_us": round(lat, 2)}
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = time_e2e(torch, wk, max(3, args.steps // 2), 2)
+        e_ms = allmax(world, e_ms)
+        e2e = {"value": world * wk.keys_per_step() / (e_ms / 1e3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v, cores, dt, sample = cpu_oracle_layer()
+        cpu = {"value": v, "unit": "keys/s", "cores": cores, "kind": "oracle", "sample": sample,
+               "seconds": round(dt, 2)}
+    if rank == 0:
+        line = {"metric": "compressed-key logits keys/s (whole step, b=3 and b=4)", "value": value, "unit": "keys/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32+s8",
+                "data": "synthetic",
+                "config": {"workload": "llama3.1-8b-layer-kv8x32768-gqa4-d128", "kv_heads": 8, "tokens": 32768,
+                           "q_heads": 32, "d": 128, "bits": [3, 4], "kv_dtype": "bf16",
+                           "l2": "flushed between steps (256 MB write)", "parallelism": f"replicas x{world}"},
+                "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": wk.launches_per_step * args.steps, "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

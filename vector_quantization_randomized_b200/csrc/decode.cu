@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const DArgs a) {
   __shared__ float4 wv[CH];
   __shared__ float stat[QCHUNK][2];
   __shared__ float vc[16];
+  __shared__ uint4 afrag[SC::FR / 4 * 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int chunk_id = blockIdx.x % a.nch;
   const int rest = blockIdx.x / a.nch;
@@ -65,10 +66,13 @@ __global__ void __launch_bounds__(128) decode_kernel(const DArgs a) {
   const int64_t vbase = (int64_t)bg * a.max_tokens;
 
   // 1) logits of the chunk's tokens for the 4 query heads
+  grid_dependency_wait();  // query prep (previous grid) complete
+  const uint8_t* prep = a.prep + (int64_t)(bg * a.nqc + qc) * a.prep_bytes;
+  if (ntok > 0) SC::stage(afrag, prep);
+  __syncthreads();
   if (ntok > 0) {
-    const uint8_t* prep = a.prep + (int64_t)(bg * a.nqc + qc) * a.prep_bytes;
     SC sc;
-    sc.load(prep, lane);
+    sc.load(reinterpret_cast<const uint8_t*>(afrag), lane);
     const int g = lane >> 2, t = lane & 3;
     const float4 qs = reinterpret_cast<const float4*>(prep + SC::FR * 128)[g & 3];
     const int nsub = (ntok + 7) / 8;
@@ -221,8 +225,16 @@ __global__ void __launch_bounds__(128) combine_kernel(const CArgs a) {
 
 template <int KB, int SI, int VKB>
 int launch_decode(const DArgs& a, int blocks, cudaStream_t st) {
-  decode_kernel<KB, SI, VKB><<<blocks, 128, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(128);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<KB, SI, VKB>, a);
   if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_decode_attn: launch failed: %s", cudaGetErrorString(e));
   return TQ_OK;
 }

@@ -38,14 +38,11 @@ __global__ void __launch_bounds__(128) logits_kernel(const LArgs a) {
   using SC = Scan<DP, KB, SI>;
   constexpr int NH = DP / 128;
   constexpr int SW = SI > 0 ? SI : 1;
+  __shared__ uint4 afrag[SC::FR / 4 * 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int chunk = blockIdx.x / a.nsplit, split = blockIdx.x % a.nsplit;
   const int head = chunk / a.nqc, qc = chunk % a.nqc;
-  const uint8_t* prep = a.prep + (int64_t)chunk * a.prep_bytes;
-  SC sc;
-  sc.load(prep, lane);
   const int g = lane >> 2, t = lane & 3;
-  const float4 qs = reinterpret_cast<const float4*>(prep + SC::FR * 128)[g & 3];
   const int qrow = QCHUNK * qc + (g & 3);
   const bool qvalid = (lane < 16) && (qrow < a.group);
   const int64_t n_sub = (a.n_keys + 7) / 8;
@@ -55,12 +52,21 @@ __global__ void __launch_bounds__(128) logits_kernel(const LArgs a) {
   const int64_t vbase = (int64_t)head * a.n_keys;
   float* out = a.logits + ((int64_t)head * a.group + qrow) * a.n_keys;
 
+  // first code words do not depend on the query prep: fetch them before waiting for it
   uint32_t bw[KB][NH], sw[SW];
   int64_t s = s_begin + warp;
   if (s < s_end) {
     const int64_t kk = 8 * s + g;
     load_words<DP, KB, SI>(a.codes, a.tb, a.m, vbase + kk, kk < a.n_keys, t, bw, sw);
   }
+  grid_dependency_wait();
+  const uint8_t* prep = a.prep + (int64_t)chunk * a.prep_bytes;
+  SC::stage(afrag, prep);
+  const float4 qs = reinterpret_cast<const float4*>(prep + SC::FR * 128)[g & 3];
+  __syncthreads();
+  SC sc;
+  sc.load(reinterpret_cast<const uint8_t*>(afrag), lane);
+
   for (; s < s_end; s += 4) {
     uint32_t cbw[KB][NH], csw[SW];
 #pragma unroll
@@ -100,8 +106,17 @@ __global__ void __launch_bounds__(128) logits_kernel(const LArgs a) {
 
 template <int DP, int KB, int SI>
 int launch_logits(const LArgs& a, int chunks, cudaStream_t st) {
-  logits_kernel<DP, KB, SI><<<chunks * a.nsplit, 128, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(chunks * a.nsplit);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, logits_kernel<DP, KB, SI>, a);
   if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_logits: launch failed: %s", cudaGetErrorString(e));
   return TQ_OK;
 }
@@ -191,9 +206,10 @@ extern "C" int tq_logits(const tq_params* p, const float* q, int n_q, int group,
   a.prep_bytes = tqd::prep_chunk_bytes(sh.fr);
   a.logits = logits;
   a.kappa = (float)(std::sqrt(M_PI / 2.0) / (m > 0 ? m : 1));
+  // about four 128-thread CTAs per SM, each with at least 16 subtiles per warp
   const int64_t n_sub = (n_keys + 7) / 8;
-  const int64_t target = (int64_t)sm_count() * 8;
-  a.nsplit = (int)std::max<int64_t>(1, std::min<int64_t>((target + chunks - 1) / chunks, (n_sub + 3) / 4));
+  const int64_t target = (int64_t)sm_count() * 4;
+  a.nsplit = (int)std::max<int64_t>(1, std::min<int64_t>((target + chunks - 1) / chunks, (n_sub + 63) / 64));
   const int si = sh.nsi;
   if (p->d_pad == 128) {
     switch (kb) {

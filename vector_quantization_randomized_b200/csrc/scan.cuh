@@ -87,16 +87,23 @@ struct Scan {
 
   uint32_t A[FR];
 
+  // A fragments of a chunk: fr/4 x 32 uint4, lane-interleaved (global or shared memory)
   __device__ __forceinline__ void load(const uint8_t* chunk, int lane) {
     const uint4* f = reinterpret_cast<const uint4*>(chunk);
 #pragma unroll
     for (int k = 0; k < FR / 4; ++k) {
-      uint4 v = __ldg(f + k * 32 + lane);
+      uint4 v = f[k * 32 + lane];
       A[4 * k] = v.x;
       A[4 * k + 1] = v.y;
       A[4 * k + 2] = v.z;
       A[4 * k + 3] = v.w;
     }
+  }
+
+  // Stage a chunk's fragments in shared memory (whole CTA), then every warp loads from there.
+  __device__ __forceinline__ static void stage(uint4* smem, const uint8_t* chunk) {
+    const uint4* f = reinterpret_cast<const uint4*>(chunk);
+    for (int k = threadIdx.x; k < FR / 4 * 32; k += blockDim.x) smem[k] = __ldg(f + k);
   }
 
   // bw[p][h]: word (t + 4h) of bit-plane p of this lane's key; sw[i]: sign word (t + 4i)
@@ -127,6 +134,10 @@ struct Scan {
     }
   }
 };
+
+// Programmatic dependent launch: wait until the preceding grid (query prep)
+// has completed and its writes are visible.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 
 // Combine the digit rows of an accumulator: thread (g, t) holds rows g, g+8
 // (digits g>>2 and 2+(g>>2) of query g&3) for keys 2t, 2t+1.  Returns, in
