@@ -380,8 +380,95 @@ def traffic_record(kernel_file_label):
 
 
 # --------------------------------------------------------------------------- secondary workloads
+def gpu_kv(torch, n_seq, n_heads, n_tokens, d, seed):
+    """Keys/values with the synthetic law, drawn on the GPU (bf16 [n_seq*n_heads*n_tokens, d]).
+    Same law as workloads.head_vectors; used where host generation of GBs would dominate."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    out = torch.empty((n_seq * n_heads, n_tokens, d), dtype=torch.bfloat16, device="cuda")
+    for i in range(n_seq * n_heads):
+        sigma = torch.exp(0.5 * torch.randn(d, generator=g, device="cuda"))
+        outl = torch.randperm(d, generator=g, device="cuda")[:4]
+        sigma[outl] *= 20.0
+        rho = torch.exp(0.3 * torch.randn(n_tokens, generator=g, device="cuda"))
+        z = torch.randn((n_tokens, d), generator=g, device="cuda")
+        out[i] = (z * sigma[None, :] * rho[:, None]).to(torch.bfloat16)
+    return out.reshape(-1, d)
+
+
 def run_secondary(args, world, rank, local, torch, tq, wl):
-    raise SystemExit(f"workload {args.workload}: not available yet")
+    """Other workloads (their own JSON line): 'decode' = 64 sequences x 8 KV heads x 16384 tokens
+    (K product b=3, V MSE b=3, 32 query heads); 'quantize' = 2^20 bf16 vectors at b=2,3,4."""
+    peak, peak_kind = measured_peaks()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    if args.workload == "decode":
+        B, Hkv, T, d, Hq = 64, 8, 16384, 128, 32
+        kp = tq.Params(d, 3, tq.TQ_MODE_PROD, 128, wl.SEED_PARAMS)
+        vp = tq.Params(d, 3, tq.TQ_MODE_MSE, 0, wl.SEED_PARAMS + 1)
+        n = B * Hkv * T
+        bufs = {}
+        for name, p, seed in (("k", kp, wl.SEED_KEYS), ("v", vp, wl.SEED_VALUES)):
+            x = gpu_kv(torch, B, Hkv, T, d, seed)
+            c = torch.empty(p.code_bytes(n), dtype=torch.uint8, device="cuda")
+            nn = torch.empty(n, dtype=torch.int16, device="cuda")
+            rn = torch.empty(n, dtype=torch.int16, device="cuda") if p.mode == tq.TQ_MODE_PROD else None
+            tq.tq_quantize(p, x, c, nn, rn)
+            torch.cuda.synchronize()
+            del x
+            bufs[name] = (c, nn, rn)
+        q = torch.randn((B, Hq, d), device="cuda")
+        out = torch.empty((B, Hq, d), device="cuda")
+        ws = torch.empty(tq.tq_decode_attn_workspace(kp, B, Hq, Hkv, T), dtype=torch.uint8, device="cuda")
+        sl = torch.full((B,), T, dtype=torch.int32, device="cuda")
+        run = lambda: tq.tq_decode_attn(kp, vp, q, Hkv, bufs["k"][0], bufs["k"][1], bufs["k"][2], bufs["v"][0],
+                                        bufs["v"][1], sl, T, out, ws)
+        for _ in range(args.warmup):
+            run()
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record()
+        for _ in range(args.steps):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        mbytes = bufs["k"][0].numel() + 4 * n + bufs["v"][0].numel() + 2 * n + q.numel() * 4
+        gbs = mbytes / (ms / 1e3) / 1e9
+        line = {"metric": "decode attention tokens/s", "value": n / (ms / 1e3), "unit": "tokens/s",
+                "ms_per_step": ms, "config": {"workload": "decode-64x8x16384-Kprod3-Vmse3-hq32"},
+                "metric_bytes": mbytes, "gbs": round(gbs, 1), "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4),
+                "frac_measured": round(gbs / peak, 4)}
+    elif args.workload == "quantize":
+        n, d = 1 << 20, 128
+        x = gpu_kv(torch, 1, 8, n // 8, d, wl.SEED_KEYS)
+        res = {}
+        for b in (2, 3, 4):
+            p = tq.Params(d, b, tq.TQ_MODE_PROD, 128, wl.SEED_PARAMS)
+            c = torch.empty(p.code_bytes(n), dtype=torch.uint8, device="cuda")
+            nn = torch.empty(n, dtype=torch.int16, device="cuda")
+            rn = torch.empty(n, dtype=torch.int16, device="cuda")
+            run = lambda: tq.tq_quantize(p, x, c, nn, rn)
+            for _ in range(args.warmup):
+                run()
+            torch.cuda.synchronize()
+            e0, e1 = ev(), ev()
+            e0.record()
+            for _ in range(args.steps):
+                run()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+            byts = n * d * 2 + c.numel() + 4 * n
+            gbs = byts / (ms / 1e3) / 1e9
+            res[f"b{b}"] = {"us": round(ms * 1000, 2), "vectors_per_s": n / (ms / 1e3), "gbs": round(gbs, 1),
+                            "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4), "frac_measured": round(gbs / peak, 4)}
+        line = {"metric": "quantize vectors/s", "value": res["b4"]["vectors_per_s"], "unit": "vectors/s",
+                "config": {"workload": "quantize-2^20x128-bf16-prod-m128"}, "per_bits": res}
+    else:
+        raise SystemExit(f"workload {args.workload}: not available yet")
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
 
 
 # --------------------------------------------------------------------------- main

@@ -80,9 +80,9 @@ __global__ void __launch_bounds__(128) decode_kernel(const DArgs a) {
       uint32_t bw[KB][1], sw[SW];
       const int tk = 8 * s + g;
       load_words<DP, KB, SI>(a.kcodes, a.ktb, a.km, vbase + t0 + tk, tk < ntok, t, bw, sw);
-      int accC[4] = {0, 0, 0, 0}, accS[4] = {0, 0, 0, 0};
+      int accC[2][4] = {}, accS[2][4] = {};
       sc.run(accC, accS, bw, sw);
-      double c0, c1, z0 = 0.0, z1 = 0.0;
+      float c0, c1, z0 = 0.f, z1 = 0.f;
       combine_digits(accC, lane, c0, c1);
       if constexpr (SI > 0) combine_digits(accS, lane, z0, z1);
       if (lane < 16) {
@@ -93,10 +93,10 @@ __global__ void __launch_bounds__(128) decode_kernel(const DArgs a) {
           if (tok < ntok) {
             const int64_t v = vbase + t0 + tok;
             const float n = __half2float(__ushort_as_half(a.knorms[v]));
-            float l = (float)((e ? c1 : c0) * (double)qs.x) - qs.y;
+            float l = fmaf(e ? c1 : c0, qs.x, -qs.y);
             if constexpr (SI > 0) {
               const float gm = __half2float(__ushort_as_half(a.krnorms[v]));
-              l = fmaf(gm * a.kappa, (float)((e ? z1 : z0) * (double)qs.z) - qs.w, l);
+              l = fmaf(gm * a.kappa, fmaf(e ? z1 : z0, qs.z, -qs.w), l);
             }
             val = n * l * a.sl2;
           }

@@ -80,9 +80,9 @@ __global__ void __launch_bounds__(128) logits_kernel(const LArgs a) {
       const int64_t kk = 8 * sn + g;
       load_words<DP, KB, SI>(a.codes, a.tb, a.m, vbase + kk, kk < a.n_keys, t, bw, sw);
     }
-    int accC[4] = {0, 0, 0, 0}, accS[4] = {0, 0, 0, 0};
+    int accC[2][4] = {}, accS[2][4] = {};
     sc.run(accC, accS, cbw, csw);
-    double c0, c1, z0 = 0.0, z1 = 0.0;
+    float c0, c1, z0 = 0.f, z1 = 0.f;
     combine_digits(accC, lane, c0, c1);
     if constexpr (SI > 0) combine_digits(accS, lane, z0, z1);
     if (qvalid) {
@@ -92,16 +92,146 @@ __global__ void __launch_bounds__(128) logits_kernel(const LArgs a) {
         if (key < a.n_keys) {
           const int64_t v = vbase + key;
           const float n = __half2float(__ushort_as_half(a.norms[v]));
-          float l = (float)((e ? c1 : c0) * (double)qs.x) - qs.y;
+          float l = fmaf(e ? c1 : c0, qs.x, -qs.y);
           if constexpr (SI > 0) {
             const float gm = __half2float(__ushort_as_half(a.rnorms[v]));
-            l = fmaf(gm * a.kappa, (float)((e ? z1 : z0) * (double)qs.z) - qs.w, l);
+            l = fmaf(gm * a.kappa, fmaf(e ? z1 : z0, qs.z, -qs.w), l);
           }
           out[key] = n * l;
         }
       }
     }
   }
+}
+
+// Streaming variant for key ranges whose 8-key subtiles never straddle a
+// 32-vector tile (head offsets that are multiples of 8): each warp keeps a
+// ring of RS subtiles in shared memory filled by cp.async (16-byte copies of
+// the plane rows, sign rows and the 8 norms / residual norms), so RS-1
+// subtiles (~3.8 KB per warp) are always in flight from HBM.
+constexpr int RS = 8;
+
+template <int DP, int KB, int SI>
+struct Ring {
+  static constexpr int PLANE = 8 * (DP / 8);         // bytes of one plane for 8 keys
+  static constexpr int SIGN = SI ? 8 * 32 * SI : 0;  // bytes reserved for 8 keys' sign rows (m <= 128*SI)
+  static constexpr int STAGE = KB * PLANE + SIGN + 32;
+};
+
+template <int DP, int KB, int SI>
+__global__ void __launch_bounds__(128) logits_ring_kernel(const LArgs a) {
+  using SC = Scan<DP, KB, SI>;
+  using RG = Ring<DP, KB, SI>;
+  constexpr int NH = DP / 128;
+  constexpr int SW = SI > 0 ? SI : 1;
+  __shared__ uint4 afrag[SC::FR / 4 * 32];
+  __shared__ __align__(16) uint8_t ring[4][RS][RG::STAGE];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int chunk = blockIdx.x / a.nsplit, split = blockIdx.x % a.nsplit;
+  const int head = chunk / a.nqc, qc = chunk % a.nqc;
+  const int g = lane >> 2, t = lane & 3;
+  const int qrow = QCHUNK * qc + (g & 3);
+  const bool qvalid = (lane < 16) && (qrow < a.group);
+  const int64_t n_sub = (a.n_keys + 7) / 8;
+  const int64_t per = (n_sub + a.nsplit - 1) / a.nsplit;
+  const int64_t s_begin = (int64_t)split * per;
+  const int64_t s_end = min(n_sub, s_begin + per);
+  const int64_t vbase = (int64_t)head * a.n_keys;
+  float* out = a.logits + ((int64_t)head * a.group + qrow) * a.n_keys;
+  const int sbytes = a.m / 8;  // sign bytes per key
+  const int n_sign_cp = SI ? (8 * sbytes) / 16 : 0;
+  const int n_cp = KB * 8 + n_sign_cp + 2;
+
+  // copy subtile s into ring stage st (whole subtile lies in one tile; tail keys of the
+  // last tile are zero-filled codes, their logits are not written)
+  auto issue = [&](int64_t s, int st) {
+    if (s < s_end) {
+      const int64_t v0 = vbase + 8 * s;
+      const uint8_t* tb = a.codes + (v0 >> 5) * a.tb;
+      const int slot0 = (int)(v0 & 31);
+      uint8_t* dst = ring[warp][st];
+      for (int c = lane; c < n_cp; c += 32) {
+        const uint8_t* src;
+        uint8_t* d;
+        if (c < KB * 8) {
+          const int p = c >> 3, r = c & 7;
+          src = tb + p * TILE * (DP / 8) + (slot0 + r) * (DP / 8);
+          d = dst + p * RG::PLANE + r * (DP / 8);
+          if (DP == 256) {  // two 16-byte halves per 32-byte row
+            cp_async16(d, src);
+            cp_async16(d + 16, src + 16);
+            continue;
+          }
+        } else if (c < KB * 8 + n_sign_cp) {
+          const int k = c - KB * 8;
+          src = tb + KB * TILE * (DP / 8) + slot0 * sbytes + 16 * k;
+          d = dst + KB * RG::PLANE + 16 * k;
+        } else if (c == KB * 8 + n_sign_cp) {
+          src = reinterpret_cast<const uint8_t*>(a.norms + v0);
+          d = dst + KB * RG::PLANE + RG::SIGN;
+        } else {
+          if (!SI) continue;
+          src = reinterpret_cast<const uint8_t*>(a.rnorms + v0);
+          d = dst + KB * RG::PLANE + RG::SIGN + 16;
+        }
+        cp_async16(d, src);
+      }
+    }
+    cp_async_commit();
+  };
+
+  int64_t s = s_begin + warp;
+#pragma unroll 1
+  for (int i = 0; i < RS - 1; ++i) issue(s + 4 * i, i);
+  grid_dependency_wait();
+  const uint8_t* prep = a.prep + (int64_t)chunk * a.prep_bytes;
+  SC::stage(afrag, prep);
+  const float4 qs = reinterpret_cast<const float4*>(prep + SC::FR * 128)[g & 3];
+  __syncthreads();
+  SC sc;
+  sc.load(reinterpret_cast<const uint8_t*>(afrag), lane);
+
+  int st = 0;
+  for (; s < s_end; s += 4) {
+    issue(s + 4 * (RS - 1), (st + RS - 1) % RS);
+    cp_async_wait<RS - 1>();
+    __syncwarp();
+    const uint8_t* src = ring[warp][st];
+    uint32_t bw[KB][NH], sw[SW];
+#pragma unroll
+    for (int p = 0; p < KB; ++p)
+#pragma unroll
+      for (int h = 0; h < NH; ++h)
+        bw[p][h] = reinterpret_cast<const uint32_t*>(src + p * RG::PLANE + g * (DP / 8))[t + 4 * h];
+#pragma unroll
+    for (int i = 0; i < SW; ++i) {
+      const int w = t + 4 * i;
+      sw[i] = (SI && 32 * w < a.m) ? reinterpret_cast<const uint32_t*>(src + KB * RG::PLANE + g * sbytes)[w] : 0u;
+    }
+    int accC[2][4] = {}, accS[2][4] = {};
+    sc.run(accC, accS, bw, sw);
+    float c0, c1, z0 = 0.f, z1 = 0.f;
+    combine_digits(accC, lane, c0, c1);
+    if constexpr (SI > 0) combine_digits(accS, lane, z0, z1);
+    if (qvalid) {
+      const __half* nn = reinterpret_cast<const __half*>(src + KB * RG::PLANE + RG::SIGN);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int64_t key = 8 * s + 2 * t + e;
+        if (key < a.n_keys) {
+          float l = fmaf(e ? c1 : c0, qs.x, -qs.y);
+          if constexpr (SI > 0) {
+            const float gm = __half2float(nn[8 + 2 * t + e]);
+            l = fmaf(gm * a.kappa, fmaf(e ? z1 : z0, qs.z, -qs.w), l);
+          }
+          out[key] = __half2float(nn[2 * t + e]) * l;
+        }
+      }
+    }
+    __syncwarp();
+    st = (st + 1) % RS;
+  }
+  cp_async_wait<0>();
 }
 
 template <int DP, int KB, int SI>
@@ -116,7 +246,11 @@ int launch_logits(const LArgs& a, int chunks, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, logits_kernel<DP, KB, SI>, a);
+  // the streaming kernel needs 8-key subtiles inside one tile and 16-byte aligned norm rows
+  const bool ring_ok = (a.n_keys % 8) == 0 && tq::aligned(a.norms, 16) && (!SI || tq::aligned(a.rnorms, 16)) &&
+                       (a.m % 128 == 0 || SI == 0);
+  cudaError_t e = ring_ok ? cudaLaunchKernelEx(&cfg, logits_ring_kernel<DP, KB, SI>, a)
+                          : cudaLaunchKernelEx(&cfg, logits_kernel<DP, KB, SI>, a);
   if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_logits: launch failed: %s", cudaGetErrorString(e));
   return TQ_OK;
 }

@@ -12,17 +12,20 @@
 namespace {
 using namespace tqd;
 
+constexpr int PREP_SPLIT = 4;  // CTAs per chunk (each writes a quarter of the fragment words)
+
 __global__ void __launch_bounds__(256) qprep_kernel(const PrepArgs a) {
   __shared__ float qt[QCHUNK][256];
   __shared__ float uu[QCHUNK][256];
-  __shared__ int W[QCHUNK][4][256];
-  __shared__ int V[QCHUNK][256];
+  // int8 digits of the shifted integer weights: dw[digit][query][plane][coordinate], ds[digit][query][row]
+  __shared__ int8_t dw[4][QCHUNK][4][256];
+  __shared__ int8_t ds[4][QCHUNK][256];
   __shared__ float alpha[4];
   __shared__ float qstat[QCHUNK][2];  // sum q_rot, max |q_rot|
   __shared__ int FG[QCHUNK][2];
   // the scan kernel may be scheduled now; it waits for this grid before reading the output
   asm volatile("griddepcontrol.launch_dependents;\n" ::);
-  const int chunk = blockIdx.x;
+  const int chunk = blockIdx.x / PREP_SPLIT, part = blockIdx.x % PREP_SPLIT;
   const int outer = chunk / a.nqc, qc = chunk % a.nqc;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NT = walsh_planes(a.kb);
@@ -82,25 +85,27 @@ __global__ void __launch_bounds__(256) qprep_kernel(const PrepArgs a) {
     }
   }
   __syncthreads();
-  // u = S q_rot: thread i owns projection row i for all four queries
-  for (int i = threadIdx.x; i < a.m; i += blockDim.x) {
-    float acc[QCHUNK] = {0.f, 0.f, 0.f, 0.f};
+  // u = S q_rot: thread (row i, query pair) -- 2 x 128 FMA per thread for m <= 128
+  for (int e = threadIdx.x; e < 2 * a.m; e += blockDim.x) {
+    const int i = e % a.m, qp = e / a.m;  // queries 2qp, 2qp+1
+    float acc0 = 0.f, acc1 = 0.f;
     const uint4* srow = reinterpret_cast<const uint4*>(a.S + (size_t)i * a.dp);
+    const float* q0 = qt[2 * qp];
+    const float* q1 = qt[2 * qp + 1];
     for (int k = 0; k < a.dp / 8; ++k) {
       const uint4 v = __ldg(srow + k);
       const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[e]));
-#pragma unroll
-        for (int qq = 0; qq < QCHUNK; ++qq) {
-          acc[qq] = fmaf(f.x, qt[qq][8 * k + 2 * e], acc[qq]);
-          acc[qq] = fmaf(f.y, qt[qq][8 * k + 2 * e + 1], acc[qq]);
-        }
+      for (int h = 0; h < 4; ++h) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[h]));
+        acc0 = fmaf(f.x, q0[8 * k + 2 * h], acc0);
+        acc0 = fmaf(f.y, q0[8 * k + 2 * h + 1], acc0);
+        acc1 = fmaf(f.x, q1[8 * k + 2 * h], acc1);
+        acc1 = fmaf(f.y, q1[8 * k + 2 * h + 1], acc1);
       }
     }
-#pragma unroll
-    for (int qq = 0; qq < QCHUNK; ++qq) uu[qq][i] = acc[qq];
+    uu[2 * qp][i] = acc0;
+    uu[2 * qp + 1][i] = acc1;
   }
   __syncthreads();
   if (warp < QCHUNK) {  // scales: weights 2 alpha q_rot and 2 u become integers below 2^23
@@ -129,73 +134,77 @@ __global__ void __launch_bounds__(256) qprep_kernel(const PrepArgs a) {
     if (lane == 0) {
       FG[qi][0] = F;
       FG[qi][1] = G;
-      float4* scal = reinterpret_cast<float4*>(a.out + (int64_t)chunk * prep_chunk_bytes(a.fr) + (int64_t)a.fr * 128);
-      // sum_T alpha_T = c[L-1] (all index bits set)
-      scal[qi] = make_float4(ldexpf(1.f, -(F + 7)), a.cent[L - 1] * qstat[qi][0], ldexpf(1.f, -(G + 7)), su);
+      if (part == 0) {
+        float4* scal =
+            reinterpret_cast<float4*>(a.out + (int64_t)chunk * prep_chunk_bytes(a.fr) + (int64_t)a.fr * 128);
+        // sum_T alpha_T = c[L-1] (all index bits set)
+        scal[qi] = make_float4(ldexpf(1.f, -(F + 7)), a.cent[L - 1] * qstat[qi][0], ldexpf(1.f, -(G + 7)), su);
+      }
     }
   }
   __syncthreads();
+  // Each weight is used with one bit class only (c = coordinate % 8): shift by 7-c once and
+  // split into balanced base-256 digits.
+  auto digits = [](int X, int8_t* d0, int stride) {
+    for (int k = 0; k < 3; ++k) {
+      const int lowb = (int)(int8_t)(X & 0xFF);
+      d0[k * stride] = (int8_t)lowb;
+      X = (X - lowb) >> 8;
+    }
+    d0[3 * stride] = (int8_t)X;
+  };
   for (int e = threadIdx.x; e < QCHUNK * NT * a.dp; e += blockDim.x) {
     const int qq = e / (NT * a.dp), r = e % (NT * a.dp), T = r / a.dp, j = r % a.dp;
-    W[qq][T][j] = __float2int_rn(ldexpf(2.f * alpha[T] * qt[qq][j], FG[qq][0]));
+    const int X = __float2int_rn(ldexpf(2.f * alpha[T] * qt[qq][j], FG[qq][0])) * (1 << (7 - (j & 7)));
+    digits(X, &dw[0][qq][T][j], QCHUNK * 4 * 256);
   }
-  for (int e = threadIdx.x; e < QCHUNK * a.m; e += blockDim.x) {
-    const int qq = e / a.m, i = e % a.m;
-    V[qq][i] = __float2int_rn(ldexpf(2.f * uu[qq][i], FG[qq][1]));
+  for (int e = threadIdx.x; e < QCHUNK * 256; e += blockDim.x) {
+    const int qq = e / 256, i = e % 256;
+    const int X = (i < a.m) ? __float2int_rn(ldexpf(2.f * uu[qq][i], FG[qq][1])) * (1 << (7 - (i & 7))) : 0;
+    digits(X, &ds[0][qq][i], QCHUNK * 256);
   }
   __syncthreads();
 
-  // A fragments (layout in scan.cuh)
+  // A fragments (layout in scan.cuh); this CTA writes words w = part, part + PREP_SPLIT, ...
   const ScanShape sh(a.dp, a.kb, a.m);
   const int NH = a.dp / 128;
   uint32_t* frag = reinterpret_cast<uint32_t*>(a.out + (int64_t)chunk * prep_chunk_bytes(a.fr));
-  for (int widx = threadIdx.x; widx < 32 * a.fr; widx += blockDim.x) {
-    const int L2 = widx & 31, w = widx >> 5;
+  for (int widx = threadIdx.x; widx < 32 * a.fr / PREP_SPLIT; widx += blockDim.x) {
+    const int L2 = widx & 31, w = (widx >> 5) * PREP_SPLIT + part;
     uint32_t word = 0u;
-    if (w < 8 * sh.per_c) {
+    if (w < sh.fr) {
       const int c = w / sh.per_c, o = w % sh.per_c;
       const int g = L2 >> 2, t = L2 & 3;
-      int reg, item;
-      bool sign;
-      if (o < 4 * sh.ncp) {
+      const int slot = o >> 2;
+      int reg = o & 3, item = 0;
+      bool sign, pad = false;
+      if (slot < sh.ncp) {  // centroid k32 pair: a0,a1 -> first item, a2,a3 -> second
         sign = false;
-        reg = o & 3;
-        item = 2 * (o >> 2) + (reg >= 2 ? 1 : 0);
-      } else if (o < 4 * sh.ncp + 2 * sh.ncs) {
+        item = 2 * slot + (reg >= 2 ? 1 : 0);
+      } else if (slot < sh.ncp + sh.ncs) {  // centroid k16 single
         sign = false;
-        reg = o - 4 * sh.ncp;
         item = sh.nci - 1;
-      } else if (o < 4 * sh.ncp + 2 * sh.ncs + 4 * sh.nsp) {
+        pad = reg >= 2;
+      } else if (slot < sh.ncp + sh.ncs + sh.nsp) {  // sign k32 pair
         sign = true;
-        reg = (o - 4 * sh.ncp - 2 * sh.ncs) & 3;
         item = reg >= 2 ? 1 : 0;
-      } else {
+      } else {  // sign k16 single
         sign = true;
-        reg = o - 4 * sh.ncp - 2 * sh.ncs - 4 * sh.nsp;
         item = 0;
+        pad = reg >= 2;
       }
-      const int r = (reg & 1) ? g + 8 : g;
-      const int digit = r >> 2, qq = r & 3;
-      for (int jj = 0; jj < 4; ++jj) {
-        int X = 0;
+      if (!pad) {
+        const int r = (reg & 1) ? g + 8 : g;
+        const int digit = r >> 2, qq = r & 3;
+        const int8_t* src;
         if (sign) {
-          const int wi = t + 4 * item;
-          const int j = 32 * wi + c + 8 * jj;
-          X = (j < a.m) ? V[qq][j] : 0;
+          src = &ds[digit][qq][32 * (t + 4 * item) + c];
         } else {
           const int T = item / NH, hh = item % NH;
-          const int wi = t + 4 * hh;
-          X = W[qq][T][32 * wi + c + 8 * jj];
+          src = &dw[digit][qq][T][32 * (t + 4 * hh) + c];
         }
-        X *= (1 << (7 - c));
-        int dv[4];  // balanced base-256 digits
-        for (int k = 0; k < 3; ++k) {
-          const int lowb = (int)(int8_t)(X & 0xFF);
-          dv[k] = lowb;
-          X = (X - lowb) >> 8;
-        }
-        dv[3] = X;
-        word |= ((uint32_t)(uint8_t)(int8_t)dv[digit]) << (8 * jj);
+        word = (uint32_t)(uint8_t)src[0] | ((uint32_t)(uint8_t)src[8] << 8) | ((uint32_t)(uint8_t)src[16] << 16) |
+               ((uint32_t)(uint8_t)src[24] << 24);
       }
     }
     frag[((int64_t)(w >> 2) * 32 + L2) * 4 + (w & 3)] = word;
@@ -209,7 +218,7 @@ namespace tq {
 int launch_prep(const tqd::PrepArgs& a, cudaStream_t st) {
   const int chunks = a.n_outer * a.nqc;
   if (chunks <= 0) return TQ_OK;
-  qprep_kernel<<<chunks, 256, 0, st>>>(a);
+  qprep_kernel<<<chunks * PREP_SPLIT, 256, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(TQ_ECUDA, "query prep launch failed: %s", cudaGetErrorString(e));
   return TQ_OK;

@@ -41,7 +41,9 @@ __host__ __device__ __forceinline__ int walsh_mask(int kb, int T) {
 }
 __host__ __device__ __forceinline__ int walsh_planes(int kb) { return kb == 1 ? 1 : (kb == 2 ? 2 : 4); }
 
-// Fragment words per lane for a scan configuration (multiple of 4).
+// Fragment words per lane for a scan configuration.  Per bit class c there is
+// one 4-word slot per MMA: centroid k32 pairs, then a centroid k16 single,
+// then the sign k32 pair or k16 single (k16 slots use words 0 and 1).
 struct ScanShape {
   int nt, nci, ncp, ncs, nsi, nsp, nss, per_c, fr;
   __host__ __device__ ScanShape(int dp, int kb, int m) {
@@ -52,8 +54,8 @@ struct ScanShape {
     nsi = m == 0 ? 0 : (m > 128 ? 2 : 1);
     nsp = nsi / 2;
     nss = nsi % 2;
-    per_c = 4 * ncp + 2 * ncs + 4 * nsp + 2 * nss;
-    fr = (8 * per_c + 3) & ~3;
+    per_c = 4 * (ncp + ncs + nsp + nss);  // one 16-byte slot per MMA (k16 uses half of it)
+    fr = 8 * per_c;
   }
 };
 
@@ -81,9 +83,9 @@ struct Scan {
   static constexpr int NCI = NT * NH;
   static constexpr int NCP = NCI / 2, NCS = NCI % 2;
   static constexpr int NSP = SI / 2, NSS = SI % 2;
-  static constexpr int PER_C = 4 * NCP + 2 * NCS + 4 * NSP + 2 * NSS;
-  static constexpr int FR = (8 * PER_C + 3) & ~3;
-  static_assert(NCI <= 4, "too many plane words per lane");
+  static constexpr int NSLOT = NCP + NCS + NSP + NSS;  // MMAs per bit class
+  static constexpr int PER_C = 4 * NSLOT;
+  static constexpr int FR = 8 * PER_C;
 
   uint32_t A[FR];
 
@@ -106,8 +108,9 @@ struct Scan {
     for (int k = threadIdx.x; k < FR / 4 * 32; k += blockDim.x) smem[k] = __ldg(f + k);
   }
 
-  // bw[p][h]: word (t + 4h) of bit-plane p of this lane's key; sw[i]: sign word (t + 4i)
-  __device__ __forceinline__ void run(int (&accC)[4], int (&accS)[4], const uint32_t (&bw)[KB][NH],
+  // bw[p][h]: word (t + 4h) of bit-plane p of this lane's key; sw[i]: sign word (t + 4i).
+  // Two accumulator sets per sum (even / odd bit class) halve the dependent MMA chain.
+  __device__ __forceinline__ void run(int (&accC)[2][4], int (&accS)[2][4], const uint32_t (&bw)[KB][NH],
                                       const uint32_t (&sw)[SI > 0 ? SI : 1]) const {
     uint32_t it[NCI];
 #pragma unroll
@@ -122,15 +125,17 @@ struct Scan {
     for (int c = 0; c < 8; ++c) {
       const uint32_t mk = 0x01010101u << c;
       const int base = c * PER_C;
+      int (&aC)[4] = accC[c & 1];
+      int (&aS)[4] = accS[c & 1];
 #pragma unroll
       for (int p = 0; p < NCP; ++p)
-        mma_s8u8_16832(accC, A[base + 4 * p], A[base + 4 * p + 1], A[base + 4 * p + 2], A[base + 4 * p + 3],
+        mma_s8u8_16832(aC, A[base + 4 * p], A[base + 4 * p + 1], A[base + 4 * p + 2], A[base + 4 * p + 3],
                        it[2 * p] & mk, it[2 * p + 1] & mk);
-      if constexpr (NCS) mma_s8u8_16816(accC, A[base + 4 * NCP], A[base + 4 * NCP + 1], it[NCI - 1] & mk);
-      constexpr int o = 4 * NCP + 2 * NCS;
-      if constexpr (NSP) mma_s8u8_16832(accS, A[base + o], A[base + o + 1], A[base + o + 2], A[base + o + 3],
+      if constexpr (NCS) mma_s8u8_16816(aC, A[base + 4 * NCP], A[base + 4 * NCP + 1], it[NCI - 1] & mk);
+      constexpr int o = 4 * (NCP + NCS);
+      if constexpr (NSP) mma_s8u8_16832(aS, A[base + o], A[base + o + 1], A[base + o + 2], A[base + o + 3],
                                         sw[0] & mk, sw[SI > 1 ? 1 : 0] & mk);
-      if constexpr (NSS) mma_s8u8_16816(accS, A[base + o + 4 * NSP], A[base + o + 4 * NSP + 1], sw[0] & mk);
+      if constexpr (NSS) mma_s8u8_16816(aS, A[base + o], A[base + o + 1], sw[0] & mk);
     }
   }
 };
@@ -139,15 +144,17 @@ struct Scan {
 // has completed and its writes are visible.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 
-// Combine the digit rows of an accumulator: thread (g, t) holds rows g, g+8
-// (digits g>>2 and 2+(g>>2) of query g&3) for keys 2t, 2t+1.  Returns, in
-// lanes 0..15, the exact integer sums (as double) for query g, keys 2t, 2t+1.
-__device__ __forceinline__ void combine_digits(const int (&acc)[4], int lane, double& k0, double& k1) {
+// Combine the digit rows of an accumulator pair: thread (g, t) holds rows g,
+// g+8 (digits g>>2 and 2+(g>>2) of query g&3) for keys 2t, 2t+1.  Returns, in
+// lanes 0..15, sum_r 256^digit C[r] for query g, keys 2t, 2t+1.  Each row sum
+// is an exact int32 below 2^24 in magnitude (so exact in fp32); the weighted
+// sum is rounded to fp32 (relative 2^-24, far inside the logit tolerance).
+__device__ __forceinline__ void combine_digits(const int (&acc)[2][4], int lane, float& k0, float& k1) {
   const int g = lane >> 2;
-  const double lo = (g >> 2) ? 256.0 : 1.0;
-  const double hi = (g >> 2) ? 16777216.0 : 65536.0;
-  k0 = (double)acc[0] * lo + (double)acc[2] * hi;
-  k1 = (double)acc[1] * lo + (double)acc[3] * hi;
+  const float lo = (g >> 2) ? 256.f : 1.f;
+  const float hi = (g >> 2) ? 16777216.f : 65536.f;
+  k0 = fmaf((float)(acc[0][2] + acc[1][2]), hi, (float)(acc[0][0] + acc[1][0]) * lo);
+  k1 = fmaf((float)(acc[0][3] + acc[1][3]), hi, (float)(acc[0][1] + acc[1][1]) * lo);
   k0 += __shfl_xor_sync(FULL, k0, 16);
   k1 += __shfl_xor_sync(FULL, k1, 16);
 }
