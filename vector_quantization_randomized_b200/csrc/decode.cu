@@ -80,10 +80,11 @@ __global__ void __launch_bounds__(128) decode_kernel(const DArgs a) {
       uint32_t bw[KB][1], sw[SW];
       const int tk = 8 * s + g;
       load_words<DP, KB, SI>(a.kcodes, a.ktb, a.km, vbase + t0 + tk, tk < ntok, t, bw, sw);
-      int accC[2][4] = {}, accS[2][4] = {};
+      int accC[2][SC::NCSL][4] = {}, accS[2][4] = {}, accF[2][4];
       sc.run(accC, accS, bw, sw);
+      SC::fold(accC, accF);
       float c0, c1, z0 = 0.f, z1 = 0.f;
-      combine_digits(accC, lane, c0, c1);
+      combine_digits(accF, lane, c0, c1);
       if constexpr (SI > 0) combine_digits(accS, lane, z0, z1);
       if (lane < 16) {
 #pragma unroll

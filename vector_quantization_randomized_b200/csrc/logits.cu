@@ -80,10 +80,11 @@ __global__ void __launch_bounds__(128) logits_kernel(const LArgs a) {
       const int64_t kk = 8 * sn + g;
       load_words<DP, KB, SI>(a.codes, a.tb, a.m, vbase + kk, kk < a.n_keys, t, bw, sw);
     }
-    int accC[2][4] = {}, accS[2][4] = {};
+    int accC[2][SC::NCSL][4] = {}, accS[2][4] = {}, accF[2][4];
     sc.run(accC, accS, cbw, csw);
+    SC::fold(accC, accF);
     float c0, c1, z0 = 0.f, z1 = 0.f;
-    combine_digits(accC, lane, c0, c1);
+    combine_digits(accF, lane, c0, c1);
     if constexpr (SI > 0) combine_digits(accS, lane, z0, z1);
     if (qvalid) {
 #pragma unroll
@@ -208,10 +209,11 @@ __global__ void __launch_bounds__(128) logits_ring_kernel(const LArgs a) {
       const int w = t + 4 * i;
       sw[i] = (SI && 32 * w < a.m) ? reinterpret_cast<const uint32_t*>(src + KB * RG::PLANE + g * sbytes)[w] : 0u;
     }
-    int accC[2][4] = {}, accS[2][4] = {};
+    int accC[2][SC::NCSL][4] = {}, accS[2][4] = {}, accF[2][4];
     sc.run(accC, accS, bw, sw);
+    SC::fold(accC, accF);
     float c0, c1, z0 = 0.f, z1 = 0.f;
-    combine_digits(accC, lane, c0, c1);
+    combine_digits(accF, lane, c0, c1);
     if constexpr (SI > 0) combine_digits(accS, lane, z0, z1);
     if (qvalid) {
       const __half* nn = reinterpret_cast<const __half*>(src + KB * RG::PLANE + RG::SIGN);

@@ -109,8 +109,10 @@ struct Scan {
   }
 
   // bw[p][h]: word (t + 4h) of bit-plane p of this lane's key; sw[i]: sign word (t + 4i).
-  // Two accumulator sets per sum (even / odd bit class) halve the dependent MMA chain.
-  __device__ __forceinline__ void run(int (&accC)[2][4], int (&accS)[2][4], const uint32_t (&bw)[KB][NH],
+  // Every MMA slot accumulates into its own register set, separately for even and
+  // odd bit classes, so a subtile carries 2*NSLOT independent MMA chains.
+  static constexpr int NCSL = NCP + NCS;  // centroid slots
+  __device__ __forceinline__ void run(int (&accC)[2][NCSL][4], int (&accS)[2][4], const uint32_t (&bw)[KB][NH],
                                       const uint32_t (&sw)[SI > 0 ? SI : 1]) const {
     uint32_t it[NCI];
 #pragma unroll
@@ -125,18 +127,29 @@ struct Scan {
     for (int c = 0; c < 8; ++c) {
       const uint32_t mk = 0x01010101u << c;
       const int base = c * PER_C;
-      int (&aC)[4] = accC[c & 1];
-      int (&aS)[4] = accS[c & 1];
 #pragma unroll
       for (int p = 0; p < NCP; ++p)
-        mma_s8u8_16832(aC, A[base + 4 * p], A[base + 4 * p + 1], A[base + 4 * p + 2], A[base + 4 * p + 3],
-                       it[2 * p] & mk, it[2 * p + 1] & mk);
-      if constexpr (NCS) mma_s8u8_16816(aC, A[base + 4 * NCP], A[base + 4 * NCP + 1], it[NCI - 1] & mk);
+        mma_s8u8_16832(accC[c & 1][p], A[base + 4 * p], A[base + 4 * p + 1], A[base + 4 * p + 2],
+                       A[base + 4 * p + 3], it[2 * p] & mk, it[2 * p + 1] & mk);
+      if constexpr (NCS) mma_s8u8_16816(accC[c & 1][NCP], A[base + 4 * NCP], A[base + 4 * NCP + 1], it[NCI - 1] & mk);
       constexpr int o = 4 * (NCP + NCS);
-      if constexpr (NSP) mma_s8u8_16832(aS, A[base + o], A[base + o + 1], A[base + o + 2], A[base + o + 3],
+      if constexpr (NSP) mma_s8u8_16832(accS[c & 1], A[base + o], A[base + o + 1], A[base + o + 2], A[base + o + 3],
                                         sw[0] & mk, sw[SI > 1 ? 1 : 0] & mk);
-      if constexpr (NSS) mma_s8u8_16816(aS, A[base + o], A[base + o + 1], sw[0] & mk);
+      if constexpr (NSS) mma_s8u8_16816(accS[c & 1], A[base + o], A[base + o + 1], sw[0] & mk);
     }
+  }
+
+  // Fold the centroid chains into one [2][4] set (exact integer sums).
+  __device__ __forceinline__ static void fold(const int (&accC)[2][NCSL][4], int (&out)[2][4]) {
+#pragma unroll
+    for (int par = 0; par < 2; ++par)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        int v = 0;
+#pragma unroll
+        for (int p = 0; p < NCSL; ++p) v += accC[par][p][r];
+        out[par][r] = v;
+      }
   }
 };
 
