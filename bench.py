@@ -464,6 +464,49 @@ def run_secondary(args, world, rank, local, torch, tq, wl):
                             "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4), "frac_measured": round(gbs / peak, 4)}
         line = {"metric": "quantize vectors/s", "value": res["b4"]["vectors_per_s"], "unit": "vectors/s",
                 "config": {"workload": "quantize-2^20x128-bf16-prod-m128"}, "per_bits": res}
+    elif args.workload == "search":
+        n_db, n_q, d, k = 1000000, 10000, 200, 10
+        db = torch.from_numpy(wl.search_set(n_db, d, seed=wl.SEED_KEYS)).to(torch.bfloat16).cuda()
+        qs = torch.from_numpy(wl.search_set(n_q, d, seed=wl.SEED_QUERIES)).cuda()
+        # exact top-10 by fp32 inner product on the (bf16-rounded) database (torch.matmul, chunked)
+        dbf = db.float()
+        truth = []
+        for s0 in range(0, n_q, 1000):
+            sc = qs[s0:s0 + 1000] @ dbf.T
+            truth.append(torch.topk(sc, k, dim=1).indices.cpu())
+        truth = torch.cat(truth).numpy()
+        del dbf
+        res = {}
+        for b in (2, 4):
+            p = tq.Params(d, b, tq.TQ_MODE_PROD, 256, wl.SEED_PARAMS)
+            c = torch.empty(p.code_bytes(n_db), dtype=torch.uint8, device="cuda")
+            nn = torch.empty(n_db, dtype=torch.int16, device="cuda")
+            rn = torch.empty(n_db, dtype=torch.int16, device="cuda")
+            e0, e1 = ev(), ev()
+            e0.record()
+            tq.tq_quantize(p, db, c, nn, rn)
+            e1.record()
+            torch.cuda.synchronize()
+            q_ms = e0.elapsed_time(e1)
+            ids = torch.empty((n_q, k), dtype=torch.int32, device="cuda")
+            scs = torch.empty((n_q, k), dtype=torch.float32, device="cuda")
+            ws = torch.empty(tq.tq_search_workspace(p, n_q, n_db, k), dtype=torch.uint8, device="cuda")
+            run = lambda: tq.tq_search_topk(p, qs, c, nn, rn, n_db, k, ids, scs, ws)
+            for _ in range(max(1, args.warmup)):
+                run()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(args.steps):
+                run()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+            got = ids.cpu().numpy()
+            recall = float(np.mean([len(set(got[i]) & set(truth[i])) / k for i in range(n_q)]))
+            res[f"b{b}"] = {"search_ms": round(ms, 3), "estimates_per_s": n_q * n_db / (ms / 1e3),
+                            "recall_at_10": round(recall, 4), "quantize_db_ms": round(q_ms, 3)}
+        line = {"metric": "search estimates/s", "value": res["b4"]["estimates_per_s"], "unit": "estimates/s",
+                "config": {"workload": "search-1e6x200-1e4q-top10"}, "per_bits": res}
     else:
         raise SystemExit(f"workload {args.workload}: not available yet")
     if rank == 0:

@@ -22,14 +22,15 @@
 //    predicate is packed into a 32-bit word with one predicated OR, and the
 //    bit-planes are a few word-wide XORs.  The residual is |y| - mag[m] with
 //    the sign of s.
-//  * QJL: residuals are rounded to fp16 and written to shared memory in the
-//    UMMA K-major canonical layout; one thread issues tcgen05.mma (M=128,
-//    N=m, K=16) x 8 per half tile against S (fp16, exact) with fp32
+//  * QJL: residuals are written to shared memory in the UMMA K-major
+//    canonical layout; one thread issues tcgen05.mma (M=128, N=m, K=16)
+//    x 16 per half tile against S (fp16, exact) with fp32
 //    accumulation in tensor memory; every thread reads its own row back with
-//    tcgen05.ld.32x32b.  A projection with |z| <= max||S_i|| (||r - fp16(r)||
-//    + 2^-15 gamma) could have its sign changed by the fp16 rounding of r or
-//    the fp32 accumulation; for those (about 0.2 per vector) the thread
-//    recomputes r exactly (same code path) and the projection in fp32.
+//    tcgen05.ld.32x32b.  The residual (scaled by 2^14) is split into fp16 hi
+//    and lo parts and the MMA runs twice into the same accumulator
+//    (S r_hi + S r_lo), so z is exact to ~2^-22 before fp32 accumulation.  A
+//    projection with |z| below the accumulation bound (about 0.03 per vector)
+//    is recomputed in fp32 from hi+lo by its thread.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -64,8 +65,9 @@ struct Q2Args {
 struct Lay {
   static constexpr int XS = 0;                    // [NV][ROWB] staged input (swizzled chunks)
   static constexpr int SS = XS + NV * ROWB;       // S, canonical K-major fp16, 128 rows max
-  static constexpr int RS = SS + 128 * DP * 2;    // residuals fp16, canonical, two 128-row halves
-  static constexpr int DM = RS + NV * DP * 2;     // sign-flip masks, 64 x uint32 (bits 15, 31)
+  static constexpr int RS = SS + 128 * DP * 2;    // residuals (hi part) fp16, canonical, two 128-row halves
+  static constexpr int RL = RS + NV * DP * 2;     // residuals (lo part), same layout
+  static constexpr int DM = RL + NV * DP * 2;     // sign-flip masks, 64 x uint32 (bits 15, 31)
   static constexpr int MISC = DM + 64 * 4;        // mbarrier, tmem base, max ||S_i||
   static constexpr int TOTAL = MISC + 64;
 };
@@ -203,16 +205,11 @@ __device__ __forceinline__ void encode_row(const uint8_t* xrow, int sw, int d, c
   g2 = acc.x + acc.y;
 }
 
-// Rare path: recompute r exactly (the same code path as the main encode, on the
-// input row re-read from global memory, unswizzled) and the doubtful
-// projections z_i = S_i . r in fp32; overwrite their sign bits.
-template <int KB, int DT>
-__device__ __noinline__ void fixup_signs(const uint8_t* src, int d, const uint32_t* dmask, const Coder<KB>& cd,
-                                         const uint8_t* Ss, const uint32_t (&need)[4], uint32_t (&sgn)[4]) {
-  float2 rr[64];
-  uint32_t pp[KB][4];
-  float nn, gg;
-  encode_row<KB, DT>(src, 0, d, dmask, cd, pp, nn, gg, [&](int k, float2 rv) { rr[k] = rv; });
+// Rare path: projections whose two-pass tensor-core value is within the
+// rounding bound of zero are recomputed in fp32 from the hi+lo residual parts
+// (2^-22 relative), and their sign bits overwritten.
+__device__ __noinline__ void fixup_signs(const uint8_t* Ss, const uint8_t* rh, const uint8_t* rl, int row,
+                                         const uint32_t (&need)[4], uint32_t (&sgn)[4]) {
   for (int w = 0; w < 4; ++w) {
     uint32_t nd = need[w];
     while (nd) {
@@ -222,8 +219,10 @@ __device__ __noinline__ void fixup_signs(const uint8_t* src, int d, const uint32
       float s = 0.f;
       for (int k = 0; k < 64; ++k) {
         const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(Ss + canon(i, 2 * k)));
-        s = fmaf(sf.x, rr[k].x, s);
-        s = fmaf(sf.y, rr[k].y, s);
+        const float2 h = __half22float2(*reinterpret_cast<const __half2*>(rh + canon(row, 2 * k)));
+        const float2 l = __half22float2(*reinterpret_cast<const __half2*>(rl + canon(row, 2 * k)));
+        s = fmaf(sf.x, h.x + l.x, s);
+        s = fmaf(sf.y, h.y + l.y, s);
       }
       if (s >= 0.f) sgn[w] |= 1u << j;
       else sgn[w] &= ~(1u << j);
@@ -308,26 +307,35 @@ __global__ void __launch_bounds__(NV, 1) quantize128_kernel(const Q2Args a) {
     const bool valid = v < a.n_vec, inpad = v < a.n_pad;
     uint32_t pl[KB][4];
     float n = 0.f, g2 = 0.f;
-    // fp16 residuals go straight into the canonical A tile of the QJL MMA (zeros for rows
-    // without a vector); ||r - fp16(r)||^2 feeds the fix-up bound
+    // Residuals, scaled by 2^14 (|r| < 2 for a unit vector, so no fp16 overflow and no
+    // subnormal hi/lo parts), go straight into the canonical A tiles of the QJL MMA as
+    // an fp16 hi part and an fp16 lo part (zeros for rows without a vector).
     const int half = tid >> 7, row = tid & 127;
     uint8_t* ra = Rs + half * (128 * DP * 2);
-    float2 e2 = make_float2(0.f, 0.f);
-    uint32_t hq[4];
+    uint8_t* rl = smem + Lay::RL + half * (128 * DP * 2);
+    uint32_t hq[4], lq[4];
     auto sink = [&](int k, float2 rv) {
       if constexpr (PROD) {
-        const __half2 hv = __floats2half2_rn(rv.x, rv.y);
+        const float2 sr = __fmul2_rn(rv, make_float2(16384.f, 16384.f));
+        const __half2 hv = __floats2half2_rn(sr.x, sr.y);
+        const float2 dl = __ffma2_rn(__half22float2(hv), make_float2(-1.f, -1.f), sr);  // exact
+        const __half2 lv = __floats2half2_rn(dl.x, dl.y);
         hq[k & 3] = *reinterpret_cast<const uint32_t*>(&hv);
-        const float2 dlt = __ffma2_rn(__half22float2(hv), make_float2(-1.f, -1.f), rv);
-        e2 = __ffma2_rn(dlt, dlt, e2);
-        if ((k & 3) == 3) *reinterpret_cast<uint4*>(ra + canon(row, 2 * (k - 3))) = make_uint4(hq[0], hq[1], hq[2], hq[3]);
+        lq[k & 3] = *reinterpret_cast<const uint32_t*>(&lv);
+        if ((k & 3) == 3) {
+          *reinterpret_cast<uint4*>(ra + canon(row, 2 * (k - 3))) = make_uint4(hq[0], hq[1], hq[2], hq[3]);
+          *reinterpret_cast<uint4*>(rl + canon(row, 2 * (k - 3))) = make_uint4(lq[0], lq[1], lq[2], lq[3]);
+        }
       }
     };
     if (valid) {
       encode_row<KB, DT>(xs + tid * ROWB, tid & 7, a.d, dmask, cd, pl, n, g2, sink);
     } else if (PROD) {
 #pragma unroll
-      for (int kc = 0; kc < KCH; ++kc) *reinterpret_cast<uint4*>(ra + canon(row, 8 * kc)) = make_uint4(0, 0, 0, 0);
+      for (int kc = 0; kc < KCH; ++kc) {
+        *reinterpret_cast<uint4*>(ra + canon(row, 8 * kc)) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(rl + canon(row, 8 * kc)) = make_uint4(0, 0, 0, 0);
+      }
     }
     __syncthreads();  // every row is consumed: refill the staging buffer with the next tile
     if (tile + gridDim.x < n_tiles) issue(tile + gridDim.x);
@@ -345,7 +353,9 @@ __global__ void __launch_bounds__(NV, 1) quantize128_kernel(const Q2Args a) {
     if constexpr (PROD) {
       const float gm = sqrtf(g2);
       if (valid) a.rnorms[v] = __half_as_ushort(__float2half_rn(gm));
-      const float bound = (*smax) * (sqrtf(e2.x + e2.y) + 3.0517578125e-05f * gm);  // 2^-15
+      // |z - S_i.r'| <= max||S_i|| (2^-21 + 2^-15) gamma' covers the lo-part rounding and the
+      // fp32 accumulation of 256 exact products (gamma' = 2^14 gamma)
+      const float bound = (*smax) * (16384.f * gm) * 3.1471252e-05f;  // 2^-15 + 2^-21
       fence_async_smem();
       tc_fence_before();
       __syncthreads();
@@ -355,11 +365,14 @@ __global__ void __launch_bounds__(NV, 1) quantize128_kernel(const Q2Args a) {
         const uint32_t sB = smem_u32(Ss);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-          const uint32_t sA = smem_u32(Rs + hf * (128 * DP * 2));
 #pragma unroll
-          for (int ks = 0; ks < DP / 16; ++ks)
-            umma_f16(tmem + hf * 128, smem_desc(sA + ks * 256, lbo, sbo), smem_desc(sB + ks * 256, lbo, sbo), idesc,
-                     ks > 0 ? 1u : 0u);
+          for (int part = 0; part < 2; ++part) {  // z = S r_hi + S r_lo
+            const uint32_t sA = smem_u32(smem + (part ? Lay::RL : Lay::RS) + hf * (128 * DP * 2));
+#pragma unroll
+            for (int ks = 0; ks < DP / 16; ++ks)
+              umma_f16(tmem + hf * 128, smem_desc(sA + ks * 256, lbo, sbo), smem_desc(sB + ks * 256, lbo, sbo),
+                       idesc, (part | ks) ? 1u : 0u);
+          }
         }
         umma_commit(bar);
       }
@@ -368,24 +381,38 @@ __global__ void __launch_bounds__(NV, 1) quantize128_kernel(const Q2Args a) {
       tc_fence_after();
       // read back this vector's projections: lane = row within its half, columns [half*128, half*128 + m)
       const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(half * 128);
-      uint32_t sgn[4] = {0, 0, 0, 0}, need[4] = {0, 0, 0, 0};
+      uint32_t sgn[4] = {0, 0, 0, 0};
+      float zmin = INFINITY;
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         if (32 * w < a.m) {  // uniform: every lane of the warp executes the tcgen05.ld
           float z[32];
           tmem_ld32(taddr + 32 * w, z);
-          uint32_t word = 0, nd = 0;
+          uint32_t word = 0;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (z[j] >= 0.f) word |= 1u << j;
-            if (fabsf(z[j]) <= bound) nd |= 1u << j;
+            zmin = fminf(zmin, fabsf(z[j]));
           }
           sgn[w] = word;
-          need[w] = nd;
         }
       }
-      if (valid && (need[0] | need[1] | need[2] | need[3]))
-        fixup_signs<KB, DT>(a.x + v * a.ld_bytes, a.d, dmask, cd, Ss, need, sgn);
+      const bool doubt = valid && zmin <= bound;
+      if (__any_sync(FULL, doubt)) {  // rare, warp-uniform: find the doubtful projections
+        uint32_t need[4] = {0, 0, 0, 0};
+        for (int w = 0; w < 4; ++w) {
+          if (32 * w < a.m) {
+            float z[32];
+            tmem_ld32(taddr + 32 * w, z);
+            uint32_t nd = 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (fabsf(z[j]) <= bound) nd |= 1u << j;
+            need[w] = doubt ? nd : 0u;
+          }
+        }
+        if (doubt) fixup_signs(Ss, ra, rl, row, need, sgn);
+      }
       if (inpad) {
         uint32_t* sd = reinterpret_cast<uint32_t*>(tb + KB * TILE * (DP / 8) + slot * (a.m / 8));
 #pragma unroll
