@@ -151,6 +151,30 @@ int tq_logits(const tq_params* p, const float* q, int n_q, int group, const void
               float* logits, void* workspace, int64_t workspace_bytes, tq_stream_t stream);
 
 /*
+ * tq_logits_noalloc - tq_logits without a caller-provided workspace.
+ * The pages have no counterpart: this is an interface for callers that cannot
+ * allocate device memory when they call (for example code that runs while a
+ * CUDA graph is being captured, or a plugin whose host framework owns every
+ * device buffer and passes only inputs and outputs).  Same arguments and
+ * results as tq_logits minus the workspace; the query-prep scratch is a
+ * static device array of tq_logits_noalloc_max_scratch() bytes (1 MiB) that
+ * every device loading the library keeps until the process exits.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make
+ *    that first call before any stream capture.
+ *  - Calls needing more scratch than the array (more than about 300 query
+ *    heads at d_pad 128) return TQ_EINVAL with a message; nothing is launched.
+ *  - All calls share the one array: calls that may overlap on the GPU (other
+ *    streams, other host threads) race and must be serialised by the caller.
+ *    The scratch is fully rewritten by each call, so nothing needs clearing.
+ *  - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
+ */
+int64_t tq_logits_noalloc_max_scratch(void);
+int tq_logits_noalloc(const tq_params* p, const float* q, int n_q, int group, const void* codes,
+                      const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys, int n_kv_heads,
+                      float* logits, tq_stream_t stream);
+
+/*
  * tq_decode_attn - one decode step of attention over compressed K (product
  * code) and V (MSE code) [E4][Z1 asymmetric K/V].
  *   q: device fp32 [batch][n_q_heads][d].  K/V vector index =

@@ -5,7 +5,7 @@ the library's CUDA kernels.  PyTorch supplies device memory and streams.
 The functions keep the C names; tensors are passed by device pointer.
 
 If libtq.so is missing this module raises at import: there is no fallback.
-Build it with ``python -m vector_quantization_randomized_b200.build``.
+Build it with ``python vector_quantization_randomized_b200/build.py``.
 """
 import ctypes
 import os
@@ -20,7 +20,7 @@ TQ_MODE_PROD, TQ_MODE_MSE = 0, 1
 TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} not found: build it with `python -m vector_quantization_randomized_b200.build`")
+    raise ImportError(f"{LIB_PATH} not found: build it with `python vector_quantization_randomized_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 
@@ -40,6 +40,8 @@ _SIGS = {
     "tq_quantize": (_i32, [_P, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp]),
     "tq_logits_workspace": (_i64, [_P, _i32]),
     "tq_logits": (_i32, [_P, _vp, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _i64, _vp]),
+    "tq_logits_noalloc_max_scratch": (_i64, []),
+    "tq_logits_noalloc": (_i32, [_P, _vp, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp]),
     "tq_decode_attn_workspace": (_i64, [_P, _i32, _i32, _i32, _i64]),
     "tq_decode_attn": (_i32, [_P, _P, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _f32, _vp,
                               _vp, _i64, _vp]),
@@ -159,6 +161,16 @@ def tq_logits(p, q, group, codes, norms, rnorms, n_keys, n_kv_heads, logits, wor
     return _check(_lib.tq_logits(p.ref, _ptr(q), q.shape[0], group, _ptr(codes), _ptr(norms), _ptr(rnorms),
                                  n_keys, n_kv_heads, _ptr(logits), _ptr(workspace), workspace.numel(),
                                  _stream(stream)))
+
+
+def tq_logits_noalloc_max_scratch():
+    return _lib.tq_logits_noalloc_max_scratch()
+
+
+def tq_logits_noalloc(p, q, group, codes, norms, rnorms, n_keys, n_kv_heads, logits, stream=None):
+    """tq_logits with the library's static device scratch instead of a caller workspace."""
+    return _check(_lib.tq_logits_noalloc(p.ref, _ptr(q), q.shape[0], group, _ptr(codes), _ptr(norms), _ptr(rnorms),
+                                         n_keys, n_kv_heads, _ptr(logits), _stream(stream)))
 
 
 def tq_decode_attn_workspace(kp, batch, n_q_heads, n_kv_heads, max_tokens):

@@ -1,6 +1,7 @@
 """Build the in-tree shared library libtq.so for B200 (sm_100a).
 
-Usage: python -m vector_quantization_randomized_b200.build [--force]
+Usage: python vector_quantization_randomized_b200/build.py [--force]
+(run as a script: importing the package first would load the existing library)
 """
 import glob
 import os

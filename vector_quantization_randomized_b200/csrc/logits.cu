@@ -13,6 +13,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 
 #include "common.h"
 #include "prep.h"
@@ -361,4 +362,68 @@ extern "C" int tq_logits(const tq_params* p, const float* q, int n_q, int group,
   }
   if (rc == TQ_OK) clear_error();
   return rc;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of tq_logits.
+//
+// Some callers cannot allocate device memory at call time: code running while
+// a CUDA graph is being captured, plugins hosted by a framework that owns every
+// device buffer and hands out only inputs and outputs, or runtimes whose device
+// heap is a fixed pool.  For them the query-prep scratch that tq_logits takes as
+// `workspace` lives in a static device array instead.  Every device that loads
+// the library holds this array until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t kNoAllocScratchBytes = int64_t(1) << 20;  // 1 MiB
+__device__ __align__(256) uint8_t g_logits_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device, looked up once per device.
+int scratch_on_current_device(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_logits_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return tq::set_error(TQ_EUNSUPPORTED, "tq_logits_noalloc: device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_logits_scratch);
+    if (e != cudaSuccess || !ptr)
+      return tq::set_error(TQ_ECUDA, "tq_logits_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" int64_t tq_logits_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
+
+extern "C" int tq_logits_noalloc(const tq_params* p, const float* q, int n_q, int group, const void* codes,
+                                 const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys, int n_kv_heads,
+                                 float* logits, tq_stream_t stream) {
+  using namespace tq;
+  int rc = check_params(p, "tq_logits_noalloc");
+  if (rc) return rc;
+  if (group < 1 || n_kv_heads < 1 || (int64_t)n_kv_heads * group != n_q)
+    return set_error(TQ_EINVAL, "tq_logits_noalloc: need n_q == n_kv_heads * group");
+  const int kb = index_bits(p);
+  const tqd::ScanShape sh(p->d_pad, kb, p->mode == TQ_MODE_PROD ? p->m : 0);
+  const int64_t need = (int64_t)n_kv_heads * ((group + tqd::QCHUNK - 1) / tqd::QCHUNK) * tqd::prep_chunk_bytes(sh.fr);
+  if (need > kNoAllocScratchBytes)
+    return set_error(TQ_EINVAL,
+                     "tq_logits_noalloc: %d query heads need %lld bytes of scratch, above the static %lld; "
+                     "use tq_logits with a caller-owned workspace",
+                     n_q, (long long)need, (long long)kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  rc = scratch_on_current_device(&scratch);
+  if (rc) return rc;
+  return tq_logits(p, q, n_q, group, codes, norms, rnorms, n_keys, n_kv_heads, logits, scratch,
+                   kNoAllocScratchBytes, stream);
 }
