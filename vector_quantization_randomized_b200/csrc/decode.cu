@@ -172,6 +172,171 @@ __global__ void __launch_bounds__(128) decode_kernel(const DArgs a) {
   }
 }
 
+// Staged variant (max_tokens a multiple of 32, 16-byte aligned norm arrays): the
+// chunk's K and V code tiles and its norms are copied to shared memory with
+// cp.async before any compute, so all of a CTA's HBM reads are in flight at
+// once; the scan and the value loop then read shared memory only.
+template <int KB, int SI, int VKB>
+constexpr int staged_smem() {
+  return (CH / TILE) * TILE * (KB * 16 + 16 * SI) + (CH / TILE) * TILE * (VKB * 16) + 3 * CH * 2 + QCHUNK * CH * 4;
+}
+
+template <int KB, int SI, int VKB>
+__global__ void __launch_bounds__(128) decode_staged_kernel(const DArgs a) {
+  constexpr int DP = 128;
+  using SC = Scan<DP, KB, SI>;
+  constexpr int SW = SI > 0 ? SI : 1;
+  constexpr int KTB = TILE * (KB * DP / 8 + 16 * SI);  // m == 128 * SI
+  constexpr int VTB = TILE * (VKB * DP / 8);
+  constexpr int NT = CH / TILE;
+  __shared__ float stat[QCHUNK][2];
+  __shared__ float vc[16];
+  __shared__ uint4 afrag[SC::FR / 4 * 32];
+  // dynamic: K tiles (later reused for the weights), V tiles, norms, scores
+  extern __shared__ __align__(16) uint8_t dsm[];
+  uint8_t* kbuf = dsm;
+  uint8_t* vbuf = dsm + NT * KTB;
+  __half (*nbuf)[CH] = reinterpret_cast<__half (*)[CH]>(vbuf + NT * VTB);  // K norms, K residual norms, V norms
+  float (*sl)[CH] = reinterpret_cast<float (*)[CH]>(vbuf + NT * VTB + 3 * CH * 2);
+  float4* wv = reinterpret_cast<float4*>(kbuf);  // written after the scan no longer reads kbuf
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int chunk_id = blockIdx.x % a.nch;
+  const int rest = blockIdx.x / a.nch;
+  const int qc = rest % a.nqc;
+  const int bg = rest / a.nqc;
+  const int b = bg / a.hkv;
+  const int L = (int)min((int64_t)a.seq_lens[b], a.max_tokens);
+  const int t0 = chunk_id * CH;
+  const int ntok = max(0, min(CH, L - t0));
+  const int64_t vbase = (int64_t)bg * a.max_tokens;
+  if (threadIdx.x < (1 << VKB)) vc[threadIdx.x] = a.vcent[threadIdx.x];
+
+  if (ntok > 0) {  // stage codes and norms (whole tiles; max_tokens % 32 == 0)
+    const int ntiles = (ntok + TILE - 1) / TILE;
+    const int64_t tile0 = (vbase + t0) / TILE;
+    const uint8_t* ks = a.kcodes + tile0 * KTB;
+    const uint8_t* vs = a.vcodes + tile0 * VTB;
+    for (int e = threadIdx.x; e < ntiles * KTB / 16; e += 128) cp_async16(kbuf + 16 * e, ks + 16 * e);
+    for (int e = threadIdx.x; e < ntiles * VTB / 16; e += 128) cp_async16(vbuf + 16 * e, vs + 16 * e);
+    const int nch16 = (ntok + 7) / 8;  // 16-byte chunks of 8 norms
+    for (int e = threadIdx.x; e < 3 * nch16; e += 128) {
+      const int arr = e / nch16, c = e % nch16;
+      const uint16_t* src = arr == 0 ? a.knorms : (arr == 1 ? a.krnorms : a.vnorms);
+      cp_async16(&nbuf[arr][8 * c], src + vbase + t0 + 8 * c);
+    }
+  }
+  cp_async_commit();
+  grid_dependency_wait();  // query prep (previous grid) complete
+  const uint8_t* prep = a.prep + (int64_t)(bg * a.nqc + qc) * a.prep_bytes;
+  if (ntok > 0) SC::stage(afrag, prep);
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // 1) logits of the chunk's tokens for the 4 query heads
+  if (ntok > 0) {
+    SC sc;
+    sc.load(reinterpret_cast<const uint8_t*>(afrag), lane);
+    const int g = lane >> 2, t = lane & 3;
+    const float4 qs = reinterpret_cast<const float4*>(prep + SC::FR * 128)[g & 3];
+    const int nsub = (ntok + 7) / 8;
+    for (int s = warp; s < nsub; s += 4) {
+      const int tk = 8 * s + g;
+      const uint8_t* tb = kbuf + (tk >> 5) * KTB;
+      const int slot = tk & 31;
+      uint32_t bw[KB][1], sw[SW];
+#pragma unroll
+      for (int p = 0; p < KB; ++p) bw[p][0] = reinterpret_cast<const uint32_t*>(tb + p * TILE * 16 + slot * 16)[t];
+#pragma unroll
+      for (int i = 0; i < SW; ++i)
+        sw[i] = SI ? reinterpret_cast<const uint32_t*>(tb + KB * TILE * 16 + slot * 16 * SI)[t + 4 * i] : 0u;
+      int accC[2][SC::NCSL][4] = {}, accS[2][4] = {}, accF[2][4];
+      sc.run(accC, accS, bw, sw);
+      SC::fold(accC, accF);
+      float c0, c1, z0 = 0.f, z1 = 0.f;
+      combine_digits(accF, lane, c0, c1);
+      if constexpr (SI > 0) combine_digits(accS, lane, z0, z1);
+      if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int tok = 8 * s + 2 * t + e;
+          float val = -INFINITY;
+          if (tok < ntok) {
+            const float n = __half2float(nbuf[0][tok]);
+            float l = fmaf(e ? c1 : c0, qs.x, -qs.y);
+            if constexpr (SI > 0) {
+              const float gm = __half2float(nbuf[1][tok]);
+              l = fmaf(gm * a.kappa, fmaf(e ? z1 : z0, qs.z, -qs.w), l);
+            }
+            val = n * l * a.sl2;
+          }
+          sl[g][tok] = val;
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // 2) softmax statistics per query (warp q), weights p * n_v
+  if (ntok > 0) {
+    const int qq = warp;
+    float mx = -INFINITY;
+    for (int j = lane; j < ntok; j += 32) mx = fmaxf(mx, sl[qq][j]);
+    mx = warp_max(mx);
+    float sum = 0.f;
+    for (int j = lane; j < ntok; j += 32) {
+      const float p = exp2f(sl[qq][j] - mx);
+      sl[qq][j] = p;
+      sum += p;
+    }
+    sum = warp_sum(sum);
+    if (lane == 0) {
+      stat[qq][0] = mx;
+      stat[qq][1] = sum;
+    }
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < ntok; j += 128) {
+    const float nv = __half2float(nbuf[2][j]);
+    wv[j] = make_float4(sl[0][j] * nv, sl[1][j] * nv, sl[2][j] * nv, sl[3][j] * nv);
+  }
+  __syncthreads();
+
+  // 3) value sum in the rotated domain: thread = coordinate c; words come from shared memory
+  const int c = threadIdx.x;
+  const int w = c >> 5, bit = c & 31;
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < ntok; ++j) {
+    const uint8_t* tb = vbuf + (j >> 5) * VTB + (j & 31) * 16;
+    int idx = 0;
+#pragma unroll
+    for (int p = 0; p < VKB; ++p) idx |= ((reinterpret_cast<const uint32_t*>(tb + p * TILE * 16)[w] >> bit) & 1u) << p;
+    const float cv = vc[idx];
+    const float4 ww = wv[j];
+    acc0 = fmaf(ww.x, cv, acc0);
+    acc1 = fmaf(ww.y, cv, acc1);
+    acc2 = fmaf(ww.z, cv, acc2);
+    acc3 = fmaf(ww.w, cv, acc3);
+  }
+
+  // 4) partials
+  const int hq0 = (bg % a.hkv) * a.group + QCHUNK * qc;
+  const int nq = min(QCHUNK, a.group - QCHUNK * qc);
+  const float accs[4] = {acc0, acc1, acc2, acc3};
+#pragma unroll
+  for (int qq = 0; qq < QCHUNK; ++qq) {
+    if (qq < nq) {
+      const int64_t h = (int64_t)b * (a.hkv * a.group) + hq0 + qq;
+      float* dst = a.part + (h * a.nch + chunk_id) * (DP + 2);
+      dst[c] = accs[qq];
+      if (c == 0) {
+        dst[DP] = ntok > 0 ? stat[qq][0] : -INFINITY;
+        dst[DP + 1] = ntok > 0 ? stat[qq][1] : 0.f;
+      }
+    }
+  }
+}
+
 struct CArgs {
   const float* part;
   const int8_t* vD;
@@ -235,7 +400,19 @@ int launch_decode(const DArgs& a, int blocks, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<KB, SI, VKB>, a);
+  const bool staged = (a.max_tokens % TILE) == 0 && a.km == 128 * SI && tq::aligned(a.knorms, 16) &&
+                      tq::aligned(a.krnorms, 16) && tq::aligned(a.vnorms, 16);
+  cudaError_t e;
+  if (staged) {
+    constexpr int smem = staged_smem<KB, SI, VKB>();
+    static_assert(smem >= CH * 16, "weights alias the K tiles");
+    e = cudaFuncSetAttribute(decode_staged_kernel<KB, SI, VKB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_decode_attn: %s", cudaGetErrorString(e));
+    cfg.dynamicSmemBytes = smem;
+    e = cudaLaunchKernelEx(&cfg, decode_staged_kernel<KB, SI, VKB>, a);
+  } else {
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<KB, SI, VKB>, a);
+  }
   if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_decode_attn: launch failed: %s", cudaGetErrorString(e));
   return TQ_OK;
 }
