@@ -205,27 +205,38 @@ __device__ __forceinline__ void encode_row(const uint8_t* xrow, int sw, int d, c
   g2 = acc.x + acc.y;
 }
 
-// Rare path: projections whose two-pass tensor-core value is within the
-// rounding bound of zero are recomputed in fp32 from the hi+lo residual parts
-// (2^-22 relative), and their sign bits overwritten.
-__device__ __noinline__ void fixup_signs(const uint8_t* Ss, const uint8_t* rh, const uint8_t* rl, int row,
-                                         const uint32_t (&need)[4], uint32_t (&sgn)[4]) {
-  for (int w = 0; w < 4; ++w) {
-    uint32_t nd = need[w];
-    while (nd) {
-      const int j = __ffs(nd) - 1;
-      nd &= nd - 1;
-      const int i = 32 * w + j;
-      float s = 0.f;
-      for (int k = 0; k < 64; ++k) {
-        const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(Ss + canon(i, 2 * k)));
-        const float2 h = __half22float2(*reinterpret_cast<const __half2*>(rh + canon(row, 2 * k)));
-        const float2 l = __half22float2(*reinterpret_cast<const __half2*>(rl + canon(row, 2 * k)));
-        s = fmaf(sf.x, h.x + l.x, s);
-        s = fmaf(sf.y, h.y + l.y, s);
+// Rare path, run by the whole warp: every projection whose two-pass
+// tensor-core value lies within the rounding bound of zero is recomputed in
+// fp32 from the hi+lo residual parts (2^-22 relative), four coordinates per
+// lane and a shuffle reduction, and the owning lane overwrites its sign bit.
+// `lanes` (warp-uniform) holds the lanes with at least one such projection.
+__device__ __forceinline__ void fixup_signs(const uint8_t* Ss, const uint8_t* rh, const uint8_t* rl, int row,
+                                         const uint32_t (&need)[4], uint32_t (&sgn)[4], uint32_t lanes) {
+  const int lane = threadIdx.x & 31;
+  while (lanes) {
+    const int src = __ffs(lanes) - 1;
+    lanes &= lanes - 1;
+    const int srow = __shfl_sync(FULL, row, src);
+    const uint2 hv = *reinterpret_cast<const uint2*>(rh + canon(srow, 4 * lane));
+    const uint2 lv = *reinterpret_cast<const uint2*>(rl + canon(srow, 4 * lane));
+    const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
+    const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+    const float2 l0 = __half22float2(*reinterpret_cast<const __half2*>(&lv.x));
+    const float2 l1 = __half22float2(*reinterpret_cast<const __half2*>(&lv.y));
+    const float r0 = h0.x + l0.x, r1 = h0.y + l0.y, r2 = h1.x + l1.x, r3 = h1.y + l1.y;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t nd = __shfl_sync(FULL, need[w], src);
+      while (nd) {
+        const int j = __ffs(nd) - 1;
+        nd &= nd - 1;
+        const uint2 sv = *reinterpret_cast<const uint2*>(Ss + canon(32 * w + j, 4 * lane));
+        const float2 s0 = __half22float2(*reinterpret_cast<const __half2*>(&sv.x));
+        const float2 s1 = __half22float2(*reinterpret_cast<const __half2*>(&sv.y));
+        float s = fmaf(s0.x, r0, fmaf(s0.y, r1, fmaf(s1.x, r2, s1.y * r3)));
+        s = warp_sum(s);
+        if (lane == src) sgn[w] = s >= 0.f ? (sgn[w] | (1u << j)) : (sgn[w] & ~(1u << j));
       }
-      if (s >= 0.f) sgn[w] |= 1u << j;
-      else sgn[w] &= ~(1u << j);
     }
   }
 }
@@ -237,7 +248,7 @@ __global__ void __launch_bounds__(NV, 1) quantize128_kernel(const Q2Args a) {
   uint8_t* Ss = smem + Lay::SS;
   uint8_t* Rs = smem + Lay::RS;
   uint32_t* dmask = reinterpret_cast<uint32_t*>(smem + Lay::DM);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lay::MISC);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lay::MISC);  // [0]: half 0 done, [2]: both halves
   uint32_t* tbase = reinterpret_cast<uint32_t*>(smem + Lay::MISC + 8);
   float* smax = reinterpret_cast<float*>(smem + Lay::MISC + 12);
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -259,7 +270,10 @@ __global__ void __launch_bounds__(NV, 1) quantize128_kernel(const Q2Args a) {
       *reinterpret_cast<uint4*>(Ss + canon(row, 8 * kc)) = v;
     }
     if (warp == 0) tmem_alloc(tbase, 256);
-    if (tid == 0) mbar_init(bar, 1);
+    if (tid == 0) {
+      mbar_init(bar, 1);
+      mbar_init(bar + 2, 1);
+    }
   }
   Coder<KB> cd;
   cd.init(a.thr, a.cent);
@@ -373,46 +387,49 @@ __global__ void __launch_bounds__(NV, 1) quantize128_kernel(const Q2Args a) {
               umma_f16(tmem + hf * 128, smem_desc(sA + ks * 256, lbo, sbo), smem_desc(sB + ks * 256, lbo, sbo),
                        idesc, (part | ks) ? 1u : 0u);
           }
+          if (hf == 0) umma_commit(bar);  // the first half's warps start reading while the second computes
         }
-        umma_commit(bar);
+        umma_commit(bar + 2);
       }
-      mbar_wait(bar, phase);
+      mbar_wait(bar + 2 * half, phase);
       phase ^= 1u;
       tc_fence_after();
       // read back this vector's projections: lane = row within its half, columns [half*128, half*128 + m)
       const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(half * 128);
-      uint32_t sgn[4] = {0, 0, 0, 0};
-      float zmin = INFINITY;
+      // two loads in flight per wait; sign bits and the doubt mask (|z| within the bound) in one sweep
+      uint32_t sgn[4] = {0, 0, 0, 0}, need[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        if (32 * w < a.m) {  // uniform: every lane of the warp executes the tcgen05.ld
-          float z[32];
-          tmem_ld32(taddr + 32 * w, z);
-          uint32_t word = 0;
+      for (int w2 = 0; w2 < 4; w2 += 2) {
+        uint32_t zr[2][32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (z[j] >= 0.f) word |= 1u << j;
-            zmin = fminf(zmin, fabsf(z[j]));
-          }
-          sgn[w] = word;
-        }
-      }
-      const bool doubt = valid && zmin <= bound;
-      if (__any_sync(FULL, doubt)) {  // rare, warp-uniform: find the doubtful projections
-        uint32_t need[4] = {0, 0, 0, 0};
-        for (int w = 0; w < 4; ++w) {
-          if (32 * w < a.m) {
-            float z[32];
-            tmem_ld32(taddr + 32 * w, z);
-            uint32_t nd = 0;
+        for (int u = 0; u < 2; ++u) {
+          if (32 * (w2 + u) < a.m) {  // uniform over the warp
+            tmem_ld32_issue(taddr + 32 * (w2 + u), zr[u]);
+          } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (fabsf(z[j]) <= bound) nd |= 1u << j;
-            need[w] = doubt ? nd : 0u;
+            for (int j = 0; j < 32; ++j) zr[u][j] = 0u;
           }
         }
-        if (doubt) fixup_signs(Ss, ra, rl, row, need, sgn);
+        tmem_ld_wait(zr[0]);
+        tmem_ld_wait(zr[1]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (32 * (w2 + u) < a.m) {
+            uint32_t word = 0, nd = 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float z = __uint_as_float(zr[u][j]);
+              if (z >= 0.f) word |= 1u << j;
+              if (fabsf(z) <= bound) nd |= 1u << j;
+            }
+            sgn[w2 + u] = word;
+            need[w2 + u] = valid ? nd : 0u;
+          }
+        }
       }
+      const bool doubt = (need[0] | need[1] | need[2] | need[3]) != 0u;
+      const uint32_t doubt_lanes = __ballot_sync(FULL, doubt);
+      if (doubt_lanes) fixup_signs(Ss, ra, rl, row, need, sgn, doubt_lanes);  // warp-uniform
       if (inpad) {
         uint32_t* sd = reinterpret_cast<uint32_t*>(tb + KB * TILE * (DP / 8) + slot * (a.m / 8));
 #pragma unroll
