@@ -58,6 +58,7 @@ typedef struct CUstream_st* tq_stream_t; /* same type as cudaStream_t */
 #define TQ_EINVAL (-1)        /* invalid argument (null, size, alignment) */
 #define TQ_EUNSUPPORTED (-2)  /* valid but not implemented for this shape */
 #define TQ_ECUDA (-3)         /* CUDA launch/runtime error; see tq_last_error */
+#define TQ_ETIMEOUT (-4)      /* a bounded device-side wait gave up (tq_device_status) */
 
 /* code modes */
 #define TQ_MODE_PROD 0 /* (bits-1)-bit Lloyd-Max code + m QJL sign bits [E1][E2][E3] */
@@ -208,6 +209,29 @@ int tq_search_topk(const tq_params* p, const float* q, int n_q, const void* code
                    const uint16_t* norms, const uint16_t* rnorms, int64_t n_db, int k,
                    int32_t* ids, float* scores, void* workspace, int64_t workspace_bytes,
                    tq_stream_t stream);
+
+/*
+ * tq_device_status - report (and optionally clear) device-side wait timeouts.
+ *   The tensor-core kernels hand data between their warps on shared-memory
+ *   barriers.  Every such wait has an iteration limit; a wait that reaches it
+ *   sets a device fault word of its kernel family and the kernel returns
+ *   early (its outputs are then undefined), so the context stays usable.
+ *   This call synchronizes the current device, reads every family's fault
+ *   word and returns TQ_OK if none is set, TQ_ETIMEOUT if one is (the
+ *   message names the families), TQ_ECUDA on a CUDA error.  clear != 0
+ *   resets the words.  The pages define no such call: it belongs to the
+ *   library's error handling, not to the method.
+ */
+int tq_device_status(int clear);
+
+/*
+ * tq_diag_bounded_wait - diagnostic: one CTA waits `polls` times on a
+ *   shared-memory barrier that nothing arrives at, then gives up the way the
+ *   kernels' waits do (fault word of the diagnostic family set, kernel
+ *   returns).  Lets a caller check, without any real failure, that timeouts
+ *   reach tq_device_status.  1 <= polls <= 2^20.  Asynchronous on `stream`.
+ */
+int tq_diag_bounded_wait(int64_t polls, tq_stream_t stream);
 
 /* Message for the last failed call on this thread ("" if none). */
 const char* tq_last_error(void);

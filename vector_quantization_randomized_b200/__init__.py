@@ -15,7 +15,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtq.so")
 
-TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECUDA = 0, -1, -2, -3
+TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECUDA, TQ_ETIMEOUT = 0, -1, -2, -3, -4
 TQ_MODE_PROD, TQ_MODE_MSE = 0, 1
 TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
 
@@ -47,6 +47,8 @@ _SIGS = {
                               _vp, _i64, _vp]),
     "tq_search_workspace": (_i64, [_P, _i32, _i64, _i32]),
     "tq_search_topk": (_i32, [_P, _vp, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _vp, _i64, _vp]),
+    "tq_device_status": (_i32, [_i32]),
+    "tq_diag_bounded_wait": (_i32, [_i64, _vp]),
     "tq_last_error": (ctypes.c_char_p, []),
     "tq_version": (_i32, []),
 }
@@ -89,6 +91,16 @@ def tq_last_error():
 
 def tq_version():
     return _lib.tq_version()
+
+
+def tq_device_status(clear=False):
+    """Synchronize the device; TQ_OK, or TQ_ETIMEOUT if a bounded device wait gave up (message in tq_last_error)."""
+    return _lib.tq_device_status(1 if clear else 0)
+
+
+def tq_diag_bounded_wait(polls, stream=None):
+    """Diagnostic: a kernel whose barrier wait runs out after `polls` polls (sets the diagnostic fault word)."""
+    return _check(_lib.tq_diag_bounded_wait(polls, _stream(stream)))
 
 
 def tq_make_codebook(d_pad, kb):

@@ -272,14 +272,20 @@ int dispatch_si(int si, const LArgs& a, int chunks, cudaStream_t st) {
 namespace tq {
 // Whether the register-fed scan supports this (d_pad, kb).
 bool scan_supported(int dp, int kb) { return (dp == 128 && kb >= 1 && kb <= 3) || (dp == 256 && kb >= 1 && kb <= 2); }
+
+int64_t prep_chunk_bytes_max(int dp, int kb, int m) {
+  const tqd::ScanShape sh(dp, kb, m);
+  int64_t b = tqd::prep_chunk_bytes(sh.fr);
+  if (dp == 128) b = std::max<int64_t>(b, tqd::prep_chunk_bytes_tc(tqd::tc_kchunks(kb, m)));
+  return b;
+}
 }  // namespace tq
 
 extern "C" int64_t tq_logits_workspace(const tq_params* p, int n_q) {
   if (!p || n_q < 0) return -1;
   const int kb = p->mode == TQ_MODE_PROD ? p->bits - 1 : p->bits;
   if (kb < 1 || kb > 4 || (p->d_pad != 128 && p->d_pad != 256)) return -1;
-  const tqd::ScanShape sh(p->d_pad, kb, p->mode == TQ_MODE_PROD ? p->m : 0);
-  return (int64_t)n_q * tqd::prep_chunk_bytes(sh.fr);
+  return (int64_t)n_q * tq::prep_chunk_bytes_max(p->d_pad, kb, p->mode == TQ_MODE_PROD ? p->m : 0);
 }
 
 extern "C" int tq_logits(const tq_params* p, const float* q, int n_q, int group, const void* codes,
@@ -308,7 +314,10 @@ extern "C" int tq_logits(const tq_params* p, const float* q, int n_q, int group,
   const tqd::ScanShape sh(p->d_pad, kb, m);
   const int nqc = (group + tqd::QCHUNK - 1) / tqd::QCHUNK;
   const int chunks = n_kv_heads * nqc;
-  const int64_t need = (int64_t)chunks * tqd::prep_chunk_bytes(sh.fr);
+  const bool tc = logits_tc_supported(p->d_pad, kb, m, group, n_keys, norms, rnorms);
+  const int kc = tqd::tc_kchunks(kb, m);
+  const int64_t chunk_bytes = tc ? tqd::prep_chunk_bytes_tc(kc) : tqd::prep_chunk_bytes(sh.fr);
+  const int64_t need = (int64_t)chunks * chunk_bytes;
   if (workspace_bytes < need)
     return set_error(TQ_EINVAL, "tq_logits: workspace too small (%lld < %lld bytes)", (long long)workspace_bytes,
                      (long long)need);
@@ -327,8 +336,15 @@ extern "C" int tq_logits(const tq_params* p, const float* q, int n_q, int group,
   pa.S = p->S;
   pa.out = static_cast<uint8_t*>(workspace);
   pa.fr = sh.fr;
+  pa.layout = tc ? 1 : 0;
+  pa.kc = kc;
   rc = launch_prep(pa, st);
   if (rc) return rc;
+  if (tc) {
+    rc = launch_logits_tc(kb, m, codes, norms, rnorms, n_keys, n_kv_heads, group, pa.out, chunk_bytes, logits, st);
+    if (rc == TQ_OK) clear_error();
+    return rc;
+  }
 
   LArgs a;
   a.codes = static_cast<const uint8_t*>(codes);
@@ -414,8 +430,8 @@ extern "C" int tq_logits_noalloc(const tq_params* p, const float* q, int n_q, in
   if (group < 1 || n_kv_heads < 1 || (int64_t)n_kv_heads * group != n_q)
     return set_error(TQ_EINVAL, "tq_logits_noalloc: need n_q == n_kv_heads * group");
   const int kb = index_bits(p);
-  const tqd::ScanShape sh(p->d_pad, kb, p->mode == TQ_MODE_PROD ? p->m : 0);
-  const int64_t need = (int64_t)n_kv_heads * ((group + tqd::QCHUNK - 1) / tqd::QCHUNK) * tqd::prep_chunk_bytes(sh.fr);
+  const int64_t need = (int64_t)n_kv_heads * ((group + tqd::QCHUNK - 1) / tqd::QCHUNK) *
+                       prep_chunk_bytes_max(p->d_pad, kb, p->mode == TQ_MODE_PROD ? p->m : 0);
   if (need > kNoAllocScratchBytes)
     return set_error(TQ_EINVAL,
                      "tq_logits_noalloc: %d query heads need %lld bytes of scratch, above the static %lld; "

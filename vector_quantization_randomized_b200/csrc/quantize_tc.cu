@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(NV, 1) quantize128_kernel(const Q2Args a) {
   uint8_t* Ss = smem + Lay::SS;
   uint8_t* Rs = smem + Lay::RS;
   uint32_t* dmask = reinterpret_cast<uint32_t*>(smem + Lay::DM);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lay::MISC);  // [0]: half 0 done, [2]: both halves
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lay::MISC);  // [0]: half 0 done, [2]: half 1 done
   uint32_t* tbase = reinterpret_cast<uint32_t*>(smem + Lay::MISC + 8);
   float* smax = reinterpret_cast<float*>(smem + Lay::MISC + 12);
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -387,9 +387,10 @@ __global__ void __launch_bounds__(NV, 1) quantize128_kernel(const Q2Args a) {
               umma_f16(tmem + hf * 128, smem_desc(sA + ks * 256, lbo, sbo), smem_desc(sB + ks * 256, lbo, sbo),
                        idesc, (part | ks) ? 1u : 0u);
           }
-          if (hf == 0) umma_commit(bar);  // the first half's warps start reading while the second computes
+          // these MMAs keep the tensor pipe busy (~64 cycles each), so one issuing thread
+          // suffices; committing per half lets the first half's warps read while the second computes
+          umma_commit(bar + 2 * hf);
         }
-        umma_commit(bar + 2);
       }
       mbar_wait(bar + 2 * half, phase);
       phase ^= 1u;
@@ -502,4 +503,16 @@ int launch_quantize128(const tq_params* p, const void* x, int dtype, int64_t n_v
   return prod ? dispatch_kb2<true, TQ_F16>(kb, a, smc, st) : dispatch_kb2<false, TQ_F16>(kb, a, smc, st);
 }
 
+}  // namespace tq
+
+namespace tq {
+// Read (and optionally clear) this translation unit's device fault word.
+int fault_word_quantize(int clear, int* value) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, tqd::g_fault, sizeof(int));
+  if (e == cudaSuccess && clear) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(tqd::g_fault, &zero, sizeof(int));
+  }
+  return e == cudaSuccess ? TQ_OK : set_error(TQ_ECUDA, "tq_device_status: %s", cudaGetErrorString(e));
+}
 }  // namespace tq
