@@ -20,10 +20,11 @@
 // Warp-specialised pipeline, one persistent CTA per SM over (KV head, 128-key
 // tile) items, all hand-offs on mbarriers (waits bounded):
 //   warp 0      bulk copies of the code tiles and norms into a ring of shared-memory stages;
-//   warps 1..NISS  tcgen05.mma issue, each every NISS-th K step into its own
-//               accumulator (one thread issues an MMA only every ~50 cycles, the
-//               tensor pipe finishes one in ~17); the first also loads the B
-//               image of each KV head (bulk copy);
+//   warps 1-4   tcgen05.mma issue: two pairs take alternate items, each warp of a
+//               pair every other K step into its own partial accumulator of a ring
+//               of accumulator sets (one thread issues an MMA only every ~50
+//               cycles and waits for them to be taken before its next item); the
+//               pair that meets a new KV head first loads its B image (bulk copy);
 //   8 warps     expansion: stage -> masked words -> tcgen05.st into one of two
 //               A buffers in tensor memory (warp = lane quadrant x 4 bit classes);
 //   8 warps     epilogue: tcgen05.ld of the partial accumulators, digit
@@ -72,18 +73,19 @@ struct TL {
   static constexpr int TILEB = 32 * 16 * (KB + SI);           // one 32-key code tile
   static constexpr int NORMB = 256 * (1 + SI);                // fp16 norms (+ residual norms) of 128 keys
   static constexpr int STAGE = 4 * TILEB + NORMB;             // one item: code tiles, then norms
-  // independent accumulators per item (K-step ks feeds ks % NACC): consecutive MMAs
-  // into one accumulator serialise on it, and at N = 32 there is too little work per
-  // MMA to hide that; the epilogue adds the partial sums (exact int32)
-  static constexpr int NACC = (512 - 2 * ACOLS) / 64 < 4 ? (512 - 2 * ACOLS) / 64 : 4;
+  // Two partial accumulators per item, one per MMA-issuing warp: a thread issues a
+  // tcgen05.mma only every ~50 cycles while the tensor pipe finishes one of these
+  // in ~17, so two warps issue in parallel (K steps j, j + 2, ...) and the epilogue
+  // adds the two partial sums (exact int32).  NB accumulator sets in a ring, so the
+  // MMAs of item i wait for the epilogue of item i - NB, not i - 2.
+  static constexpr int NACC = 2;
+  static constexpr int NISS = 2 * NACC;  // two pairs of issuing warps, alternate items
   static constexpr int COLS = 512;
-  static_assert(NACC >= 2 && 64 * NACC + 2 * ACOLS <= COLS, "tensor-memory budget");
-  // one MMA-issuing warp per accumulator: a thread issues a tcgen05.mma only every
-  // ~50 cycles, while the tensor pipe finishes one of these in ~17, so issue in parallel
-  static constexpr int NISS = NACC;
+  static constexpr int NB = (COLS - 2 * ACOLS) / (32 * NACC) < 4 ? (COLS - 2 * ACOLS) / (32 * NACC) : 4;
+  static_assert(NB >= 2 && 32 * NACC * NB + 2 * ACOLS <= COLS, "tensor-memory budget");
   static constexpr int W_EXP0 = 1 + NISS, W_EPI0 = W_EXP0 + 8;  // first expansion / epilogue warp
   static constexpr int NTHREADS = (W_EPI0 + 8) * 32;
-  static_assert(KSTEPS >= NISS, "every accumulator is written by each item");
+  static_assert(KSTEPS >= NACC, "every accumulator is written by each item");
   static constexpr int smem(int stages) { return HDR + BBYTES + stages * STAGE; }
 };
 
@@ -95,9 +97,10 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // [MAX_STAGES] stage loaded
   uint64_t* empty = full + MAX_STAGES;                  // [MAX_STAGES] stage read by the expansion and epilogue warps
   uint64_t* afull = empty + MAX_STAGES;                 // [2] A buffer written (8 arrivals)
-  uint64_t* mdone = afull + 2;                          // [2] MMA done: A buffer free, accumulator full
-  uint64_t* accfree = mdone + 2;                        // [2] accumulator read (8 arrivals)
-  uint64_t* bfull = accfree + 2;                        // B image loaded
+  uint64_t* mdone = afull + 2;                          // [2] MMAs of the item done: its A buffer is free
+  uint64_t* cfull = mdone + 2;                          // [4] MMAs done: accumulator set full
+  uint64_t* accfree = cfull + 4;                        // [4] accumulator set read (8 arrivals)
+  uint64_t* bfull = accfree + 4;                        // B image loaded
   uint32_t* tbase = reinterpret_cast<uint32_t*>(bfull + 1);
   uint8_t* Bsm = smem + HDR;
   uint8_t* ring = Bsm + L::BBYTES;
@@ -115,8 +118,11 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&afull[b], 8);
-      mbar_init(&mdone[b], L::NISS);
-      mbar_init(&accfree[b], 8);
+      mbar_init(&mdone[b], L::NACC);
+    }
+    for (int c = 0; c < 4; ++c) {
+      mbar_init(&cfull[c], L::NACC);
+      mbar_init(&accfree[c], 8);
     }
     mbar_init(bfull, 1);
   }
@@ -125,10 +131,10 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tbase;
-  // tensor-memory columns: accumulator set b = NACC x 32 columns from b * NACC * 32,
+  // tensor-memory columns: accumulator set c = NACC x 32 columns from c * NACC * 32,
   // then the two A buffers
-  auto acc_col = [&](int b, int k) { return tmem + (uint32_t)(32 * (b * L::NACC + k)); };
-  auto a_col = [&](int b) { return tmem + (uint32_t)(64 * L::NACC + b * L::ACOLS); };
+  auto acc_col = [&](int c, int k) { return tmem + (uint32_t)(32 * (c * L::NACC + k)); };
+  auto a_col = [&](int b) { return tmem + (uint32_t)(32 * L::NACC * L::NB + b * L::ACOLS); };
 
   if (warp == 0) {
     // ---------------- producer: code tiles into the ring ----------------
@@ -155,39 +161,51 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       for (int i = (issued > S ? issued - S : 0); i < issued; ++i) mbar_wait(&full[i % S], (i / S) & 1);
     }
   } else if (warp < W_EXP0) {
-    // ---------------- B image + MMA issue (NISS warps, one accumulator each) ----------------
-    const int j = warp - 1;
+    // ---------------- B image + MMA issue ----------------
+    // Two pairs of issuing warps take alternate items (pair p: items i with i % 2 == p),
+    // each warp of a pair every other K step into its own partial accumulator.  A
+    // thread cannot go on to its next item until the tensor core has taken its MMAs,
+    // so the other pair keeps the tensor pipe busy meanwhile.
+    const int j = warp - 1, par = j >> 1, k = j & 1;
     if (lane == 0) {
       grid_dependency_wait();  // the B image comes from the query-prep kernel
       constexpr uint32_t idesc = idesc_u8s8_s32(TK, 32);
       const uint32_t sB = smem_u32(Bsm);
       int64_t cur = -1, head = i0 / a.tiles_per_head;
       int t = (int)(i0 % a.tiles_per_head);
-      uint32_t bph = 0;
-      int done = 0;
-      for (int i = 0; i < n; ++i, ++t) {
+      uint32_t loads = 0, waited = 0;  // B images requested so far / waited for
+      int done = -1;
+      bool ok = true;
+      for (int i = 0, c = 0, cu = 0; i < n && ok; ++i, ++t, (++c == L::NB ? (c = 0, ++cu) : 0)) {
         const int b = i & 1;
         if (t == a.tiles_per_head) t = 0, ++head;
+        const bool mine = b == par;
         if (head != cur) {
-          if (j == 0) {  // issuer 0 reloads B once every issuer's MMAs on the old one are done
+          if (mine && k == 0) {  // reload B once no MMA of either pair still reads the old one
             if (i >= 1 && !mbar_wait(&mdone[(i - 1) & 1], ((i - 1) >> 1) & 1)) break;
+            if (i >= 2 && !mbar_wait(&mdone[i & 1], ((i - 2) >> 1) & 1)) break;
             mbar_expect_tx(bfull, L::BBYTES);
             bulk_g2s(Bsm, a.prep + head * a.prep_bytes, L::BBYTES, bfull);
           }
-          if (!mbar_wait(bfull, bph)) break;
-          bph ^= 1u;
+          ++loads;
           cur = head;
         }
+        if (!mine) continue;
+        if (waited != loads) {  // the latest B image (load number loads - 1) has landed
+          if (!mbar_wait(bfull, (loads - 1) & 1)) break;
+          waited = loads;
+        }
         if (!mbar_wait(&afull[b], (i >> 1) & 1)) break;
-        if (i >= 2 && !mbar_wait(&accfree[b], ((i >> 1) - 1) & 1)) break;
+        if (cu >= 1 && !mbar_wait(&accfree[c], (cu - 1) & 1)) break;
         tc_fence_after();
-        for (int ks = j; ks < L::KSTEPS; ks += L::NISS)
-          umma_i8_ts(acc_col(b, j), a_col(b) + 8 * ks, smem_desc(sB + ks * 256, 128, L::KC * 128), idesc,
-                     ks >= L::NISS ? 1u : 0u);
+        for (int ks = k; ks < L::KSTEPS; ks += 2)
+          umma_i8_ts(acc_col(c, k), a_col(b) + 8 * ks, smem_desc(sB + ks * 256, 128, L::KC * 128), idesc,
+                     ks >= 2 ? 1u : 0u);
         umma_commit(&mdone[b]);
-        done = i + 1;
+        umma_commit(&cfull[c]);
+        done = i;
       }
-      if (done > 0) mbar_wait(&mdone[(done - 1) & 1], ((done - 1) >> 1) & 1);  // no MMA left in flight
+      if (done >= 0) mbar_wait(&mdone[done & 1], (done >> 1) & 1);  // no MMA left in flight
     }
   } else if (warp < W_EPI0) {
     // ---------------- expansion: code bits -> A in tensor memory ----------------
@@ -238,8 +256,8 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
     int64_t cur = -1, head = i0 / a.tiles_per_head;
     int t = (int)(i0 % a.tiles_per_head);
     float4 sc[2] = {};
-    for (int i = 0, s = 0, use = 0; i < n; ++i, ++t, (++s == S ? (s = 0, ++use) : 0)) {
-      const int b = i & 1;
+    for (int i = 0, s = 0, use = 0, c = 0, cu = 0; i < n;
+         ++i, ++t, (++s == S ? (s = 0, ++use) : 0), (++c == L::NB ? (c = 0, ++cu) : 0)) {
       if (t == a.tiles_per_head) t = 0, ++head;
       if (head != cur) {
         const float4* qs = reinterpret_cast<const float4*>(a.prep + head * a.prep_bytes + L::BBYTES);
@@ -255,26 +273,19 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       const float gam = SI ? __half2float(nst[128 + 32 * qd + lane]) : 0.f;
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
-      if (!mbar_wait(&mdone[b], (i >> 1) & 1)) break;
+      if (!mbar_wait(&cfull[c], cu & 1)) break;
       tc_fence_after();
       uint32_t r[16], rp[16];
       const uint32_t lrow = ((uint32_t)(32 * qd) << 16) + 16 * qp;
-      tmem_ld16_issue(acc_col(b, 0) + lrow, r);
-      tmem_ld16_issue(acc_col(b, 1) + lrow, rp);
+      tmem_ld16_issue(acc_col(c, 0) + lrow, r);
+      tmem_ld16_issue(acc_col(c, 1) + lrow, rp);
       tmem_ld_wait16(r);
       tmem_ld_wait16(rp);
 #pragma unroll
       for (int e = 0; e < 16; ++e) r[e] += rp[e];  // exact: the full sums stay below 2^24
-#pragma unroll
-      for (int k = 2; k < L::NACC; ++k) {
-        tmem_ld16_issue(acc_col(b, k) + lrow, rp);
-        tmem_ld_wait16(rp);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] += rp[e];
-      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&accfree[b]);
+      if (lane == 0) mbar_arrive(&accfree[c]);
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int q = 2 * qp + j;
