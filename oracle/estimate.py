@@ -19,6 +19,10 @@ attention and top-k search (TEST INFRASTRUCTURE).
 * Decode attention: o = sum_j softmax_j(scale * l_j) v_hat_j with the
   maximum subtracted; scale defaults to 1/sqrt(d).  Plain token-by-token
   fp64; the GPU's chunked online softmax is a reassociation of this sum.
+* Sparse V (zhidx turboquant_plus article, "Sparse V": skip the value work of
+  tokens whose attention weight is negligible): a token with softmax weight
+  p_j < v_eps contributes no value; it stays in the normalisation, so
+  |o - o_full| <= v_eps * sum over skipped tokens of |v_hat_j|.
 * Search ("TurboQuant explainer", "向量搜索"): the k database ids with the
   largest estimate, ties to the lower id.
 
@@ -74,23 +78,33 @@ def dequant_mse(idx, norm_f16, centroids, D, d):
     return unrotate(y, D)[:, :d] * norm_f16.astype(np.float64)[:, None]
 
 
-def softmax_attend(logit_row, values, scale):
-    """o = sum_j p_j values_j with p = softmax(scale * logit_row), max subtracted."""
+def softmax_weights(logit_row, scale):
+    """p = softmax(scale * logit_row), maximum subtracted."""
     s = scale * np.asarray(logit_row, dtype=np.float64)
     s = s - np.max(s)
     p = np.exp(s)
-    p = p / np.sum(p)
+    return p / np.sum(p)
+
+
+def softmax_attend(logit_row, values, scale, v_eps=0.0):
+    """o = sum_j p_j values_j with p = softmax(scale * logit_row); with v_eps > 0
+    the tokens with p_j < v_eps add nothing (Sparse V), their weight stays in
+    the normalisation."""
+    p = softmax_weights(logit_row, scale)
+    if v_eps > 0.0:
+        p = np.where(p < v_eps, 0.0, p)
     return p @ values
 
 
 def decode_attention(q, kD, kS, k_idx, k_signs, k_norm, k_rnorm, k_cent, km,
                      vD, v_idx, v_norm, v_cent, d, seq_lens, Hq, Hkv, max_tokens,
-                     scale=0.0, pairs=None):
-    """tq_decode_attn semantics.
+                     scale=0.0, pairs=None, v_eps=0.0, bound=None):
+    """tq_decode_attn semantics (v_eps > 0: Sparse V, as softmax_attend).
 
     q [B, Hq, d]; key/value vector index = (b*Hkv + g)*max_tokens + t.
     Returns out [B, Hq, d] (fp64); rows not in `pairs` (list of (b, h)) are NaN
-    when `pairs` is given.
+    when `pairs` is given.  If `bound` is an array [B, Hq] it receives
+    v_eps * sum_{p_j < v_eps} |v_hat_j|, the largest change Sparse V can make.
     """
     B = q.shape[0]
     group = Hq // Hkv
@@ -112,7 +126,10 @@ def decode_attention(q, kD, kS, k_idx, k_signs, k_norm, k_rnorm, k_cent, km,
         key = (b, g)
         if key not in cache:
             cache[key] = dequant_mse(v_idx[sl], v_norm[sl], v_cent, vD, d)
-        out[b, h] = softmax_attend(lg, cache[key], scale)
+        out[b, h] = softmax_attend(lg, cache[key], scale, v_eps)
+        if bound is not None:
+            p = softmax_weights(lg, scale)
+            bound[b, h] = v_eps * np.sum(np.linalg.norm(cache[key][p < v_eps], axis=1))
     return out
 
 
