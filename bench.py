@@ -438,6 +438,22 @@ def run_secondary(args, world, rank, local, torch, tq, wl):
                 "ms_per_step": ms, "config": {"workload": "decode-64x8x16384-Kprod3-Vmse3-hq32"},
                 "metric_bytes": mbytes, "gbs": round(gbs, 1), "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4),
                 "frac_measured": round(gbs / peak, 4)}
+        # Sparse V: same step, tokens whose attention weight is below v_eps add no value
+        sparse = {}
+        for eps in (1e-4, 1e-3):
+            run_s = lambda: tq.tq_decode_attn_sparse(kp, vp, q, Hkv, bufs["k"][0], bufs["k"][1], bufs["k"][2],
+                                                     bufs["v"][0], bufs["v"][1], sl, T, out, ws, v_eps=eps)
+            for _ in range(args.warmup):
+                run_s()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(args.steps):
+                run_s()
+            e1.record()
+            torch.cuda.synchronize()
+            ms_s = e0.elapsed_time(e1) / args.steps
+            sparse[f"v_eps={eps:g}"] = {"ms_per_step": round(ms_s, 4), "tokens_per_s": n / (ms_s / 1e3)}
+        line["sparse_v"] = sparse
     elif args.workload == "quantize":
         n, d = 1 << 20, 128
         x = gpu_kv(torch, 1, 8, n // 8, d, wl.SEED_KEYS)

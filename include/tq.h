@@ -197,6 +197,24 @@ int tq_decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int
                    void* workspace, int64_t workspace_bytes, tq_stream_t stream);
 
 /*
+ * tq_decode_attn_sparse - tq_decode_attn with Sparse V [Z1 "Sparse V": skip
+ *   the value work of tokens whose attention weight is negligible].  Same
+ *   arguments plus v_eps >= 0.  Inside each 512-token split of a sequence, a
+ *   token is dropped when its weight within the split, p_t / (split sum), is
+ *   below v_eps for every query head sharing the KV head; since that bounds its
+ *   final softmax weight from above, only tokens with final weight < v_eps are
+ *   dropped.  A dropped token adds no value but keeps its weight in the
+ *   normalisation, so |out - out_full| <= v_eps * sum over tokens with weight
+ *   < v_eps of |v_hat_t|.  v_eps = 0 gives exactly tq_decode_attn's result.
+ *   Returns TQ_EINVAL for negative or non-finite v_eps.
+ */
+int tq_decode_attn_sparse(const tq_params* kp, const tq_params* vp, const float* q, int batch,
+                          int n_q_heads, int n_kv_heads, const void* kcodes, const uint16_t* knorms,
+                          const uint16_t* krnorms, const void* vcodes, const uint16_t* vnorms,
+                          const int32_t* seq_lens, int64_t max_tokens, float scale, float v_eps,
+                          float* out, void* workspace, int64_t workspace_bytes, tq_stream_t stream);
+
+/*
  * tq_search_topk - top-k inner-product search over quantized vectors [E5].
  *   q: device fp32 [n_q][d]; codes/norms/rnorms: n_db vectors.
  *   ids: device int32 [n_q][k], scores: device fp32 [n_q][k]: the k largest

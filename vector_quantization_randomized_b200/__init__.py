@@ -45,6 +45,8 @@ _SIGS = {
     "tq_decode_attn_workspace": (_i64, [_P, _i32, _i32, _i32, _i64]),
     "tq_decode_attn": (_i32, [_P, _P, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _f32, _vp,
                               _vp, _i64, _vp]),
+    "tq_decode_attn_sparse": (_i32, [_P, _P, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _f32,
+                                     _f32, _vp, _vp, _i64, _vp]),
     "tq_search_workspace": (_i64, [_P, _i32, _i64, _i32]),
     "tq_search_topk": (_i32, [_P, _vp, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _vp, _i64, _vp]),
     "tq_device_status": (_i32, [_i32]),
@@ -196,6 +198,16 @@ def tq_decode_attn(kp, vp, q, n_kv_heads, kcodes, knorms, krnorms, vcodes, vnorm
                                       _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), _ptr(seq_lens),
                                       max_tokens, scale, _ptr(out), _ptr(workspace), workspace.numel(),
                                       _stream(stream)))
+
+
+def tq_decode_attn_sparse(kp, vp, q, n_kv_heads, kcodes, knorms, krnorms, vcodes, vnorms, seq_lens, max_tokens,
+                          out, workspace, v_eps, scale=0.0, stream=None):
+    """tq_decode_attn with Sparse V: tokens whose attention weight is below v_eps add no value."""
+    batch, n_q_heads = q.shape[0], q.shape[1]
+    return _check(_lib.tq_decode_attn_sparse(kp.ref, vp.ref, _ptr(q), batch, n_q_heads, n_kv_heads, _ptr(kcodes),
+                                             _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), _ptr(seq_lens),
+                                             max_tokens, scale, v_eps, _ptr(out), _ptr(workspace),
+                                             workspace.numel(), _stream(stream)))
 
 
 def tq_search_workspace(p, n_q, n_db, k):

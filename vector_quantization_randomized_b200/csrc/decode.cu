@@ -41,7 +41,27 @@ struct DArgs {
   int64_t prep_bytes;
   float* part;  // [b][h][chunk][dp + 2]
   float kappa, sl2;  // sqrt(pi/2)/m, scale*log2(e)
+  float veps;        // Sparse V threshold (0: off)
 };
+
+// Value weights p_j * n_v,j of token j for the 4 query heads of the chunk.
+// Sparse V ("zhidx turboquant_plus article", "Sparse V": skip the value work of
+// tokens with negligible attention weight): with veps > 0 the token is dropped
+// when p_j < veps * (chunk sum of p) for every query head of the chunk.  The
+// chunk-normalised weight bounds the final softmax weight from above (the other
+// chunks only add to the denominator), so a dropped token has final weight
+// below veps; its weight stays in the normalisation.
+__device__ __forceinline__ float4 value_weights(const float (*sl)[CH], const float (*stat)[2], int j, float nv,
+                                                float veps, int nq) {
+  float4 w = make_float4(sl[0][j] * nv, sl[1][j] * nv, sl[2][j] * nv, sl[3][j] * nv);
+  if (veps > 0.f) {
+    bool keep = false;
+#pragma unroll
+    for (int qq = 0; qq < QCHUNK; ++qq) keep |= qq < nq && sl[qq][j] >= veps * stat[qq][1];
+    if (!keep) w = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  return w;
+}
 
 template <int KB, int SI, int VKB>
 __global__ void __launch_bounds__(128) decode_kernel(const DArgs a) {
@@ -129,7 +149,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const DArgs a) {
   __syncthreads();
   for (int j = threadIdx.x; j < ntok; j += 128) {
     const float nv = __half2float(__ushort_as_half(a.vnorms[vbase + t0 + j]));
-    wv[j] = make_float4(sl[0][j] * nv, sl[1][j] * nv, sl[2][j] * nv, sl[3][j] * nv);
+    wv[j] = value_weights(sl, stat, j, nv, a.veps, min(QCHUNK, a.group - QCHUNK * qc));
   }
   __syncthreads();
 
@@ -137,7 +157,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const DArgs a) {
   const int c = threadIdx.x;  // DP == blockDim.x
   float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
   const int w = c >> 5, bit = c & 31;
-  for (int j = 0; j < ntok; ++j) {
+  auto vstep = [&](int j, const float4 ww) {
     const int64_t v = vbase + t0 + j;
     const uint8_t* tbase = a.vcodes + (v >> 5) * a.vtb + (int)(v & 31) * (DP / 8);
     int idx = 0;
@@ -147,11 +167,18 @@ __global__ void __launch_bounds__(128) decode_kernel(const DArgs a) {
       idx |= ((word >> bit) & 1u) << p;
     }
     const float cv = vc[idx];
-    const float4 ww = wv[j];
     acc0 = fmaf(ww.x, cv, acc0);
     acc1 = fmaf(ww.y, cv, acc1);
     acc2 = fmaf(ww.z, cv, acc2);
     acc3 = fmaf(ww.w, cv, acc3);
+  };
+  if (a.veps > 0.f) {  // Sparse V: dropped tokens (all four weights zero) are skipped, uniformly over the CTA
+    for (int j = 0; j < ntok; ++j) {
+      const float4 ww = wv[j];
+      if (ww.x != 0.f || ww.y != 0.f || ww.z != 0.f || ww.w != 0.f) vstep(j, ww);
+    }
+  } else {
+    for (int j = 0; j < ntok; ++j) vstep(j, wv[j]);
   }
 
   // 4) partials: [b][h][chunk][dp + 2] = (o_rot[0..dp), max (log2 units), sum)
@@ -297,7 +324,7 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const DArgs a) {
   __syncthreads();
   for (int j = threadIdx.x; j < ntok; j += 128) {
     const float nv = __half2float(nbuf[2][j]);
-    wv[j] = make_float4(sl[0][j] * nv, sl[1][j] * nv, sl[2][j] * nv, sl[3][j] * nv);
+    wv[j] = value_weights(sl, stat, j, nv, a.veps, min(QCHUNK, a.group - QCHUNK * qc));
   }
   __syncthreads();
 
@@ -305,18 +332,25 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const DArgs a) {
   const int c = threadIdx.x;
   const int w = c >> 5, bit = c & 31;
   float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll 4
-  for (int j = 0; j < ntok; ++j) {
+  auto vstep = [&](int j, const float4 ww) {
     const uint8_t* tb = vbuf + (j >> 5) * VTB + (j & 31) * 16;
     int idx = 0;
 #pragma unroll
     for (int p = 0; p < VKB; ++p) idx |= ((reinterpret_cast<const uint32_t*>(tb + p * TILE * 16)[w] >> bit) & 1u) << p;
     const float cv = vc[idx];
-    const float4 ww = wv[j];
     acc0 = fmaf(ww.x, cv, acc0);
     acc1 = fmaf(ww.y, cv, acc1);
     acc2 = fmaf(ww.z, cv, acc2);
     acc3 = fmaf(ww.w, cv, acc3);
+  };
+  if (a.veps > 0.f) {  // Sparse V: dropped tokens (all four weights zero) are skipped, uniformly over the CTA
+    for (int j = 0; j < ntok; ++j) {
+      const float4 ww = wv[j];
+      if (ww.x != 0.f || ww.y != 0.f || ww.z != 0.f || ww.w != 0.f) vstep(j, ww);
+    }
+  } else {
+#pragma unroll 4
+    for (int j = 0; j < ntok; ++j) vstep(j, wv[j]);
   }
 
   // 4) partials
@@ -447,11 +481,11 @@ extern "C" int64_t tq_decode_attn_workspace(const tq_params* kp, int batch, int 
   return prep + decode_ws_parts(batch, n_q_heads, max_tokens);
 }
 
-extern "C" int tq_decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int batch, int n_q_heads,
-                              int n_kv_heads, const void* kcodes, const uint16_t* knorms, const uint16_t* krnorms,
-                              const void* vcodes, const uint16_t* vnorms, const int32_t* seq_lens,
-                              int64_t max_tokens, float scale, float* out, void* workspace,
-                              int64_t workspace_bytes, tq_stream_t stream) {
+namespace {
+int decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int batch, int n_q_heads, int n_kv_heads,
+                const void* kcodes, const uint16_t* knorms, const uint16_t* krnorms, const void* vcodes,
+                const uint16_t* vnorms, const int32_t* seq_lens, int64_t max_tokens, float scale, float v_eps,
+                float* out, void* workspace, int64_t workspace_bytes, tq_stream_t stream) {
   using namespace tq;
   int rc = check_params(kp, "tq_decode_attn(kp)");
   if (rc) return rc;
@@ -526,6 +560,7 @@ extern "C" int tq_decode_attn(const tq_params* kp, const tq_params* vp, const fl
   a.kappa = (float)(std::sqrt(M_PI / 2.0) / kp->m);
   const float sc = scale != 0.f ? scale : (float)(1.0 / std::sqrt((double)kp->d));
   a.sl2 = sc * 1.4426950408889634f;
+  a.veps = v_eps;
   const int64_t blocks64 = (int64_t)batch * n_kv_heads * nqc * nch;
   if (blocks64 > 0x7fffffff) return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: grid too large");
   const int blocks = (int)blocks64;
@@ -550,4 +585,25 @@ extern "C" int tq_decode_attn(const tq_params* kp, const tq_params* vp, const fl
   if (e != cudaSuccess) return set_error(TQ_ECUDA, "tq_decode_attn: combine launch failed: %s", cudaGetErrorString(e));
   clear_error();
   return TQ_OK;
+}
+}  // namespace
+
+extern "C" int tq_decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int batch, int n_q_heads,
+                              int n_kv_heads, const void* kcodes, const uint16_t* knorms, const uint16_t* krnorms,
+                              const void* vcodes, const uint16_t* vnorms, const int32_t* seq_lens,
+                              int64_t max_tokens, float scale, float* out, void* workspace,
+                              int64_t workspace_bytes, tq_stream_t stream) {
+  return decode_attn(kp, vp, q, batch, n_q_heads, n_kv_heads, kcodes, knorms, krnorms, vcodes, vnorms, seq_lens,
+                     max_tokens, scale, 0.f, out, workspace, workspace_bytes, stream);
+}
+
+extern "C" int tq_decode_attn_sparse(const tq_params* kp, const tq_params* vp, const float* q, int batch,
+                                     int n_q_heads, int n_kv_heads, const void* kcodes, const uint16_t* knorms,
+                                     const uint16_t* krnorms, const void* vcodes, const uint16_t* vnorms,
+                                     const int32_t* seq_lens, int64_t max_tokens, float scale, float v_eps,
+                                     float* out, void* workspace, int64_t workspace_bytes, tq_stream_t stream) {
+  if (!(v_eps >= 0.f) || !std::isfinite(v_eps))
+    return tq::set_error(TQ_EINVAL, "tq_decode_attn_sparse: v_eps must be finite and >= 0");
+  return decode_attn(kp, vp, q, batch, n_q_heads, n_kv_heads, kcodes, knorms, krnorms, vcodes, vnorms, seq_lens,
+                     max_tokens, scale, v_eps, out, workspace, workspace_bytes, stream);
 }
