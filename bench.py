@@ -120,7 +120,9 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- distributed
-def dist_setup(args):
+def dist_setup(args=None):
+    """One process per GPU (RANK/LOCAL_RANK/WORLD_SIZE/MASTER_* from the launcher).
+    NCCL on GPUs; gloo where there is no GPU (the host-side plumbing, tested on CPU)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -128,9 +130,12 @@ def dist_setup(args):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -143,13 +148,21 @@ def barrier(world):
 
 
 def allmax(world, v):
+    """Maximum of v over the ranks (every rank takes part, in the same order)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(world, units_per_rank, max_ms):
+    """Whole-job throughput: every rank processes units_per_rank; the job takes
+    the slowest rank's time."""
+    return world * units_per_rank / (max_ms / 1e3)
 
 
 # --------------------------------------------------------------------------- workloads
@@ -573,7 +586,7 @@ def main():
     clocks = sampler.stop()
     ms = statistics.mean(step_ms)
     ms_max = allmax(world, sum(step_ms)) / args.steps
-    value = world * wk.keys_per_step() / (ms_max / 1e3)
+    value = weak_scaling_value(world, wk.keys_per_step(), ms_max)
 
     # dominant API call in the step and its roofline
     kinds = {}
@@ -609,7 +622,7 @@ def main():
     if not args.no_e2e:
         e_ms, h2d, d2h = time_e2e(torch, wk, max(3, args.steps // 2), 2)
         e_ms = allmax(world, e_ms)
-        e2e = {"value": world * wk.keys_per_step() / (e_ms / 1e3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": weak_scaling_value(world, wk.keys_per_step(), e_ms), "unit": "keys/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
