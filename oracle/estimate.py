@@ -16,6 +16,8 @@ attention and top-k search (TEST INFRASTRUCTURE).
 * MSE-only values ("TurboQuant explainer", "速度" - logits from compressed KV;
   zhidx turboquant_plus article - asymmetric K/V):
       v_hat = n * D o (H c[idx]) / sqrt(d_pad), first d coordinates.
+* Product-code reconstruction (the map Q^-1 of "第二步：QJL"):
+      x_hat = n * D o (H (c[idx] + sqrt(pi/2)/m * gamma * S^T (2s-1))) / sqrt(d_pad).
 * Decode attention: o = sum_j softmax_j(scale * l_j) v_hat_j with the
   maximum subtracted; scale defaults to 1/sqrt(d).  Plain token-by-token
   fp64; the GPU's chunked online softmax is a reassociation of this sum.
@@ -76,6 +78,20 @@ def dequant_mse(idx, norm_f16, centroids, D, d):
     """v_hat rows [n, d] (fp64) from MSE-only codes."""
     y = np.asarray(centroids, dtype=np.float64)[idx]
     return unrotate(y, D)[:, :d] * norm_f16.astype(np.float64)[:, None]
+
+
+def dequant_prod(idx, signs, norm_f16, rnorm_f16, centroids, D, S, m, d):
+    """x_hat rows [n, d] (fp64) from product codes: the inverse map Q^-1 of
+    "TurboQuant explainer" (m.163.com), "第二步：QJL" (the QJL part is
+    r_hat = sqrt(pi/2)/m * gamma * S^T sigma with sigma = 2s - 1, so that
+    E[<y, Q^-1(Q(x))>] = <y, x>), added to the Lloyd-Max centroids in the
+    rotated domain and rotated back:
+        x_hat = n * D H (c[idx] + r_hat) / sqrt(d_pad), first d coordinates.
+    <q, x_hat> is exactly the logit estimate of `logits_from_codes` (linearity)."""
+    y = np.asarray(centroids, dtype=np.float64)[idx]
+    sigma = 2.0 * np.asarray(signs, dtype=np.float64) - 1.0                # [n, m]
+    r_hat = (np.sqrt(np.pi / 2.0) / m) * rnorm_f16.astype(np.float64)[:, None] * (sigma @ np.asarray(S, dtype=np.float64))
+    return unrotate(y + r_hat, D)[:, :d] * norm_f16.astype(np.float64)[:, None]
 
 
 def softmax_weights(logit_row, scale):
