@@ -135,6 +135,24 @@ int tq_quantize(const tq_params* p, const void* x, int dtype, int64_t n_vec, int
                 void* codes, uint16_t* norms, uint16_t* rnorms, tq_stream_t stream);
 
 /*
+ * tq_dequantize - the reconstruction x_hat = Q^-1(codes) [E2: the QJL part is
+ *   sqrt(pi/2)/m * gamma * S^T sigma, sigma = 2s - 1, which makes
+ *   E[<y, Q^-1(Q(x))>] = <y, x>]:
+ *     product mode  x_hat = n D H (c[idx] + sqrt(pi/2)/m * gamma * S^T sigma) / sqrt(d_pad)
+ *     MSE mode      x_hat = n D H c[idx] / sqrt(d_pad)
+ *   first d coordinates.  <q, x_hat> equals the tq_logits estimate for every q
+ *   (the estimate is linear in the key).  Re-encoding stored tokens at a lower
+ *   bit width (temporal decay [Z1]) is tq_dequantize followed by tq_quantize
+ *   with the lower-width parameters.
+ *   codes, norms, rnorms: as written by tq_quantize for n_vec vectors (rnorms
+ *   NULL in MSE mode).  out: device fp32 [n_vec][ld], ld >= d; columns d..ld-1
+ *   are not written.  codes 16-byte aligned.
+ */
+int tq_dequantize(const tq_params* p, const void* codes, const uint16_t* norms,
+                  const uint16_t* rnorms, int64_t n_vec, float* out, int64_t ld,
+                  tq_stream_t stream);
+
+/*
  * tq_logits - attention logits straight from the codes [E2][E4].
  *   q: device fp32 [n_q][d], n_q = n_kv_heads*group; query head h reads KV
  *      head h/group (GQA).

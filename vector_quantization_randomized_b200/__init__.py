@@ -38,6 +38,7 @@ _SIGS = {
     "tq_make_params": (_i32, [_i32, _i32, _u64, _vp, _vp]),
     "tq_code_bytes": (_i64, [_i32, _i32, _i32, _i64]),
     "tq_quantize": (_i32, [_P, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "tq_dequantize": (_i32, [_P, _vp, _vp, _vp, _i64, _vp, _i64, _vp]),
     "tq_logits_workspace": (_i64, [_P, _i32]),
     "tq_logits": (_i32, [_P, _vp, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _i64, _vp]),
     "tq_logits_noalloc_max_scratch": (_i64, []),
@@ -165,6 +166,13 @@ def tq_quantize(p, x, codes, norms, rnorms=None, n_vec=None, ld=None, stream=Non
     ld = x.stride(0) if ld is None else ld
     return _check(_lib.tq_quantize(p.ref, _ptr(x), _dtype_code(x), n_vec, ld, _ptr(codes), _ptr(norms),
                                    _ptr(rnorms), _stream(stream)))
+
+
+def tq_dequantize(p, codes, norms, rnorms, n_vec, out, ld=None, stream=None):
+    """Reconstruction x_hat = Q^-1(codes) into out (device fp32 [n_vec, ld])."""
+    ld = out.stride(0) if ld is None else ld
+    return _check(_lib.tq_dequantize(p.ref, _ptr(codes), _ptr(norms), _ptr(rnorms), n_vec, _ptr(out), ld,
+                                     _stream(stream)))
 
 
 def tq_logits_workspace(p, n_q):
