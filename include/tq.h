@@ -170,6 +170,19 @@ int tq_logits(const tq_params* p, const float* q, int n_q, int group, const void
               float* logits, void* workspace, int64_t workspace_bytes, tq_stream_t stream);
 
 /*
+ * tq_logits_ld - tq_logits writing row h of the logits at logits + h*ld_logits
+ *   (ld_logits >= n_keys; columns past n_keys untouched).  Mixed bit widths
+ *   along a sequence (older tokens re-encoded at a lower width, temporal decay
+ *   [Z1]) are scanned with one call per width segment into one logits matrix:
+ *   segment k's call gets its own parameters and codes, n_keys = the segment's
+ *   length, logits + (segment start) and ld_logits = the whole length.
+ */
+int tq_logits_ld(const tq_params* p, const float* q, int n_q, int group, const void* codes,
+                 const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys, int n_kv_heads,
+                 float* logits, int64_t ld_logits, void* workspace, int64_t workspace_bytes,
+                 tq_stream_t stream);
+
+/*
  * tq_logits_noalloc - tq_logits without a caller-provided workspace.
  * The pages have no counterpart: this is an interface for callers that cannot
  * allocate device memory when they call (for example code that runs while a

@@ -41,6 +41,7 @@ _SIGS = {
     "tq_dequantize": (_i32, [_P, _vp, _vp, _vp, _i64, _vp, _i64, _vp]),
     "tq_logits_workspace": (_i64, [_P, _i32]),
     "tq_logits": (_i32, [_P, _vp, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _i64, _vp]),
+    "tq_logits_ld": (_i32, [_P, _vp, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _i64, _vp, _i64, _vp]),
     "tq_logits_noalloc_max_scratch": (_i64, []),
     "tq_logits_noalloc": (_i32, [_P, _vp, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp]),
     "tq_decode_attn_workspace": (_i64, [_P, _i32, _i32, _i32, _i64]),
@@ -183,6 +184,13 @@ def tq_logits(p, q, group, codes, norms, rnorms, n_keys, n_kv_heads, logits, wor
     return _check(_lib.tq_logits(p.ref, _ptr(q), q.shape[0], group, _ptr(codes), _ptr(norms), _ptr(rnorms),
                                  n_keys, n_kv_heads, _ptr(logits), _ptr(workspace), workspace.numel(),
                                  _stream(stream)))
+
+
+def tq_logits_ld(p, q, group, codes, norms, rnorms, n_keys, n_kv_heads, logits, ld_logits, workspace, stream=None):
+    """tq_logits writing query row h at logits + h*ld_logits (pass a column-offset view for a segment)."""
+    return _check(_lib.tq_logits_ld(p.ref, _ptr(q), q.shape[0], group, _ptr(codes), _ptr(norms), _ptr(rnorms),
+                                    n_keys, n_kv_heads, _ptr(logits), ld_logits, _ptr(workspace), workspace.numel(),
+                                    _stream(stream)))
 
 
 def tq_logits_noalloc_max_scratch():

@@ -31,6 +31,7 @@ struct LArgs {
   const uint8_t* prep;
   int64_t prep_bytes;
   float* logits;
+  int64_t ld;  // logits row stride (>= n_keys)
   float kappa;
 };
 
@@ -51,7 +52,7 @@ __global__ void __launch_bounds__(128) logits_kernel(const LArgs a) {
   const int64_t s_begin = (int64_t)split * per;
   const int64_t s_end = min(n_sub, s_begin + per);
   const int64_t vbase = (int64_t)head * a.n_keys;
-  float* out = a.logits + ((int64_t)head * a.group + qrow) * a.n_keys;
+  float* out = a.logits + ((int64_t)head * a.group + qrow) * a.ld;
 
   // first code words do not depend on the query prep: fetch them before waiting for it
   uint32_t bw[KB][NH], sw[SW];
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(128) logits_ring_kernel(const LArgs a) {
   const int64_t s_begin = (int64_t)split * per;
   const int64_t s_end = min(n_sub, s_begin + per);
   const int64_t vbase = (int64_t)head * a.n_keys;
-  float* out = a.logits + ((int64_t)head * a.group + qrow) * a.n_keys;
+  float* out = a.logits + ((int64_t)head * a.group + qrow) * a.ld;
   const int sbytes = a.m / 8;  // sign bytes per key
   const int n_sign_cp = SI ? (8 * sbytes) / 16 : 0;
   const int n_cp = KB * 8 + n_sign_cp + 2;
@@ -288,12 +289,14 @@ extern "C" int64_t tq_logits_workspace(const tq_params* p, int n_q) {
   return (int64_t)n_q * tq::prep_chunk_bytes_max(p->d_pad, kb, p->mode == TQ_MODE_PROD ? p->m : 0);
 }
 
-extern "C" int tq_logits(const tq_params* p, const float* q, int n_q, int group, const void* codes,
-                         const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys, int n_kv_heads,
-                         float* logits, void* workspace, int64_t workspace_bytes, tq_stream_t stream) {
+extern "C" int tq_logits_ld(const tq_params* p, const float* q, int n_q, int group, const void* codes,
+                            const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys, int n_kv_heads,
+                            float* logits, int64_t ld_logits, void* workspace, int64_t workspace_bytes,
+                            tq_stream_t stream) {
   using namespace tq;
   int rc = check_params(p, "tq_logits");
   if (rc) return rc;
+  if (ld_logits < n_keys) return set_error(TQ_EINVAL, "tq_logits: ld_logits < n_keys");
   const int kb = index_bits(p);
   const bool prod = p->mode == TQ_MODE_PROD;
   if (!scan_supported(p->d_pad, kb))
@@ -341,7 +344,8 @@ extern "C" int tq_logits(const tq_params* p, const float* q, int n_q, int group,
   rc = launch_prep(pa, st);
   if (rc) return rc;
   if (tc) {
-    rc = launch_logits_tc(kb, m, codes, norms, rnorms, n_keys, n_kv_heads, group, pa.out, chunk_bytes, logits, st);
+    rc = launch_logits_tc(kb, m, codes, norms, rnorms, n_keys, n_kv_heads, group, pa.out, chunk_bytes, logits,
+                          ld_logits, st);
     if (rc == TQ_OK) clear_error();
     return rc;
   }
@@ -358,6 +362,7 @@ extern "C" int tq_logits(const tq_params* p, const float* q, int n_q, int group,
   a.prep = pa.out;
   a.prep_bytes = tqd::prep_chunk_bytes(sh.fr);
   a.logits = logits;
+  a.ld = ld_logits;
   a.kappa = (float)(std::sqrt(M_PI / 2.0) / (m > 0 ? m : 1));
   // about four 128-thread CTAs per SM, each with at least 16 subtiles per warp
   const int64_t n_sub = (n_keys + 7) / 8;
@@ -378,6 +383,13 @@ extern "C" int tq_logits(const tq_params* p, const float* q, int n_q, int group,
   }
   if (rc == TQ_OK) clear_error();
   return rc;
+}
+
+extern "C" int tq_logits(const tq_params* p, const float* q, int n_q, int group, const void* codes,
+                         const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys, int n_kv_heads,
+                         float* logits, void* workspace, int64_t workspace_bytes, tq_stream_t stream) {
+  return tq_logits_ld(p, q, n_q, group, codes, norms, rnorms, n_keys, n_kv_heads, logits, n_keys, workspace,
+                      workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------

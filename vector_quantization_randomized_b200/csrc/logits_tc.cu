@@ -58,6 +58,7 @@ struct TArgs {
   const uint8_t* prep;   // per KV head: B image + per-query scalars
   int64_t prep_bytes;
   float* logits;
+  int64_t ld;            // logits row stride
   float kappa;           // sqrt(pi/2) / m
   int stages;            // ring stages (<= MAX_STAGES)
 };
@@ -301,7 +302,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
                                        fmaf((float)(int)r[8 * j + 5], 256.f, (float)(int)r[8 * j + 4])));
             l = fmaf(gam * a.kappa, fmaf(sg, sc[j].z, -sc[j].w), l);
           }
-          a.logits[(head * a.group + q) * a.n_keys + key] = nrm * l;
+          a.logits[(head * a.group + q) * a.ld + key] = nrm * l;
         }
       }
     }
@@ -350,7 +351,7 @@ bool logits_tc_supported(int dp, int kb, int m, int group, int64_t n_keys, const
 // Scan with the query-prep output `prep` (layout 1, one chunk per KV head).
 int launch_logits_tc(int kb, int m, const void* codes, const uint16_t* norms, const uint16_t* rnorms,
                      int64_t n_keys, int n_kv_heads, int group, const uint8_t* prep, int64_t prep_bytes,
-                     float* logits, cudaStream_t st) {
+                     float* logits, int64_t ld, cudaStream_t st) {
   TArgs a;
   a.codes = static_cast<const uint8_t*>(codes);
   a.norms = norms;
@@ -363,6 +364,7 @@ int launch_logits_tc(int kb, int m, const void* codes, const uint16_t* norms, co
   a.prep = prep;
   a.prep_bytes = prep_bytes;
   a.logits = logits;
+  a.ld = ld;
   a.kappa = (float)(std::sqrt(M_PI / 2.0) / (m > 0 ? m : 1));
   a.stages = MAX_STAGES;
   const int sm = sm_count();

@@ -16,7 +16,7 @@ int sm_count();
 bool logits_tc_supported(int dp, int kb, int m, int group, int64_t n_keys, const void* norms, const void* rnorms);
 int launch_logits_tc(int kb, int m, const void* codes, const uint16_t* norms, const uint16_t* rnorms,
                      int64_t n_keys, int n_kv_heads, int group, const uint8_t* prep, int64_t prep_bytes,
-                     float* logits, cudaStream_t st);
+                     float* logits, int64_t ld, cudaStream_t st);
 // Bytes of query-prep scratch per chunk of 4 queries, the larger of both layouts.
 int64_t prep_chunk_bytes_max(int dp, int kb, int m);
 }  // namespace tq
