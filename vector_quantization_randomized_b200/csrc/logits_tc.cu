@@ -25,8 +25,8 @@
 //               of accumulator sets (one thread issues an MMA only every ~50
 //               cycles and waits for them to be taken before its next item); the
 //               pair that meets a new KV head first loads its B image (bulk copy);
-//   8 warps     expansion: stage -> masked words -> tcgen05.st into one of two
-//               A buffers in tensor memory (warp = lane quadrant x 4 bit classes);
+//   8 warps     expansion: stage -> masked words -> tcgen05.st into one of two or
+//               three A buffers in tensor memory (warp = lane quadrant x 4 bit classes);
 //   8 warps     epilogue: tcgen05.ld of the partial accumulators, digit
 //               combination, norms, logits (warp = lane quadrant x 2 queries).
 #include <cuda_runtime.h>
@@ -82,8 +82,11 @@ struct TL {
   static constexpr int NACC = 2;
   static constexpr int NISS = 2 * NACC;  // two pairs of issuing warps, alternate items
   static constexpr int COLS = 512;
-  static constexpr int NB = (COLS - 2 * ACOLS) / (32 * NACC) < 4 ? (COLS - 2 * ACOLS) / (32 * NACC) : 4;
-  static_assert(NB >= 2 && 32 * NACC * NB + 2 * ACOLS <= COLS, "tensor-memory budget");
+  // A buffers: three where they fit beside three accumulator sets (b <= 3), else two;
+  // the expansion of item i then waits for the MMAs of item i - NA
+  static constexpr int NA = 3 * ACOLS + 3 * 32 * NACC <= COLS ? 3 : 2;
+  static constexpr int NB = (COLS - NA * ACOLS) / (32 * NACC) < 4 ? (COLS - NA * ACOLS) / (32 * NACC) : 4;
+  static_assert(NB >= 2 && 32 * NACC * NB + NA * ACOLS <= COLS, "tensor-memory budget");
   static constexpr int W_EXP0 = 1 + NISS, W_EPI0 = W_EXP0 + 8;  // first expansion / epilogue warp
   static constexpr int NTHREADS = (W_EPI0 + 8) * 32;
   static_assert(KSTEPS >= NACC, "every accumulator is written by each item");
@@ -97,9 +100,9 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // [MAX_STAGES] stage loaded
   uint64_t* empty = full + MAX_STAGES;                  // [MAX_STAGES] stage read by the expansion and epilogue warps
-  uint64_t* afull = empty + MAX_STAGES;                 // [2] A buffer written (8 arrivals)
-  uint64_t* mdone = afull + 2;                          // [2] MMAs of the item done: its A buffer is free
-  uint64_t* cfull = mdone + 2;                          // [4] MMAs done: accumulator set full
+  uint64_t* afull = empty + MAX_STAGES;                 // [3] A buffer written (8 arrivals)
+  uint64_t* mdone = afull + 3;                          // [3] MMAs of the item done: its A buffer is free
+  uint64_t* cfull = mdone + 3;                          // [4] MMAs done: accumulator set full
   uint64_t* accfree = cfull + 4;                        // [4] accumulator set read (8 arrivals)
   uint64_t* bfull = accfree + 4;                        // B image loaded
   uint32_t* tbase = reinterpret_cast<uint32_t*>(bfull + 1);
@@ -117,7 +120,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 16);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&afull[b], 8);
       mbar_init(&mdone[b], L::NACC);
     }
@@ -178,13 +181,13 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       int done = -1;
       bool ok = true;
       for (int i = 0, c = 0, cu = 0; i < n && ok; ++i, ++t, (++c == L::NB ? (c = 0, ++cu) : 0)) {
-        const int b = i & 1;
+        const int b = i % L::NA, ua = i / L::NA;  // A buffer and its use count
         if (t == a.tiles_per_head) t = 0, ++head;
-        const bool mine = b == par;
+        const bool mine = (i & 1) == par;
         if (head != cur) {
           if (mine && k == 0) {  // reload B once no MMA of either pair still reads the old one
-            if (i >= 1 && !mbar_wait(&mdone[(i - 1) & 1], ((i - 1) >> 1) & 1)) break;
-            if (i >= 2 && !mbar_wait(&mdone[i & 1], ((i - 2) >> 1) & 1)) break;
+            if (i >= 1 && !mbar_wait(&mdone[(i - 1) % L::NA], ((i - 1) / L::NA) & 1)) break;
+            if (i >= 2 && !mbar_wait(&mdone[(i - 2) % L::NA], ((i - 2) / L::NA) & 1)) break;
             mbar_expect_tx(bfull, L::BBYTES);
             bulk_g2s(Bsm, a.prep + head * a.prep_bytes, L::BBYTES, bfull);
           }
@@ -196,7 +199,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
           if (!mbar_wait(bfull, (loads - 1) & 1)) break;
           waited = loads;
         }
-        if (!mbar_wait(&afull[b], (i >> 1) & 1)) break;
+        if (!mbar_wait(&afull[b], ua & 1)) break;
         if (cu >= 1 && !mbar_wait(&accfree[c], (cu - 1) & 1)) break;
         tc_fence_after();
         for (int ks = k; ks < L::KSTEPS; ks += 2)
@@ -206,7 +209,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
         umma_commit(&cfull[c]);
         done = i;
       }
-      if (done >= 0) mbar_wait(&mdone[done & 1], (done >> 1) & 1);  // no MMA left in flight
+      if (done >= 0) mbar_wait(&mdone[done % L::NA], (done / L::NA) & 1);  // no MMA left in flight
     }
   } else if (warp < W_EPI0) {
     // ---------------- expansion: code bits -> A in tensor memory ----------------
@@ -214,9 +217,9 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
     const int qd = warp & 3;   // tensor-memory lane quadrant = 32-key code tile within the item
     const int cg = ew >> 2;    // bit classes 4cg .. 4cg+3
     for (int i = 0, s = 0, use = 0; i < n; ++i, (++s == S ? (s = 0, ++use) : 0)) {
-      const int b = i & 1;
+      const int b = i % L::NA, ua = i / L::NA;
       if (!mbar_wait(&full[s], use & 1)) break;
-      if (i >= 2 && !mbar_wait(&mdone[b], ((i >> 1) - 1) & 1)) break;  // MMA of item i-2 has read A[b]
+      if (ua >= 1 && !mbar_wait(&mdone[b], (ua - 1) & 1)) break;  // MMAs of item i - NA have read A[b]
       const uint8_t* st = ring + s * L::STAGE + qd * L::TILEB + lane * 16;
       uint4 pw[KB + SI];
 #pragma unroll

@@ -247,6 +247,19 @@ __global__ void __launch_bounds__(256) qprep_kernel(const PrepArgs a) {
   }
 }
 
+// frexpf's exponent (x = f 2^e, 0.5 <= f < 1) and ldexpf(1, k), read from / written
+// into the fp32 bit pattern for normal values (exact), the library calls otherwise.
+__device__ __forceinline__ int frexp_exponent(float x) {
+  const uint32_t b = __float_as_uint(x) & 0x7FFFFFFFu;
+  if (b >= 0x00800000u && b < 0x7F800000u) return (int)(b >> 23) - 126;
+  int e;
+  frexpf(x, &e);
+  return e;
+}
+__device__ __forceinline__ float pow2f(int k) {
+  return (k >= -126 && k <= 127) ? __uint_as_float((uint32_t)(127 + k) << 23) : ldexpf(1.f, k);
+}
+
 // Query prep for the tensor-memory scan (d_pad 128): one CTA of 512 threads per
 // chunk of 4 queries writes the B image of layout 1 (scan.cuh) and the per-query
 // scalars.  Same integer weights as qprep_kernel: X = round(2 alpha_T q_rot_j 2^F)
@@ -282,7 +295,8 @@ __global__ void __launch_bounds__(512) qprep_tc_kernel(const PrepArgs a) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) sv[k] = __ldg(srow + k);
   }
-  if (tid < L) cent_s[tid] = __ldg(a.cent + tid);
+  // the centroid load stays in flight while the query warps rotate
+  const float cent_r = tid < L ? __ldg(a.cent + tid) : 0.f;
   if (warp < QCHUNK) {  // q_rot = H D q / sqrt(128): warp = query, lane holds coordinates lane + 32 i
     const int qi = warp;
     const bool valid = QCHUNK * qc + qi < a.group;
@@ -324,6 +338,7 @@ __global__ void __launch_bounds__(512) qprep_tc_kernel(const PrepArgs a) {
       qstat[qi][1] = mx;
     }
   }
+  if (tid < L) cent_s[tid] = cent_r;
   __syncthreads();
   if (tid < NT) {  // Walsh coefficients of the odd-symmetric codebook (fp64)
     const int mask = walsh_mask(a.kb, tid);
@@ -372,59 +387,49 @@ __global__ void __launch_bounds__(512) qprep_tc_kernel(const PrepArgs a) {
     mu = warp_max(mu);
     float amax = 0.f;
     for (int T = 0; T < NT; ++T) amax = fmaxf(amax, fabsf(alpha[T]));
-    int F = 0, G = 0;
     const float mc = 2.f * amax * qstat[qi][1], ms = 2.f * mu;
-    if (mc > 0.f) {
-      int e;
-      frexpf(mc, &e);
-      F = 23 - e;
-    }
-    if (ms > 0.f) {
-      int e;
-      frexpf(ms, &e);
-      G = 23 - e;
-    }
+    const int F = mc > 0.f ? 23 - frexp_exponent(mc) : 0;
+    const int G = ms > 0.f ? 23 - frexp_exponent(ms) : 0;
     if (lane == 0) {
-      FGs[qi][0] = ldexpf(1.f, F);
-      FGs[qi][1] = ldexpf(1.f, G);
+      FGs[qi][0] = pow2f(F);
+      FGs[qi][1] = pow2f(G);
       float4* scal = reinterpret_cast<float4*>(a.out + (int64_t)chunk * prep_chunk_bytes_tc(KC) + (int64_t)KC * 512);
       // sum_T alpha_T = c[L-1] (all index bits set)
-      scal[qi] = make_float4(ldexpf(1.f, -(F + 7)), cent_s[L - 1] * qstat[qi][0], ldexpf(1.f, -(G + 7)), su);
+      scal[qi] = make_float4(pow2f(-(F + 7)), cent_s[L - 1] * qstat[qi][0], pow2f(-(G + 7)), su);
     }
   }
   __syncthreads();
-  // B image rows, one thread per (query q, plane P, bit class c): the 16 weights of
-  // coordinates 32w + 8b + c (byte 4w + b of K chunk 8P + c) give the 4 digit rows
-  // 8q + r0 + d (r0 = 0 centroid, 4 sign); the other 4 rows of the chunk are zero.
-  // Scaling by the power of two 2^F (2^G) is exact, as in ldexpf.
-  if (tid < QCHUNK * NP * 8) {
-    const int c = tid & 7, pq = tid >> 3;
+  // B image words, one thread per (query q, plane P, bit class c, word w): the 4
+  // weights of coordinates 32w + 8b + c (bytes 4w + b of K chunk 8P + c) give word
+  // w of the 4 digit rows 8q + r0 + d (r0 = 0 centroid, 4 sign); the same word of
+  // the chunk's other 4 rows is zero.  Scaling by the power of two 2^F (2^G) is
+  // exact, as in ldexpf.
+  for (int e = tid; e < QCHUNK * NP * 32; e += 512) {
+    const int w = e & 3, c = (e >> 2) & 7, pq = e >> 5;
     const int q = pq / NP, P = pq - q * NP;
     const bool cen = P < NT;
     const float scale = cen ? 2.f * alpha[P] * FGs[q][0] : 2.f * FGs[q][1];
     const float* src = cen ? qTf : uTf;
-    uint32_t W[4][4] = {};
+    uint32_t W[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int w = 0; w < 4; ++w)
+    for (int b = 0; b < 4; ++b) {
+      const int j = 32 * w + 8 * b + c;
+      int X = (cen || j < a.m) ? __float2int_rn(src[4 * j + q] * scale) * (1 << (7 - c)) : 0;
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int j = 32 * w + 8 * b + c;
-        int X = (cen || j < a.m) ? __float2int_rn(src[4 * j + q] * scale) * (1 << (7 - c)) : 0;
-#pragma unroll
-        for (int d = 0; d < 3; ++d) {
-          const int lowb = (int)(int8_t)(X & 0xFF);
-          W[d][w] |= (uint32_t)(uint8_t)lowb << (8 * b);
-          X = (X - lowb) >> 8;
-        }
-        W[3][w] |= (uint32_t)(uint8_t)X << (8 * b);
+      for (int d = 0; d < 3; ++d) {
+        const int lowb = (int)(int8_t)(X & 0xFF);
+        W[d] |= (uint32_t)(uint8_t)lowb << (8 * b);
+        X = (X - lowb) >> 8;
       }
-    uint4* dst = reinterpret_cast<uint4*>(a.out + (int64_t)chunk * prep_chunk_bytes_tc(KC) + q * (KC * 128) +
-                                          (8 * P + c) * 128);
+      W[3] |= (uint32_t)(uint8_t)X << (8 * b);
+    }
+    uint32_t* dst = reinterpret_cast<uint32_t*>(a.out + (int64_t)chunk * prep_chunk_bytes_tc(KC) + q * (KC * 128) +
+                                                (8 * P + c) * 128) + w;
     const int r0 = cen ? 0 : 4;
 #pragma unroll
     for (int d = 0; d < 4; ++d) {
-      dst[r0 + d] = make_uint4(W[d][0], W[d][1], W[d][2], W[d][3]);
-      dst[(r0 ^ 4) + d] = make_uint4(0, 0, 0, 0);
+      dst[4 * (r0 + d)] = W[d];
+      dst[4 * ((r0 ^ 4) + d)] = 0u;
     }
   }
 }

@@ -68,7 +68,7 @@ struct Lay {
   static constexpr int RS = SS + 128 * DP * 2;    // residuals (hi part) fp16, canonical, two 128-row halves
   static constexpr int RL = RS + NV * DP * 2;     // residuals (lo part), same layout
   static constexpr int DM = RL + NV * DP * 2;     // sign-flip masks, 64 x uint32 (bits 15, 31)
-  static constexpr int MISC = DM + 64 * 4;        // mbarrier, tmem base, max ||S_i||
+  static constexpr int MISC = DM + 64 * 4;        // mbarriers (+0, +16), tmem base (+8), max ||S_i|| (+12), 8 floats (+32)
   static constexpr int TOTAL = MISC + 64;
 };
 
@@ -293,18 +293,31 @@ __global__ void __launch_bounds__(NV, 1) quantize128_kernel(const Q2Args a) {
   if (tile < n_tiles) issue(tile);
   __syncthreads();
   if constexpr (PROD) {
-    if (warp == 0) {  // max_i ||S_i|| (slightly inflated so the bound stays a bound)
-      float mx = 0.f;
-      for (int row = tid; row < a.m; row += 32) {
-        float s = 0.f;
-        for (int k = 0; k < DP; ++k) {
-          const float v = __half2float(*reinterpret_cast<const __half*>(Ss + canon(row, k)));
-          s = fmaf(v, v, s);
+    // max_i ||S_i|| (slightly inflated so the bound stays a bound): two threads per
+    // row, 16-byte reads of the canonical layout, then a block-wide maximum
+    float s = 0.f;
+    if (tid < 2 * a.m) {
+      const int row = tid >> 1, k0 = (tid & 1) * (DP / 2);
+#pragma unroll 4
+      for (int k = k0; k < k0 + DP / 2; k += 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(Ss + canon(row, k));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[h]));
+          s = fmaf(f.x, f.x, fmaf(f.y, f.y, s));
         }
-        mx = fmaxf(mx, s);
       }
-      mx = warp_max(mx);
-      if (tid == 0) *smax = sqrtf(mx) * 1.0001f;
+    }
+    s += __shfl_xor_sync(FULL, s, 1);  // the row's two halves
+    const float wmx = warp_max(s);
+    float* wmax = reinterpret_cast<float*>(smem + Lay::MISC + 32);  // 8 floats after the barriers
+    if ((tid & 31) == 0) wmax[warp] = wmx;
+    __syncthreads();
+    if (tid == 0) {
+      float mx = 0.f;
+      for (int w = 0; w < NV / 32; ++w) mx = fmaxf(mx, wmax[w]);
+      *smax = sqrtf(mx) * 1.0001f;
     }
     tc_fence_before();
     __syncthreads();
