@@ -60,8 +60,11 @@ def measured_peaks():
 
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock/throttle sampling around the timed region: sampling runs
+    every 20 ms from before the warm-up (start() waits for the first sample) to
+    after the timing; stop() keeps the samples within 150 ms of the timed window
+    (set by window()), or the nearest sample on each side if none falls inside."""
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -75,6 +78,7 @@ class ClockSampler:
             pass
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
@@ -82,10 +86,16 @@ class ClockSampler:
             os.close(fd)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
+            deadline = time.time() + 5.0
+            while time.time() < deadline and os.path.getsize(self.path) == 0:
+                time.sleep(0.02)
         except Exception:
             self.proc = None
+
+    def window(self, t0, t1):
+        self.t0, self.t1 = t0, t1
 
     def stop(self):
         if self.proc is None:
@@ -102,13 +112,22 @@ class ClockSampler:
             if len(parts) < 9:
                 continue
             try:
-                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), hw=parts[5], hwt=parts[6],
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                rows.append(dict(t=ts, sm=float(parts[1]), smax=float(parts[2]), hw=parts[5], hwt=parts[6],
                                  swt=parts[7], swp=parts[8]))
-            except ValueError:
+            except (ValueError, IndexError):
                 continue
         os.unlink(self.path)
         if not rows:
             return None
+        if self.t0 is not None:
+            inside = [r for r in rows if self.t0 - 0.15 <= r["t"] <= self.t1 + 0.15]
+            if not inside:
+                before = [r for r in rows if r["t"] < self.t0]
+                after = [r for r in rows if r["t"] > self.t1]
+                inside = before[-1:] + after[:1]
+            rows = inside or rows
         reasons = set()
         for r in rows:
             for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
@@ -242,7 +261,7 @@ def l2_flush(torch, buf):
     buf.zero_()
 
 
-def time_steps(torch, wk, steps, warmup, world, flush):
+def time_steps(torch, wk, steps, warmup, world, flush, sampler=None):
     """Device-timed steps: per-step and per-call CUDA events on the launching stream."""
     calls = wk.calls()
     for _ in range(warmup):
@@ -252,6 +271,7 @@ def time_steps(torch, wk, steps, warmup, world, flush):
     barrier(world)
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
+    t_wall0 = time.time()
     for s in range(steps):
         l2_flush(torch, flush)
         ev[s][0].record()
@@ -259,7 +279,10 @@ def time_steps(torch, wk, steps, warmup, world, flush):
             f()
             ev[s][i + 1].record()
     torch.cuda.synchronize()
+    t_wall1 = time.time()
     barrier(world)
+    if sampler is not None:
+        sampler.window(t_wall0, t_wall1)
     step_ms = [ev[s][0].elapsed_time(ev[s][-1]) for s in range(steps)]
     per_call = {}
     for i, (label, _) in enumerate(calls):
@@ -582,7 +605,7 @@ def main():
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
     sampler = ClockSampler(local)
     sampler.start()
-    step_ms, per_call = time_steps(torch, wk, args.steps, args.warmup, world, flush)
+    step_ms, per_call = time_steps(torch, wk, args.steps, args.warmup, world, flush, sampler)
     clocks = sampler.stop()
     ms = statistics.mean(step_ms)
     ms_max = allmax(world, sum(step_ms)) / args.steps
