@@ -216,16 +216,17 @@ class Layer:
                 ws=torch.empty(tq.tq_logits_workspace(kp, self.q.shape[0]), dtype=torch.uint8, device=dev))
         self.launches_per_step = len(self.BITS) * 4   # quantize K, quantize V, logits prep + scan
 
-    def calls(self):
-        """The step as a list of (label, callable)."""
+    def calls(self, inputs=None):
+        """The step as a list of (label, callable); `inputs` = (K, V, q) device tensors (default: the layer's)."""
         tq = self.tq
+        K, V, q = inputs if inputs is not None else (self.K, self.V, self.q)
         out = []
         for b in self.BITS:
             B = self.bufs[b]
             kp, vp = self.kp[b], self.vp[b]
-            out.append((f"tq_quantize_K_b{b}", lambda kp=kp, B=B: tq.tq_quantize(kp, self.K, B["kc"], B["kn"], B["krn"])))
-            out.append((f"tq_quantize_V_b{b}", lambda vp=vp, B=B: tq.tq_quantize(vp, self.V, B["vc"], B["vn"])))
-            out.append((f"tq_logits_b{b}", lambda kp=kp, B=B: tq.tq_logits(kp, self.q, self.GROUP, B["kc"], B["kn"],
+            out.append((f"tq_quantize_K_b{b}", lambda kp=kp, B=B: tq.tq_quantize(kp, K, B["kc"], B["kn"], B["krn"])))
+            out.append((f"tq_quantize_V_b{b}", lambda vp=vp, B=B: tq.tq_quantize(vp, V, B["vc"], B["vn"])))
+            out.append((f"tq_logits_b{b}", lambda kp=kp, B=B: tq.tq_logits(kp, q, self.GROUP, B["kc"], B["kn"],
                                                                            B["krn"], self.T, self.H_KV, B["lg"],
                                                                            B["ws"])))
         return out
@@ -291,28 +292,49 @@ def time_steps(torch, wk, steps, warmup, world, flush, sampler=None):
 
 
 def time_e2e(torch, wk, steps, warmup):
-    """Same step through the public API with pinned host buffers: H2D inputs, step, D2H results."""
+    """Same step through the public API with pinned host buffers: every step copies
+    its inputs host -> device and reads its logits back device -> host, all inside
+    the timed region.  The next step's inputs are uploaded on a second stream into
+    the other of two device input sets while the current step computes (events
+    order each copy before its step and after the step that last read that set)."""
     hin = [t.cpu().pin_memory() for t in wk.host_inputs()]
     hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in wk.host_outputs()]
-    din, dout = wk.host_inputs(), wk.host_outputs()
-    calls = wk.calls()
+    dsets = [wk.host_inputs(), [torch.empty_like(t) for t in wk.host_inputs()]]
+    dout = wk.host_outputs()
+    calls = [wk.calls(tuple(ds)) for ds in dsets]
+    comp = torch.cuda.current_stream()
+    copy = torch.cuda.Stream()
+    copied = [torch.cuda.Event() for _ in range(2)]
+    consumed = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        for h, d in zip(hin, din):
-            d.copy_(h, non_blocking=True)
-        for _, f in calls:
-            f()
-        for h, d in zip(hout, dout):
-            h.copy_(d, non_blocking=True)
+    def upload(k):
+        with torch.cuda.stream(copy):
+            for h, d in zip(hin, dsets[k]):
+                d.copy_(h, non_blocking=True)
+            copied[k].record(copy)
 
-    for _ in range(warmup):
-        one()
+    def run(n):
+        upload(0)
+        for s in range(n):
+            k = s % 2
+            if s + 1 < n:
+                if s >= 1:
+                    copy.wait_event(consumed[1 - k])   # step s-1 has finished reading that set
+                upload(1 - k)
+            comp.wait_event(copied[k])
+            for _, f in calls[k]:
+                f()
+            consumed[k].record(comp)
+            for h, d in zip(hout, dout):
+                h.copy_(d, non_blocking=True)
+
+    run(warmup)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
+    e0.record(comp)
+    copy.wait_event(e0)
+    run(steps)
+    e1.record(comp)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     h2d = sum(t.numel() * t.element_size() for t in hin)
