@@ -328,35 +328,59 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const DArgs a) {
   }
   __syncthreads();
 
-  // 3) value sum in the rotated domain: thread = coordinate c; words come from shared memory
-  const int c = threadIdx.x;
-  const int w = c >> 5, bit = c & 31;
-  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+  // 3) value sum in the rotated domain.  Lane = bit position: coordinates 32w + lane
+  //    (w = 0..3), so one 16-byte broadcast load per plane brings the four words of a
+  //    token; warp wp takes tokens wp, wp + 4, ...; the warps' partial sums meet in
+  //    shared memory behind the weights (the K tiles are no longer read).
+  float acc[QCHUNK][4] = {};
   auto vstep = [&](int j, const float4 ww) {
     const uint8_t* tb = vbuf + (j >> 5) * VTB + (j & 31) * 16;
-    int idx = 0;
+    uint32_t wd[VKB][4];
 #pragma unroll
-    for (int p = 0; p < VKB; ++p) idx |= ((reinterpret_cast<const uint32_t*>(tb + p * TILE * 16)[w] >> bit) & 1u) << p;
-    const float cv = vc[idx];
-    acc0 = fmaf(ww.x, cv, acc0);
-    acc1 = fmaf(ww.y, cv, acc1);
-    acc2 = fmaf(ww.z, cv, acc2);
-    acc3 = fmaf(ww.w, cv, acc3);
+    for (int p = 0; p < VKB; ++p) {
+      const uint4 v = *reinterpret_cast<const uint4*>(tb + p * TILE * 16);
+      wd[p][0] = v.x;
+      wd[p][1] = v.y;
+      wd[p][2] = v.z;
+      wd[p][3] = v.w;
+    }
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      int idx = 0;
+#pragma unroll
+      for (int p = 0; p < VKB; ++p) idx |= ((wd[p][w] >> lane) & 1u) << p;
+      const float cv = vc[idx];
+      acc[0][w] = fmaf(ww.x, cv, acc[0][w]);
+      acc[1][w] = fmaf(ww.y, cv, acc[1][w]);
+      acc[2][w] = fmaf(ww.z, cv, acc[2][w]);
+      acc[3][w] = fmaf(ww.w, cv, acc[3][w]);
+    }
   };
-  if (a.veps > 0.f) {  // Sparse V: dropped tokens (all four weights zero) are skipped, uniformly over the CTA
-    for (int j = 0; j < ntok; ++j) {
+  if (a.veps > 0.f) {  // Sparse V: dropped tokens (all four weights zero) are skipped, uniformly over the warp
+    for (int j = warp; j < ntok; j += 4) {
       const float4 ww = wv[j];
       if (ww.x != 0.f || ww.y != 0.f || ww.z != 0.f || ww.w != 0.f) vstep(j, ww);
     }
   } else {
-#pragma unroll 4
-    for (int j = 0; j < ntok; ++j) vstep(j, wv[j]);
+#pragma unroll 2
+    for (int j = warp; j < ntok; j += 4) vstep(j, wv[j]);
   }
+  float* red = reinterpret_cast<float*>(kbuf + CH * 16);  // [4 warps][QCHUNK][DP]
+#pragma unroll
+  for (int qq = 0; qq < QCHUNK; ++qq)
+#pragma unroll
+    for (int w = 0; w < 4; ++w) red[(warp * QCHUNK + qq) * DP + 32 * w + lane] = acc[qq][w];
+  __syncthreads();
+  const int c = threadIdx.x;
+  float accs[4];
+#pragma unroll
+  for (int qq = 0; qq < QCHUNK; ++qq)
+    accs[qq] = (red[(0 * QCHUNK + qq) * DP + c] + red[(1 * QCHUNK + qq) * DP + c]) +
+               (red[(2 * QCHUNK + qq) * DP + c] + red[(3 * QCHUNK + qq) * DP + c]);
 
   // 4) partials
   const int hq0 = (bg % a.hkv) * a.group + QCHUNK * qc;
   const int nq = min(QCHUNK, a.group - QCHUNK * qc);
-  const float accs[4] = {acc0, acc1, acc2, acc3};
 #pragma unroll
   for (int qq = 0; qq < QCHUNK; ++qq) {
     if (qq < nq) {
@@ -439,7 +463,7 @@ int launch_decode(const DArgs& a, int blocks, cudaStream_t st) {
   cudaError_t e;
   if (staged) {
     constexpr int smem = staged_smem<KB, SI, VKB>();
-    static_assert(smem >= CH * 16, "weights alias the K tiles");
+    static_assert((CH / TILE) * TILE * (KB * 16 + 16 * SI) >= 2 * CH * 16, "weights and warp sums alias the K tiles");
     e = cudaFuncSetAttribute(decode_staged_kernel<KB, SI, VKB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_decode_attn: %s", cudaGetErrorString(e));
     cfg.dynamicSmemBytes = smem;
