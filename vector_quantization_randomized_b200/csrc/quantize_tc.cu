@@ -142,6 +142,13 @@ __device__ __forceinline__ float rotate_half(const uint8_t* xrow, int sw, int h,
   return ss.x + ss.y;
 }
 
+// a * b clamped to [0, 1] in one instruction
+__device__ __forceinline__ float mul_sat(float a, float b) {
+  float r;
+  asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 // Scalar code of one coordinate.  The predicate bits are shifted in at the
 // bottom of 32-bit words (one funnel shift of a sign bit each), so a word is
 // filled from its highest coordinate down; the centroid magnitude is picked
@@ -165,11 +172,13 @@ struct Coder {
     }
     mag0 = cent[L / 2];
   }
-  // Shifts [y <= 0] into wn and [|y| > t_{L/2+k}] into wp[k].  Returns y - c[idx].
+  // Shifts [y <= 0] into wn and [|y| > t_{L/2+k}] into wp[k].  Returns y - c[idx]
+  // (RES) or 0.
   //  * e = t - |y| is < 0 exactly when |y| > t (a zero difference is +0), so its
   //    sign bit is the predicate, and sat(-2^126 e) is 1 or 0 with it (a nonzero
   //    e is at least an ulp of t, far above 2^-126).
   //  * y - 2^-149 (no flush to zero) has its sign bit set exactly when y <= 0.
+  template <bool RES>
   __device__ __forceinline__ float code(float y, uint32_t& wn, uint32_t (&wp)[NP1]) const {
     const float a = fabsf(y);
     float mg = mag0;
@@ -177,11 +186,12 @@ struct Coder {
     for (int k = 0; k < NPT; ++k) {
       const float e = tp[k] - a;
       wp[k] = __funnelshift_l(__float_as_uint(e), wp[k], 1);
-      mg = fmaf(__saturatef(e * -0x1p126f), dmag[k], mg);
+      if constexpr (RES) mg = fmaf(mul_sat(e, -0x1p126f), dmag[k], mg);
     }
     const float ys = y - 0x1p-149f;
     wn = __funnelshift_l(__float_as_uint(ys), wn, 1);
-    return y - copysignf(mg, ys);  // c[idx] = (y > 0) ? +mag[m] : -mag[m]
+    if constexpr (RES) return y - copysignf(mg, ys);  // c[idx] = (y > 0) ? +mag[m] : -mag[m]
+    return 0.f;
   }
   // bit-plane words from the predicate words (ws = [y > 0])
   __device__ __forceinline__ void planes(uint32_t ws, const uint32_t (&wp)[NP1], uint32_t (&pl)[KB]) const {
@@ -199,10 +209,11 @@ struct Coder {
 
 // Code of this thread's half of one rotated row (y from rotate_half, ss its
 // return value).  Both threads of the vector (lanes l and l ^ 16) must call it
-// together: the norms are completed with a shuffle.  The residual pair of
-// coordinates (64h + 2k, 64h + 2k + 1) is handed to sink(k, r) as soon as it
-// is known (k descending within each code word); pl[b][w] is plane b's word 2h + w.
-template <int KB, class Sink>
+// together: the norms are completed with a shuffle.  With RES, the residual
+// pair of coordinates (64h + 2k, 64h + 2k + 1) is handed to sink(k, r) as soon
+// as it is known (k descending within each code word) and g2 is its squared
+// norm; pl[b][w] is plane b's word 2h + w.
+template <int KB, bool RES, class Sink>
 __device__ __forceinline__ void code_half(float2 (&y)[32], float ss, const Coder<KB>& cd, uint32_t (&pl)[KB][2],
                                           float& n, float& g2, Sink&& sink) {
   ss += __shfl_xor_sync(FULL, ss, 16);
@@ -218,19 +229,23 @@ __device__ __forceinline__ void code_half(float2 (&y)[32], float ss, const Coder
 #pragma unroll
     for (int k = 15; k >= 0; --k) {
       const float2 v = __fmul2_rn(y[16 * w + k], sc2);
-      const float r1 = cd.code(v.y, wn, wp);  // bit 2k + 1
-      const float r0 = cd.code(v.x, wn, wp);  // bit 2k
-      const float2 rv = make_float2(r0, r1);
-      acc = __ffma2_rn(rv, rv, acc);
-      sink(16 * w + k, rv);
+      const float r1 = cd.template code<RES>(v.y, wn, wp);  // bit 2k + 1
+      const float r0 = cd.template code<RES>(v.x, wn, wp);  // bit 2k
+      if constexpr (RES) {
+        const float2 rv = make_float2(r0, r1);
+        acc = __ffma2_rn(rv, rv, acc);
+        sink(16 * w + k, rv);
+      }
     }
     uint32_t p[KB];
     cd.planes(~wn, wp, p);
 #pragma unroll
     for (int b = 0; b < KB; ++b) pl[b][w] = p[b];
   }
-  g2 = acc.x + acc.y;
-  g2 += __shfl_xor_sync(FULL, g2, 16);
+  if constexpr (RES) {
+    g2 = acc.x + acc.y;
+    g2 += __shfl_xor_sync(FULL, g2, 16);
+  }
 }
 
 // Rare path, run by the whole warp: every projection whose two-pass
@@ -413,7 +428,7 @@ __global__ void __launch_bounds__(NT, 1) quantize128_kernel(const Q2Args a) {
       }
     };
     // every thread codes (rows past n_vec hold zeros), so the pair's shuffles are full-warp
-    code_half<KB>(y, ss, cd, pl, n, g2, sink);
+    code_half<KB, PROD>(y, ss, cd, pl, n, g2, sink);
     if constexpr (PROD) {
       // |z - S_i.r'| <= max||S_i|| (2^-21 + 2^-15) gamma' covers the lo-part rounding and the
       // fp32 accumulation of 256 exact products (gamma' = 2^14 gamma)
