@@ -282,6 +282,83 @@ int tq_device_status(int clear);
  */
 int tq_diag_bounded_wait(int64_t polls, tq_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Polar-coordinate stage 1 ("PolarQuant").
+ *
+ * [E1] same page, "第一步：PolarQuant", and "它到底怎么做到的？ / 第一步：
+ * PolarQuant —— 换个坐标系压缩": after the random rotation the vector is
+ * rewritten as a radius and angles; the angles follow a known, concentrated
+ * Beta law, so they are coded with fixed tables and no normalisation constant.
+ * The pages give no formulas; this library reads them as follows.
+ *   - y = H D (x/||x||) / sqrt(d_pad) as in tq_quantize; ||x|| kept as fp16.
+ *   - Recursive pairwise polar form: level 1 turns coordinates (2i, 2i+1) into
+ *     a radius and a full angle theta = atan2(y_2i+1, y_2i) in [0, 2 pi);
+ *     level l >= 2 turns radii (2i, 2i+1) of level l-1 into a radius and
+ *     psi = atan2(r_2i+1, r_2i) in [0, pi/2]; the last radius is 1.
+ *   - For a uniform direction theta is uniform and, at level l,
+ *     sin^2 psi ~ Beta(2^(l-2), 2^(l-2)); each level has a Lloyd-Max table.
+ *   - w bits per coordinate (1..3): a level-1 angle gets b1 = w+1 bits
+ *     (2^b1 equal cells, centroids at their middles), a higher-level angle
+ *     b2 = w-1 bits (w = 1: decoded at pi/4).
+ *   - Decisions: theta -> floor(theta 2^b1 / 2 pi); psi -> #{t : psi > t}.
+ * Code record: w*d_pad/8 bytes per vector, vectors consecutive; one
+ * little-endian bit stream, LSB first: the d_pad/2 level-1 indices (b1 bits
+ * each), then the level-2 indices (d_pad/4), ..., the last level (1), b2 bits
+ * each; unused bits zero.
+ *
+ * Tables (fp32, tq_polar_table_floats(d_pad, w) values, L1 = 2^b1, L2 = 2^b2):
+ *   [0, L1)            level-1 centroid angles (j + 1/2) 2 pi / L1
+ *   [L1, 3 L1)         (cos, sin) of those, interleaved
+ *   then for each level l = 2 .. log2(d_pad), 4 L2 - 1 values:
+ *                      L2 centroid angles (Lloyd-Max fixed point, fp32),
+ *                      L2 - 1 thresholds (fp32 midpoints of neighbouring
+ *                      fp32 centroids), (cos, sin) of the centroids.
+ * -------------------------------------------------------------------------*/
+typedef struct tq_polar_params {
+  int32_t d;      /* input dimension, 1..d_pad */
+  int32_t d_pad;  /* rotation size, 128 or 256 */
+  int32_t w;      /* bits per coordinate, 1..3 */
+  int32_t reserved;
+  const float* tables;    /* device, from tq_polar_make_tables */
+  const int8_t* signs_D;  /* device, d_pad signs (tq_make_params) */
+} tq_polar_params;
+
+/* Number of fp32 table values for (d_pad, w); -1 on bad arguments. */
+int64_t tq_polar_table_floats(int d_pad, int w);
+
+/* tq_polar_make_tables - the tables above, host memory (d_pad: power of two
+ * 4..4096, w: 1..3).  Lloyd-Max on each level's angle law by Gauss-Legendre
+ * quadrature in fp64; centroids rounded to fp32.  TQ_EINVAL on bad arguments. */
+int tq_polar_make_tables(int d_pad, int w, float* tables);
+
+/* Bytes of a polar code buffer holding n_vec records. */
+int64_t tq_polar_code_bytes(int d_pad, int w, int64_t n_vec);
+
+/*
+ * tq_polar_quantize - encode n_vec vectors (x: device, rows of d elements of
+ *   dtype, stride ld elements; 16-byte alignment as tq_quantize).  codes:
+ *   device, tq_polar_code_bytes bytes, 16-byte aligned; norms: device fp16.
+ */
+int tq_polar_quantize(const tq_polar_params* p, const void* x, int dtype, int64_t n_vec, int64_t ld,
+                      void* codes, uint16_t* norms, tq_stream_t stream);
+
+/*
+ * tq_polar_dequantize - x_hat = n D H y_hat / sqrt(d_pad) (first d
+ *   coordinates), y_hat rebuilt from the table centroids, top radius 1.
+ *   out: device fp32 rows of stride ld (>= d).
+ */
+int tq_polar_dequantize(const tq_polar_params* p, const void* codes, const uint16_t* norms, int64_t n_vec,
+                        float* out, int64_t ld, tq_stream_t stream);
+
+/*
+ * tq_polar_logits - l[h][k] = n_k <q~_h, y_hat_k> with q~ = H D q / sqrt(d_pad)
+ *   (= <q, x_hat_k>).  q: device fp32 [n_kv_heads*group][d]; query head h uses
+ *   KV head h / group, whose keys are records h/group * n_keys .. + n_keys - 1.
+ *   logits: device fp32 [n_kv_heads*group][n_keys].  1 <= group <= 8.
+ */
+int tq_polar_logits(const tq_polar_params* p, const float* q, int group, const void* codes,
+                    const uint16_t* norms, int64_t n_keys, int n_kv_heads, float* logits, tq_stream_t stream);
+
 /* Message for the last failed call on this thread ("" if none). */
 const char* tq_last_error(void);
 

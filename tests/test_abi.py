@@ -120,3 +120,34 @@ def test_validation_rejects_null_and_misaligned():
     assert lib.tq_decode_attn(ctypes.byref(st), ctypes.byref(st), base16, 1, 4, 1, base16, base16, base16, base16,
                               base16, base16, 64, 0.0, base16, base16, 1 << 20, None) == tq.TQ_EUNSUPPORTED
     assert lib.tq_code_bytes(-1, 1, 1, 1) == -1
+
+
+@pytest.mark.parametrize("d_pad", [128, 256])
+@pytest.mark.parametrize("w", [1, 2, 3])
+def test_polar_tables_match_oracle(d_pad, w):
+    """The library's angle tables (C++ Gauss-Legendre Lloyd iteration) equal the oracle's
+    (betainc masses, adaptive-quadrature moments) value for value."""
+    from oracle import polar
+    t = tq.tq_polar_make_tables(d_pad, w)
+    c1, per_level = polar.tables(d_pad, w)
+    L1, L2 = len(c1), len(per_level[0][0])
+    assert len(t) == tq._lib.tq_polar_table_floats(d_pad, w) == 3 * L1 + len(per_level) * (4 * L2 - 1)
+    assert np.array_equal(t[:L1], c1)
+    assert np.allclose(t[L1:3 * L1:2], np.cos(c1.astype(np.float64)), atol=1e-7)
+    assert np.allclose(t[L1 + 1:3 * L1:2], np.sin(c1.astype(np.float64)), atol=1e-7)
+    off = 3 * L1
+    for c, th in per_level:
+        assert np.array_equal(t[off:off + L2], c)
+        assert np.array_equal(t[off + L2:off + 2 * L2 - 1], th)
+        cs = t[off + 2 * L2 - 1:off + 4 * L2 - 1]
+        assert np.allclose(cs[0::2], np.cos(c.astype(np.float64)), atol=1e-7)
+        assert np.allclose(cs[1::2], np.sin(c.astype(np.float64)), atol=1e-7)
+        off += 4 * L2 - 1
+
+
+def test_polar_sizes_and_validation():
+    assert tq.tq_polar_code_bytes(128, 2, 10) == 10 * 32
+    assert tq._lib.tq_polar_table_floats(100, 2) == -1
+    assert tq._lib.tq_polar_table_floats(128, 4) == -1
+    bad = tq.tq_polar_params(128, 128, 4, 0, None, None)
+    assert tq._lib.tq_polar_quantize(ctypes.byref(bad), None, 2, 1, 128, None, None, None) == tq.TQ_EINVAL

@@ -31,7 +31,13 @@ class tq_params(ctypes.Structure):
                 ("signs_D", ctypes.c_void_p), ("S", ctypes.c_void_p)]
 
 
+class tq_polar_params(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("d_pad", ctypes.c_int32), ("w", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("tables", ctypes.c_void_p), ("signs_D", ctypes.c_void_p)]
+
+
 _P = ctypes.POINTER(tq_params)
+_PP = ctypes.POINTER(tq_polar_params)
 _vp, _i32, _i64, _u64, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_float
 _SIGS = {
     "tq_make_codebook": (_i32, [_i32, _i32, _vp, _vp]),
@@ -53,6 +59,12 @@ _SIGS = {
     "tq_search_topk": (_i32, [_P, _vp, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _vp, _i64, _vp]),
     "tq_device_status": (_i32, [_i32]),
     "tq_diag_bounded_wait": (_i32, [_i64, _vp]),
+    "tq_polar_table_floats": (_i64, [_i32, _i32]),
+    "tq_polar_make_tables": (_i32, [_i32, _i32, _vp]),
+    "tq_polar_code_bytes": (_i64, [_i32, _i32, _i64]),
+    "tq_polar_quantize": (_i32, [_PP, _vp, _i32, _i64, _i64, _vp, _vp, _vp]),
+    "tq_polar_dequantize": (_i32, [_PP, _vp, _vp, _i64, _vp, _i64, _vp]),
+    "tq_polar_logits": (_i32, [_PP, _vp, _i32, _vp, _vp, _i64, _i32, _vp, _vp]),
     "tq_last_error": (ctypes.c_char_p, []),
     "tq_version": (_i32, []),
 }
@@ -234,3 +246,58 @@ def tq_search_topk(p, q, codes, norms, rnorms, n_db, k, ids, scores, workspace, 
     return _check(_lib.tq_search_topk(p.ref, _ptr(q), q.shape[0], _ptr(codes), _ptr(norms), _ptr(rnorms), n_db,
                                       k, _ptr(ids), _ptr(scores), _ptr(workspace), workspace.numel(),
                                       _stream(stream)))
+
+
+# ---- polar-coordinate stage 1 -------------------------------------------------
+def tq_polar_make_tables(d_pad, w):
+    """Host: the polar code's angle tables (fp32, layout of include/tq.h)."""
+    n = _lib.tq_polar_table_floats(d_pad, w)
+    if n < 0:
+        raise TQError(TQ_EINVAL, "tq_polar_table_floats: bad arguments")
+    t = np.zeros(n, np.float32)
+    _check(_lib.tq_polar_make_tables(d_pad, w, t.ctypes.data))
+    return t
+
+
+def tq_polar_code_bytes(d_pad, w, n_vec):
+    return _lib.tq_polar_code_bytes(d_pad, w, n_vec)
+
+
+class PolarParams:
+    """A polar-code quantizer: host-made tables and sign flips copied to the device, plus the C struct."""
+
+    def __init__(self, d, w, seed=42, d_pad=None, device="cuda"):
+        import torch
+        d_pad = d_pad or (128 if d <= 128 else 256)
+        self.d, self.d_pad, self.w, self.seed = d, d_pad, w, seed
+        t = tq_polar_make_tables(d_pad, w)
+        D, _ = tq_make_params(d_pad, 0, seed)
+        self.host = dict(tables=t, D=D)
+        self.tables = torch.from_numpy(t).to(device)
+        self.D = torch.from_numpy(D).to(device)
+        self.struct = tq_polar_params(d, d_pad, w, 0, _ptr(self.tables), _ptr(self.D))
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+    def code_bytes(self, n_vec):
+        return tq_polar_code_bytes(self.d_pad, self.w, n_vec)
+
+
+def tq_polar_quantize(p, x, codes, norms, n_vec=None, ld=None, stream=None):
+    """Polar-code rows of x (device [n, ld] fp32/fp16/bf16) into codes / norms."""
+    n_vec = x.shape[0] if n_vec is None else n_vec
+    ld = x.stride(0) if ld is None else ld
+    return _check(_lib.tq_polar_quantize(p.ref, _ptr(x), _dtype_code(x), n_vec, ld, _ptr(codes), _ptr(norms),
+                                         _stream(stream)))
+
+
+def tq_polar_dequantize(p, codes, norms, n_vec, out, ld=None, stream=None):
+    ld = out.stride(0) if ld is None else ld
+    return _check(_lib.tq_polar_dequantize(p.ref, _ptr(codes), _ptr(norms), n_vec, _ptr(out), ld, _stream(stream)))
+
+
+def tq_polar_logits(p, q, group, codes, norms, n_keys, n_kv_heads, logits, stream=None):
+    return _check(_lib.tq_polar_logits(p.ref, _ptr(q), group, _ptr(codes), _ptr(norms), n_keys, n_kv_heads,
+                                       _ptr(logits), _stream(stream)))

@@ -1,0 +1,512 @@
+// Polar-coordinate stage 1 ("TurboQuant explainer" (m.163.com),
+// "第一步：PolarQuant" and "第一步：PolarQuant —— 换个坐标系压缩"): the
+// rotated unit vector y is rewritten in recursive pairwise polar form - level 1
+// turns coordinate pairs into (radius, full angle theta), level l >= 2 turns
+// pairs of level-(l-1) radii into (radius, psi in [0, pi/2]) - and every
+// angle is coded with its level's Lloyd-Max table (level 1: 2^(w+1) equal
+// cells; higher levels: 2^(w-1) cells of the law sin^2 psi ~ Beta).
+//
+//  * tq_polar_quantize: a warp per vector, lane l holding coordinates
+//    NI l .. NI l + NI - 1 (NI = d_pad / 32).  Rotation by in-lane and
+//    shuffle Walsh-Hadamard stages; the levels whose pairs lie inside a lane
+//    are formed there, the others across lanes with shuffles.  Indices are
+//    OR-ed into the warp's record in shared memory and stored by the first
+//    lanes as consecutive words.
+//  * tq_polar_dequantize: a warp per vector; each lane rebuilds its radius
+//    from the root down (cos / sin of its ancestors' centroids), then its
+//    coordinates, then the inverse rotation.
+//  * tq_polar_logits: a thread per key; the record is held in registers and
+//    the tree is walked depth first (every bit position is a compile-time
+//    constant), accumulating <q~, y_hat> for the key's query group from
+//    rotated queries in shared memory.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "common.h"
+#include "device.cuh"
+#include "prep.h"
+
+namespace {
+using namespace tqd;
+
+constexpr float kTwoPi = 6.283185307179586f;
+
+template <int DP, int W>
+struct PL {
+  static constexpr int NI = DP / 32;                          // coordinates per lane
+  static constexpr int LV = DP == 128 ? 7 : 8;                // levels
+  static constexpr int LI = NI == 4 ? 2 : 3;                  // levels formed inside a lane
+  static constexpr int B1 = W + 1, B2 = W - 1;
+  static constexpr int L1 = 1 << B1, L2 = 1 << B2;
+  static constexpr int NW = W * DP / 32;                      // 32-bit words of a record
+  static constexpr int T1 = 3 * L1;                           // table offset of level 2
+  static constexpr int TL = 4 * L2 - 1;                       // table values per level >= 2
+  // bit position of index u of level l (l = 1: pair u)
+  static constexpr __host__ __device__ int pos(int l, int u) {
+    int p = l == 1 ? B1 * u : B1 * (DP / 2);
+    for (int k = 2; k < l; ++k) p += B2 * (DP >> k);
+    return l == 1 ? p : p + B2 * u;
+  }
+};
+
+struct PArgs {
+  const uint8_t* x;
+  int64_t n_vec, ld;  // ld in elements (quantize) or floats (dequantize)
+  int d;
+  const float* tables;
+  const int8_t* D;
+  uint8_t* codes;
+  const uint8_t* ccodes;
+  uint16_t* norms;
+  const uint16_t* cnorms;
+  float* out;
+  // logits
+  const float* q;
+  float* logits;
+  int64_t n_keys;
+  int group;
+};
+
+template <int DT>
+__device__ __forceinline__ float load_elem(const uint8_t* row, int j) {
+  if constexpr (DT == TQ_F32) return reinterpret_cast<const float*>(row)[j];
+  if constexpr (DT == TQ_F16) return __half2float(reinterpret_cast<const __half*>(row)[j]);
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(row)[j]);
+}
+
+// ---- quantize ---------------------------------------------------------------
+template <int DP, int W, int DT>
+__global__ void __launch_bounds__(256) polar_quantize_kernel(const PArgs a) {
+  using P = PL<DP, W>;
+  constexpr int NI = P::NI;
+  __shared__ uint32_t rec[8][P::NW];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  // thresholds of the higher levels (uniform over the block)
+  float thr[P::LV - 1][P::L2 > 1 ? P::L2 - 1 : 1];
+#pragma unroll
+  for (int l = 2; l <= P::LV; ++l)
+#pragma unroll
+    for (int j = 0; j < P::L2 - 1; ++j) thr[l - 2][j] = __ldg(a.tables + P::T1 + (l - 2) * P::TL + P::L2 + j);
+  float dsg[NI];
+#pragma unroll
+  for (int k = 0; k < NI; ++k) dsg[k] = (float)a.D[NI * lane + k];
+  if (lane < P::NW) rec[wib][lane] = 0u;
+  __syncwarp();
+  const float rs = rsqrtf((float)DP);
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t v = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib; v < a.n_vec; v += warps) {
+    const uint8_t* row = a.x + v * a.ld * (DT == TQ_F32 ? 4 : 2);
+    float y[NI];
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < NI; ++k) {
+      const int j = NI * lane + k;
+      y[k] = j < a.d ? load_elem<DT>(row, j) * dsg[k] : 0.f;
+      ss = fmaf(y[k], y[k], ss);
+    }
+    ss = warp_sum(ss);
+    const float n = sqrtf(ss);
+    // Walsh-Hadamard: in-lane stages, then across lanes
+#pragma unroll
+    for (int hs = 1; hs < NI; hs <<= 1)
+#pragma unroll
+      for (int k = 0; k < NI; ++k)
+        if ((k & hs) == 0) {
+          const float u = y[k], w = y[k + hs];
+          y[k] = u + w;
+          y[k + hs] = u - w;
+        }
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1)
+#pragma unroll
+      for (int k = 0; k < NI; ++k) {
+        const float o = __shfl_xor_sync(FULL, y[k], s);
+        y[k] = (lane & s) ? (o - y[k]) : (y[k] + o);
+      }
+    const float sc = n > 0.f ? rs / n : 0.f;
+#pragma unroll
+    for (int k = 0; k < NI; ++k) y[k] *= sc;
+
+    uint32_t* r = rec[wib];
+    auto put = [&](int p, uint32_t idx) {  // OR `idx` in at bit position p
+      if (idx == 0u) return;
+      atomicOr(&r[p >> 5], idx << (p & 31));
+      if ((p & 31) != 0 && (idx >> (32 - (p & 31))) != 0u) atomicOr(&r[(p >> 5) + 1], idx >> (32 - (p & 31)));
+    };
+    auto angle_index = [&](int l, float psi) {
+      int ix = 0;
+#pragma unroll
+      for (int j = 0; j < P::L2 - 1; ++j) ix += psi > thr[l - 2][j] ? 1 : 0;
+      return (uint32_t)ix;
+    };
+    // level 1
+    float rad[NI / 2];
+#pragma unroll
+    for (int j = 0; j < NI / 2; ++j) {
+      const float x0 = y[2 * j], x1 = y[2 * j + 1];
+      float t = atan2f(x1, x0) * (P::L1 / kTwoPi);
+      if (t < 0.f) t += (float)P::L1;
+      put(P::pos(1, (NI / 2) * lane + j), (uint32_t)min((int)t, P::L1 - 1));
+      rad[j] = sqrtf(fmaf(x0, x0, x1 * x1));
+    }
+    // levels inside the lane
+#pragma unroll
+    for (int l = 2; l <= P::LI; ++l) {
+      const int cnt = NI >> l;  // nodes of level l in this lane
+#pragma unroll
+      for (int j = 0; j < cnt; ++j) {
+        const float ra = rad[2 * j], rb = rad[2 * j + 1];
+        if constexpr (P::B2 > 0) put(P::pos(l, cnt * lane + j), angle_index(l, atan2f(rb, ra)));
+        rad[j] = sqrtf(fmaf(ra, ra, rb * rb));
+      }
+    }
+    // levels across lanes: node = lane >> (l - LI), partner lane differs in bit l - LI - 1
+    float R = rad[0];
+#pragma unroll
+    for (int l = P::LI + 1; l <= P::LV; ++l) {
+      const int s = 1 << (l - P::LI - 1);
+      const float o = __shfl_xor_sync(FULL, R, s);
+      const float ra = (lane & s) ? o : R, rb = (lane & s) ? R : o;
+      if constexpr (P::B2 > 0)
+        if ((lane & (2 * s - 1)) == 0) put(P::pos(l, lane >> (l - P::LI)), angle_index(l, atan2f(rb, ra)));
+      R = sqrtf(fmaf(ra, ra, rb * rb));
+    }
+    __syncwarp();
+    if (lane < P::NW) {
+      reinterpret_cast<uint32_t*>(a.codes + v * (P::NW * 4))[lane] = r[lane];
+      r[lane] = 0u;
+    }
+    if (lane == 0) a.norms[v] = __half_as_ushort(__float2half_rn(n));
+    __syncwarp();
+  }
+}
+
+// ---- dequantize ---------------------------------------------------------------
+template <int DP, int W>
+__global__ void __launch_bounds__(256) polar_dequantize_kernel(const PArgs a) {
+  using P = PL<DP, W>;
+  constexpr int NI = P::NI;
+  __shared__ uint32_t rec[8][P::NW + 1];
+  __shared__ float tab[P::T1 + (P::LV - 1) * P::TL];
+  for (int i = threadIdx.x; i < P::T1 + (P::LV - 1) * P::TL; i += blockDim.x) tab[i] = a.tables[i];
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  float dsg[NI];
+#pragma unroll
+  for (int k = 0; k < NI; ++k) dsg[k] = (float)a.D[NI * lane + k];
+  if (lane == 0) rec[wib][P::NW] = 0u;
+  const float rs = rsqrtf((float)DP);
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t v = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib; v < a.n_vec; v += warps) {
+    uint32_t* r = rec[wib];
+    if (lane < P::NW) r[lane] = __ldg(reinterpret_cast<const uint32_t*>(a.ccodes + v * (P::NW * 4)) + lane);
+    __syncwarp();
+    auto get = [&](int p, int width) {
+      const uint64_t w64 = (uint64_t)r[p >> 5] | ((uint64_t)r[(p >> 5) + 1] << 32);
+      return (int)((w64 >> (p & 31)) & ((1u << width) - 1u));
+    };
+    auto cs = [&](int l, int ix) {  // (cos, sin) of the centroid ix of level l >= 2
+      const float* t = tab + P::T1 + (l - 2) * P::TL + 2 * P::L2 - 1;
+      return make_float2(t[2 * ix], t[2 * ix + 1]);
+    };
+    // root to this lane's node of level LI
+    float R = 1.f;
+#pragma unroll
+    for (int l = P::LV; l > P::LI; --l) {
+      const int ix = P::B2 > 0 ? get(P::pos(l, lane >> (l - P::LI)), P::B2) : 0;
+      const float2 c = cs(l, ix);
+      R *= ((lane >> (l - P::LI - 1)) & 1) ? c.y : c.x;
+    }
+    // levels inside the lane, from LI down to 2
+    float rad[NI / 2];
+    rad[0] = R;
+#pragma unroll
+    for (int l = P::LI; l >= 2; --l) {
+      const int cnt = NI >> l;
+#pragma unroll
+      for (int j = cnt - 1; j >= 0; --j) {
+        const int ix = P::B2 > 0 ? get(P::pos(l, cnt * lane + j), P::B2) : 0;
+        const float2 c = cs(l, ix);
+        const float pr = rad[j];
+        rad[2 * j] = pr * c.x;
+        rad[2 * j + 1] = pr * c.y;
+      }
+    }
+    float y[NI];
+#pragma unroll
+    for (int j = 0; j < NI / 2; ++j) {
+      const int ix = get(P::pos(1, (NI / 2) * lane + j), P::B1);
+      y[2 * j] = rad[j] * tab[P::L1 + 2 * ix];
+      y[2 * j + 1] = rad[j] * tab[P::L1 + 2 * ix + 1];
+    }
+    __syncwarp();
+    // inverse rotation D H y / sqrt(DP), times the norm
+#pragma unroll
+    for (int hs = 1; hs < NI; hs <<= 1)
+#pragma unroll
+      for (int k = 0; k < NI; ++k)
+        if ((k & hs) == 0) {
+          const float u = y[k], w = y[k + hs];
+          y[k] = u + w;
+          y[k + hs] = u - w;
+        }
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1)
+#pragma unroll
+      for (int k = 0; k < NI; ++k) {
+        const float o = __shfl_xor_sync(FULL, y[k], s);
+        y[k] = (lane & s) ? (o - y[k]) : (y[k] + o);
+      }
+    const float nrm = __half2float(__ushort_as_half(__ldg(a.cnorms + v))) * rs;
+    float* orow = a.out + v * a.ld;
+#pragma unroll
+    for (int k = 0; k < NI; ++k) {
+      const int c = NI * lane + k;
+      if (c < a.d) orow[c] = y[k] * nrm * dsg[k];
+    }
+  }
+}
+
+// ---- logits ---------------------------------------------------------------------
+template <int DP, int W, int G>
+__global__ void __launch_bounds__(128) polar_logits_kernel(const PArgs a) {
+  using P = PL<DP, W>;
+  __shared__ float qt[G][DP];
+  __shared__ float2 cs1[P::L1];
+  __shared__ float2 csh[P::LV - 1][P::L2];
+  const int tid = threadIdx.x;
+  const int kv = blockIdx.y;
+  for (int i = tid; i < P::L1; i += blockDim.x) cs1[i] = make_float2(a.tables[P::L1 + 2 * i], a.tables[P::L1 + 2 * i + 1]);
+  for (int i = tid; i < (P::LV - 1) * P::L2; i += blockDim.x) {
+    const int l = i / P::L2, j = i % P::L2;
+    const float* t = a.tables + P::T1 + l * P::TL + 2 * P::L2 - 1;
+    csh[l][j] = make_float2(t[2 * j], t[2 * j + 1]);
+  }
+  // rotated queries q~ = H D q / sqrt(DP) of this KV head's group
+  for (int i = tid; i < G * DP; i += blockDim.x) {
+    const int g = i / DP, j = i % DP;
+    qt[g][j] = (g < a.group && j < a.d) ? a.q[((int64_t)kv * a.group + g) * a.d + j] * (float)a.D[j] : 0.f;
+  }
+  __syncthreads();
+  for (int hs = 1; hs < DP; hs <<= 1) {
+    for (int i = tid; i < G * DP / 2; i += blockDim.x) {
+      const int g = i / (DP / 2), p = i % (DP / 2);
+      const int j = ((p & ~(hs - 1)) << 1) | (p & (hs - 1));
+      const float u = qt[g][j], w = qt[g][j + hs];
+      qt[g][j] = u + w;
+      qt[g][j + hs] = u - w;
+    }
+    __syncthreads();
+  }
+  const int64_t key = (int64_t)blockIdx.x * blockDim.x + tid;
+  if (key >= a.n_keys) return;
+  const int64_t vi = (int64_t)kv * a.n_keys + key;
+  uint32_t r[P::NW + 1];
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.ccodes + vi * (P::NW * 4));
+#pragma unroll
+    for (int i = 0; i < P::NW / 4; ++i) {
+      const uint4 u = __ldg(src + i);
+      r[4 * i] = u.x;
+      r[4 * i + 1] = u.y;
+      r[4 * i + 2] = u.z;
+      r[4 * i + 3] = u.w;
+    }
+    r[P::NW] = 0u;
+  }
+  auto get = [&](int p, int width) {  // p is a compile-time constant after unrolling
+    const uint64_t w64 = (uint64_t)r[p >> 5] | ((uint64_t)r[(p >> 5) + 1] << 32);
+    return (int)((w64 >> (p & 31)) & ((1u << width) - 1u));
+  };
+  float acc[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) acc[g] = 0.f;
+  float st[P::LV + 1];  // radius of the current node of each level, root first
+  st[P::LV] = 1.f;
+#pragma unroll
+  for (int u = 0; u < DP / 4; ++u) {  // level-2 nodes in order
+    // refresh the levels whose node changes at u (all indices are constants here)
+#pragma unroll
+    for (int l = P::LV; l >= 3; --l) {
+      if ((u & ((1 << (l - 3)) - 1)) == 0) {  // a new node of level l - 1 starts at u
+        const int node = u >> (l - 3);         // node of level l - 1; its parent is node >> 1 of level l
+        const int ix = P::B2 > 0 ? get(P::pos(l, node >> 1), P::B2) : 0;
+        const float2 c = csh[l - 2][ix];
+        st[l - 1] = st[l] * ((node & 1) ? c.y : c.x);
+      }
+    }
+    const int ix2 = P::B2 > 0 ? get(P::pos(2, u), P::B2) : 0;
+    const float2 c2 = csh[0][ix2];
+    const float ra = st[2] * c2.x, rb = st[2] * c2.y;
+    const float2 t0 = cs1[get(P::pos(1, 2 * u), P::B1)];
+    const float2 t1 = cs1[get(P::pos(1, 2 * u + 1), P::B1)];
+    const float y0 = ra * t0.x, y1 = ra * t0.y, y2 = rb * t1.x, y3 = rb * t1.y;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float4 qq = *reinterpret_cast<const float4*>(&qt[g][4 * u]);
+      acc[g] = fmaf(y0, qq.x, fmaf(y1, qq.y, fmaf(y2, qq.z, fmaf(y3, qq.w, acc[g]))));
+    }
+  }
+  const float n = __half2float(__ushort_as_half(__ldg(a.cnorms + vi))) * rsqrtf((float)DP);
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+    if (g < a.group) a.logits[((int64_t)kv * a.group + g) * a.n_keys + key] = acc[g] * n;
+}
+
+int launch_err(const char* who) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "%s: launch failed: %s", who, cudaGetErrorString(e));
+  return TQ_OK;
+}
+
+int check_polar(const tq_polar_params* p, const char* who) {
+  if (!p) return tq::set_error(TQ_EINVAL, "%s: NULL params", who);
+  if (p->d_pad != 128 && p->d_pad != 256) return tq::set_error(TQ_EUNSUPPORTED, "%s: d_pad must be 128 or 256", who);
+  if (p->d < 1 || p->d > p->d_pad) return tq::set_error(TQ_EINVAL, "%s: d out of range", who);
+  if (p->w < 1 || p->w > 3) return tq::set_error(TQ_EINVAL, "%s: w must be 1..3", who);
+  if (!p->tables || !p->signs_D) return tq::set_error(TQ_EINVAL, "%s: NULL tables or signs", who);
+  return TQ_OK;
+}
+
+int grid_for(int64_t n_vec) {
+  return (int)std::max<int64_t>(1, std::min<int64_t>((n_vec + 7) / 8, (int64_t)tq::sm_count() * 16));
+}
+
+template <int DP, int W>
+int quantize_dw(int dtype, const PArgs& a, cudaStream_t st) {
+  const int g = grid_for(a.n_vec);
+  if (dtype == TQ_F32)
+    polar_quantize_kernel<DP, W, TQ_F32><<<g, 256, 0, st>>>(a);
+  else if (dtype == TQ_F16)
+    polar_quantize_kernel<DP, W, TQ_F16><<<g, 256, 0, st>>>(a);
+  else
+    polar_quantize_kernel<DP, W, TQ_BF16><<<g, 256, 0, st>>>(a);
+  return launch_err("tq_polar_quantize");
+}
+
+template <int DP, int W>
+int dequantize_dw(const PArgs& a, cudaStream_t st) {
+  polar_dequantize_kernel<DP, W><<<grid_for(a.n_vec), 256, 0, st>>>(a);
+  return launch_err("tq_polar_dequantize");
+}
+
+template <int DP, int W>
+int logits_dw(const PArgs& a, int n_kv, cudaStream_t st) {
+  const dim3 grid((unsigned)((a.n_keys + 127) / 128), (unsigned)n_kv);
+  if (a.group <= 1)
+    polar_logits_kernel<DP, W, 1><<<grid, 128, 0, st>>>(a);
+  else if (a.group <= 2)
+    polar_logits_kernel<DP, W, 2><<<grid, 128, 0, st>>>(a);
+  else if (a.group <= 4)
+    polar_logits_kernel<DP, W, 4><<<grid, 128, 0, st>>>(a);
+  else
+    polar_logits_kernel<DP, W, 8><<<grid, 128, 0, st>>>(a);
+  return launch_err("tq_polar_logits");
+}
+
+#define TQ_POLAR_DISPATCH(dp, w, CALL) \
+  ((dp) == 128 ? ((w) == 1 ? CALL(128, 1) : (w) == 2 ? CALL(128, 2) : CALL(128, 3)) \
+               : ((w) == 1 ? CALL(256, 1) : (w) == 2 ? CALL(256, 2) : CALL(256, 3)))
+
+}  // namespace
+
+extern "C" int tq_polar_quantize(const tq_polar_params* p, const void* x, int dtype, int64_t n_vec, int64_t ld,
+                                 void* codes, uint16_t* norms, tq_stream_t stream) {
+  using namespace tq;
+  int rc = check_polar(p, "tq_polar_quantize");
+  if (rc) return rc;
+  if (n_vec < 0) return set_error(TQ_EINVAL, "tq_polar_quantize: n_vec < 0");
+  if (n_vec == 0) {
+    clear_error();
+    return TQ_OK;
+  }
+  if (dtype != TQ_F32 && dtype != TQ_F16 && dtype != TQ_BF16) return set_error(TQ_EINVAL, "tq_polar_quantize: dtype");
+  if (!x || !codes || !norms) return set_error(TQ_EINVAL, "tq_polar_quantize: NULL pointer argument");
+  if (ld < p->d) return set_error(TQ_EINVAL, "tq_polar_quantize: ld < d");
+  const int es = dtype == TQ_F32 ? 4 : 2;
+  if (!aligned(x, 16) || ((ld * es) % 16) != 0 || !aligned(codes, 16) || !aligned(norms, 2))
+    return set_error(TQ_EINVAL, "tq_polar_quantize: x, ld*elem and codes must be 16-byte aligned");
+  PArgs a{};
+  a.x = static_cast<const uint8_t*>(x);
+  a.n_vec = n_vec;
+  a.ld = ld;
+  a.d = p->d;
+  a.tables = p->tables;
+  a.D = p->signs_D;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.norms = norms;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define Q_CALL(DP, W) quantize_dw<DP, W>(dtype, a, st)
+  rc = TQ_POLAR_DISPATCH(p->d_pad, p->w, Q_CALL);
+#undef Q_CALL
+  if (rc == TQ_OK) clear_error();
+  return rc;
+}
+
+extern "C" int tq_polar_dequantize(const tq_polar_params* p, const void* codes, const uint16_t* norms, int64_t n_vec,
+                                   float* out, int64_t ld, tq_stream_t stream) {
+  using namespace tq;
+  int rc = check_polar(p, "tq_polar_dequantize");
+  if (rc) return rc;
+  if (n_vec < 0) return set_error(TQ_EINVAL, "tq_polar_dequantize: n_vec < 0");
+  if (n_vec == 0) {
+    clear_error();
+    return TQ_OK;
+  }
+  if (!codes || !norms || !out) return set_error(TQ_EINVAL, "tq_polar_dequantize: NULL pointer argument");
+  if (ld < p->d) return set_error(TQ_EINVAL, "tq_polar_dequantize: ld < d");
+  if (!aligned(codes, 16) || !aligned(out, 4)) return set_error(TQ_EINVAL, "tq_polar_dequantize: misaligned pointer");
+  PArgs a{};
+  a.n_vec = n_vec;
+  a.ld = ld;
+  a.d = p->d;
+  a.tables = p->tables;
+  a.D = p->signs_D;
+  a.ccodes = static_cast<const uint8_t*>(codes);
+  a.cnorms = norms;
+  a.out = out;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define D_CALL(DP, W) dequantize_dw<DP, W>(a, st)
+  rc = TQ_POLAR_DISPATCH(p->d_pad, p->w, D_CALL);
+#undef D_CALL
+  if (rc == TQ_OK) clear_error();
+  return rc;
+}
+
+extern "C" int tq_polar_logits(const tq_polar_params* p, const float* q, int group, const void* codes,
+                               const uint16_t* norms, int64_t n_keys, int n_kv_heads, float* logits,
+                               tq_stream_t stream) {
+  using namespace tq;
+  int rc = check_polar(p, "tq_polar_logits");
+  if (rc) return rc;
+  if (group < 1 || group > 8) return set_error(TQ_EINVAL, "tq_polar_logits: group must be 1..8");
+  if (n_keys < 0 || n_kv_heads < 0) return set_error(TQ_EINVAL, "tq_polar_logits: negative size");
+  if (n_keys == 0 || n_kv_heads == 0) {
+    clear_error();
+    return TQ_OK;
+  }
+  if (n_kv_heads > 65535) return set_error(TQ_EUNSUPPORTED, "tq_polar_logits: more than 65535 KV heads");
+  if (!q || !codes || !norms || !logits) return set_error(TQ_EINVAL, "tq_polar_logits: NULL pointer argument");
+  if (!aligned(codes, 16) || !aligned(q, 4) || !aligned(logits, 4))
+    return set_error(TQ_EINVAL, "tq_polar_logits: misaligned pointer");
+  PArgs a{};
+  a.d = p->d;
+  a.tables = p->tables;
+  a.D = p->signs_D;
+  a.ccodes = static_cast<const uint8_t*>(codes);
+  a.cnorms = norms;
+  a.q = q;
+  a.logits = logits;
+  a.n_keys = n_keys;
+  a.group = group;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define L_CALL(DP, W) logits_dw<DP, W>(a, n_kv_heads, st)
+  rc = TQ_POLAR_DISPATCH(p->d_pad, p->w, L_CALL);
+#undef L_CALL
+  if (rc == TQ_OK) clear_error();
+  return rc;
+}
