@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="layer", choices=["layer", "decode", "quantize", "search"])
+    ap.add_argument("--workload", default="layer", choices=["layer", "decode", "quantize", "search", "polar"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-kernels", action="store_true")
@@ -456,7 +456,9 @@ def gpu_kv(torch, n_seq, n_heads, n_tokens, d, seed):
 
 def run_secondary(args, world, rank, local, torch, tq, wl):
     """Other workloads (their own JSON line): 'decode' = 64 sequences x 8 KV heads x 16384 tokens
-    (K product b=3, V MSE b=3, 32 query heads); 'quantize' = 2^20 bf16 vectors at b=2,3,4."""
+    (K product b=3, V MSE b=3, 32 query heads); 'quantize' = 2^20 bf16 vectors at b=2,3,4;
+    'search' = 10^4 queries over 10^6 vectors; 'polar' = the polar-coordinate code on the
+    layer's keys (quantize + logits at w = 2, 3)."""
     peak, peak_kind = measured_peaks()
     ev = lambda: torch.cuda.Event(enable_timing=True)
     if args.workload == "decode":
@@ -538,6 +540,41 @@ def run_secondary(args, world, rank, local, torch, tq, wl):
                             "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4), "frac_measured": round(gbs / peak, 4)}
         line = {"metric": "quantize vectors/s", "value": res["b4"]["vectors_per_s"], "unit": "vectors/s",
                 "config": {"workload": "quantize-2^20x128-bf16-prod-m128"}, "per_bits": res}
+    elif args.workload == "polar":
+        # polar-coordinate stage 1 on the layer's keys: 8 KV heads x 32768 tokens, d 128, bf16,
+        # 32 query heads (GQA 4); quantize then logits, at w = 2 and 3 bits per coordinate
+        H, T, d, G = 8, 32768, 128, 4
+        n = H * T
+        x = gpu_kv(torch, 1, H, T, d, wl.SEED_KEYS)
+        q = torch.randn((H * G, d), device="cuda")
+        calls, byts = [], {}
+        for w in (2, 3):
+            p = tq.PolarParams(d, w, seed=wl.SEED_PARAMS)
+            c = torch.empty(p.code_bytes(n), dtype=torch.uint8, device="cuda")
+            nn = torch.empty(n, dtype=torch.int16, device="cuda")
+            lg = torch.empty((H * G, T), device="cuda")
+            calls.append((f"polar_quantize_w{w}", lambda p=p, c=c, nn=nn: tq.tq_polar_quantize(p, x, c, nn)))
+            calls.append((f"polar_logits_w{w}",
+                          lambda p=p, c=c, nn=nn, lg=lg: tq.tq_polar_logits(p, q, G, c, nn, T, H, lg)))
+            byts[f"polar_quantize_w{w}"] = n * d * 2 + c.numel() + 2 * n
+            byts[f"polar_logits_w{w}"] = c.numel() + 2 * n + q.numel() * 4
+
+        class _Calls:
+            def calls(self):
+                return calls
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+        step_ms, per_call = time_steps(torch, _Calls(), args.steps, args.warmup, world, flush)
+        ms = statistics.median(step_ms)
+        kern = {}
+        for lab, ts in per_call.items():
+            us = statistics.median(ts) * 1000
+            gbs = byts[lab] / (us / 1e6) / 1e9
+            kern[lab] = {"us": round(us, 2), "gbs": round(gbs, 1), "frac_measured": round(gbs / peak, 4)}
+        line = {"metric": "polar-code keys/s (quantize + logits, w=2 and w=3)", "value": 2 * n / (ms / 1e3),
+                "unit": "keys/s", "ms_per_step": ms,
+                "config": {"workload": "polar-kv8x32768-gqa4-d128-bf16", "w": [2, 3],
+                           "l2": "flushed between steps (256 MB write)"},
+                "kernels": kern}
     elif args.workload == "search":
         n_db, n_q, d, k = 1000000, 10000, 200, 10
         db = torch.from_numpy(wl.search_set(n_db, d, seed=wl.SEED_KEYS)).to(torch.bfloat16).cuda()

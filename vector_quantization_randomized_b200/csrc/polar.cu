@@ -9,9 +9,12 @@
 //  * tq_polar_quantize: a warp per vector, lane l holding coordinates
 //    NI l .. NI l + NI - 1 (NI = d_pad / 32).  Rotation by in-lane and
 //    shuffle Walsh-Hadamard stages; the levels whose pairs lie inside a lane
-//    are formed there, the others across lanes with shuffles.  Indices are
-//    OR-ed into the warp's record in shared memory and stored by the first
-//    lanes as consecutive words.
+//    are formed there, the others across lanes with shuffles.  No angle is
+//    computed: a level-1 cell is the quadrant (signs) and the position inside
+//    it (cross products with the cell boundaries), a higher-level decision
+//    psi > t is rb cos t > ra sin t.  Indices are OR-ed into the warp's
+//    record in shared memory and stored by the first lanes as consecutive
+//    words.
 //  * tq_polar_dequantize: a warp per vector; each lane rebuilds its radius
 //    from the root down (cos / sin of its ancestors' centroids), then its
 //    coordinates, then the inverse rotation.
@@ -32,8 +35,6 @@
 
 namespace {
 using namespace tqd;
-
-constexpr float kTwoPi = 6.283185307179586f;
 
 template <int DP, int W>
 struct PL {
@@ -85,12 +86,13 @@ __global__ void __launch_bounds__(256) polar_quantize_kernel(const PArgs a) {
   constexpr int NI = P::NI;
   __shared__ uint32_t rec[8][P::NW];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  // thresholds of the higher levels (uniform over the block)
-  float thr[P::LV - 1][P::L2 > 1 ? P::L2 - 1 : 1];
+  // (cos t, sin t) of the higher levels' thresholds t: psi > t exactly when rb cos t > ra sin t
+  // (psi = atan2(rb, ra) and t both in [0, pi/2])
+  float thc[P::LV - 1][P::L2 > 1 ? P::L2 - 1 : 1], ths[P::LV - 1][P::L2 > 1 ? P::L2 - 1 : 1];
 #pragma unroll
   for (int l = 2; l <= P::LV; ++l)
 #pragma unroll
-    for (int j = 0; j < P::L2 - 1; ++j) thr[l - 2][j] = __ldg(a.tables + P::T1 + (l - 2) * P::TL + P::L2 + j);
+    for (int j = 0; j < P::L2 - 1; ++j) sincosf(__ldg(a.tables + P::T1 + (l - 2) * P::TL + P::L2 + j), &ths[l - 2][j], &thc[l - 2][j]);
   float dsg[NI];
 #pragma unroll
   for (int k = 0; k < NI; ++k) dsg[k] = (float)a.D[NI * lane + k];
@@ -137,20 +139,27 @@ __global__ void __launch_bounds__(256) polar_quantize_kernel(const PArgs a) {
       atomicOr(&r[p >> 5], idx << (p & 31));
       if ((p & 31) != 0 && (idx >> (32 - (p & 31))) != 0u) atomicOr(&r[(p >> 5) + 1], idx >> (32 - (p & 31)));
     };
-    auto angle_index = [&](int l, float psi) {
+    auto angle_index = [&](int l, float ra, float rb) {
       int ix = 0;
 #pragma unroll
-      for (int j = 0; j < P::L2 - 1; ++j) ix += psi > thr[l - 2][j] ? 1 : 0;
+      for (int j = 0; j < P::L2 - 1; ++j) ix += rb * thc[l - 2][j] > ra * ths[l - 2][j] ? 1 : 0;
       return (uint32_t)ix;
     };
-    // level 1
+    // level 1: cell floor(theta L1 / 2 pi) of theta = atan2(x1, x0) in [0, 2 pi), by the quadrant
+    // (signs) and the position inside it (cross products with the cell boundaries)
     float rad[NI / 2];
 #pragma unroll
     for (int j = 0; j < NI / 2; ++j) {
       const float x0 = y[2 * j], x1 = y[2 * j + 1];
-      float t = atan2f(x1, x0) * (P::L1 / kTwoPi);
-      if (t < 0.f) t += (float)P::L1;
-      put(P::pos(1, (NI / 2) * lane + j), (uint32_t)min((int)t, P::L1 - 1));
+      const int qd = x1 > 0.f ? (x0 > 0.f ? 0 : 1) : (x1 < 0.f ? (x0 < 0.f ? 2 : 3) : (x0 < 0.f ? 2 : 0));
+      const float u = qd == 0 ? x0 : qd == 1 ? x1 : qd == 2 ? -x0 : -x1;  // rotated into [0, pi/2)
+      const float w = qd == 0 ? x1 : qd == 1 ? -x0 : qd == 2 ? -x1 : x0;
+      int sub = 0;
+      if constexpr (P::L1 == 8) sub = w >= u ? 1 : 0;
+      if constexpr (P::L1 == 16)
+        sub = (w * 0.92387953f >= u * 0.38268343f ? 1 : 0) + (w >= u ? 1 : 0) +
+              (w * 0.38268343f >= u * 0.92387953f ? 1 : 0);  // boundaries pi/8, pi/4, 3 pi/8
+      put(P::pos(1, (NI / 2) * lane + j), (uint32_t)(qd * (P::L1 / 4) + sub));
       rad[j] = sqrtf(fmaf(x0, x0, x1 * x1));
     }
     // levels inside the lane
@@ -160,7 +169,7 @@ __global__ void __launch_bounds__(256) polar_quantize_kernel(const PArgs a) {
 #pragma unroll
       for (int j = 0; j < cnt; ++j) {
         const float ra = rad[2 * j], rb = rad[2 * j + 1];
-        if constexpr (P::B2 > 0) put(P::pos(l, cnt * lane + j), angle_index(l, atan2f(rb, ra)));
+        if constexpr (P::B2 > 0) put(P::pos(l, cnt * lane + j), angle_index(l, ra, rb));
         rad[j] = sqrtf(fmaf(ra, ra, rb * rb));
       }
     }
@@ -172,7 +181,7 @@ __global__ void __launch_bounds__(256) polar_quantize_kernel(const PArgs a) {
       const float o = __shfl_xor_sync(FULL, R, s);
       const float ra = (lane & s) ? o : R, rb = (lane & s) ? R : o;
       if constexpr (P::B2 > 0)
-        if ((lane & (2 * s - 1)) == 0) put(P::pos(l, lane >> (l - P::LI)), angle_index(l, atan2f(rb, ra)));
+        if ((lane & (2 * s - 1)) == 0) put(P::pos(l, lane >> (l - P::LI)), angle_index(l, ra, rb));
       R = sqrtf(fmaf(ra, ra, rb * rb));
     }
     __syncwarp();
