@@ -72,13 +72,6 @@ struct PArgs {
   int group;
 };
 
-template <int DT>
-__device__ __forceinline__ float load_elem(const uint8_t* row, int j) {
-  if constexpr (DT == TQ_F32) return reinterpret_cast<const float*>(row)[j];
-  if constexpr (DT == TQ_F16) return __half2float(reinterpret_cast<const __half*>(row)[j]);
-  return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(row)[j]);
-}
-
 // ---- quantize ---------------------------------------------------------------
 template <int DP, int W, int DT>
 __global__ void __launch_bounds__(256) polar_quantize_kernel(const PArgs a) {
@@ -104,11 +97,35 @@ __global__ void __launch_bounds__(256) polar_quantize_kernel(const PArgs a) {
     const uint8_t* row = a.x + v * a.ld * (DT == TQ_F32 ? 4 : 2);
     float y[NI];
     float ss = 0.f;
+    // groups of 4 elements (d is a multiple of 4, of 8 for 16-bit types): one 8- or 16-byte load each
 #pragma unroll
-    for (int k = 0; k < NI; ++k) {
-      const int j = NI * lane + k;
-      y[k] = j < a.d ? load_elem<DT>(row, j) * dsg[k] : 0.f;
-      ss = fmaf(y[k], y[k], ss);
+    for (int g4 = 0; g4 < NI / 4; ++g4) {
+      const int j = NI * lane + 4 * g4;
+      float e[4] = {0.f, 0.f, 0.f, 0.f};
+      if (j < a.d) {
+        if constexpr (DT == TQ_F32) {
+          const float4 f = __ldg(reinterpret_cast<const float4*>(row) + (j >> 2));
+          e[0] = f.x, e[1] = f.y, e[2] = f.z, e[3] = f.w;
+        } else {
+          const uint2 u = __ldg(reinterpret_cast<const uint2*>(row) + (j >> 2));
+          const uint32_t wd[2] = {u.x, u.y};
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if constexpr (DT == TQ_BF16) {
+              e[2 * h] = __uint_as_float(wd[h] << 16);
+              e[2 * h + 1] = __uint_as_float(wd[h] & 0xFFFF0000u);
+            } else {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wd[h]));
+              e[2 * h] = f.x, e[2 * h + 1] = f.y;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        y[4 * g4 + k] = e[k] * dsg[4 * g4 + k];
+        ss = fmaf(y[4 * g4 + k], y[4 * g4 + k], ss);
+      }
     }
     ss = warp_sum(ss);
     const float n = sqrtf(ss);
