@@ -5,7 +5,8 @@
  * then a Walsh-Hadamard transform), a per-vector norm, a Lloyd-Max scalar
  * code and a 1-bit QJL sketch of the residual, and computes attention logits,
  * decode attention and top-k inner-product search directly from the packed
- * codes.
+ * codes.  A second stage-1 code rewrites the rotated vector in recursive
+ * polar form and codes its angles with per-level tables (tq_polar_*).
  *
  * Sources (web articles about Google's TurboQuant; they print no code):
  *  [E1] "TurboQuant explainer" (m.163.com), section "TurboQuant 怎么做的",
