@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const DArgs a) {
   constexpr int VTB = TILE * (VKB * DP / 8);
   constexpr int NT = CH / TILE;
   __shared__ float stat[QCHUNK][2];
-  __shared__ float vc[16];
+  __shared__ __half vch[16];
   __shared__ uint4 afrag[SC::FR / 4 * 32];
   // dynamic: K tiles (later reused for the weights), V tiles, norms, scores
   extern __shared__ __align__(16) uint8_t dsm[];
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const DArgs a) {
   const int t0 = chunk_id * CH;
   const int ntok = max(0, min(CH, L - t0));
   const int64_t vbase = (int64_t)bg * a.max_tokens;
-  if (threadIdx.x < (1 << VKB)) vc[threadIdx.x] = a.vcent[threadIdx.x];
+  if (threadIdx.x < (1 << VKB)) vch[threadIdx.x] = __float2half_rn(a.vcent[threadIdx.x]);
 
   if (ntok > 0) {  // stage codes and norms (whole tiles; max_tokens % 32 == 0)
     const int ntiles = (ntok + TILE - 1) / TILE;
@@ -326,50 +326,68 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const DArgs a) {
     const float nv = __half2float(nbuf[2][j]);
     wv[j] = value_weights(sl, stat, j, nv, a.veps, min(QCHUNK, a.group - QCHUNK * qc));
   }
+  // tokens past ntok up to the next multiple of 16 take part in the last MMA step with weight 0
+  // (their codes are staged: whole 32-token tiles)
+  for (int j = ntok + threadIdx.x; j < ((ntok + 15) & ~15); j += 128) wv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
 
-  // 3) value sum in the rotated domain.  Lane = bit position: coordinates 32w + lane
-  //    (w = 0..3), so one 16-byte broadcast load per plane brings the four words of a
-  //    token; warp wp takes tokens wp, wp + 4, ...; the warps' partial sums meet in
-  //    shared memory behind the weights (the K tiles are no longer read).
-  float acc[QCHUNK][4] = {};
-  auto vstep = [&](int j, const float4 ww) {
-    const uint8_t* tb = vbuf + (j >> 5) * VTB + (j & 31) * 16;
-    uint32_t wd[VKB][4];
+  // 3) value sum in the rotated domain on the tensor cores: o_rot[q][c] = sum_t w_{t,q} c[idx_{t,c}]
+  //    as mma.sync m16n8k16, A = centroids of 16 coordinates (rows) x 16 tokens in fp16, B = the
+  //    weights p n_v of those tokens for the query heads (columns; 4 of 8 used) in fp16, fp32
+  //    accumulation.  Block j covers coordinates 16j .. 16j + 15, so thread (g, t4) needs
+  //    coordinates 32w + g + 8k of each token: one shift and mask per plane word gives their
+  //    index bits, one byte each.  Warp wp takes the 16-token steps wp, wp + 4, ...
+  const int g = lane >> 2, t4 = lane & 3;
+  float acc[8][4] = {};
+  const float* wf = reinterpret_cast<const float*>(wv);
+  const int nstep = (ntok + 15) >> 4;
+  for (int st = warp; st < nstep; st += 4) {
+    const int tb0 = 16 * st + 2 * t4;  // this thread's tokens: tb0, tb0 + 1, tb0 + 8, tb0 + 9
+    uint32_t b0 = 0u, b1 = 0u;
+    if (g < QCHUNK) {
+      b0 = pack_half2(wf[4 * tb0 + g], wf[4 * (tb0 + 1) + g]);
+      b1 = pack_half2(wf[4 * (tb0 + 8) + g], wf[4 * (tb0 + 9) + g]);
+    }
+    if (a.veps > 0.f && __all_sync(FULL, (b0 | b1) == 0u)) continue;  // Sparse V: every weight dropped
+    uint32_t ib[4][4];  // [token][word]: byte k = index of coordinate 32 word + g + 8k
 #pragma unroll
-    for (int p = 0; p < VKB; ++p) {
-      const uint4 v = *reinterpret_cast<const uint4*>(tb + p * TILE * 16);
-      wd[p][0] = v.x;
-      wd[p][1] = v.y;
-      wd[p][2] = v.z;
-      wd[p][3] = v.w;
+    for (int tk = 0; tk < 4; ++tk) {
+      const int tok = tb0 + (tk & 1) + 8 * (tk >> 1);
+      const uint8_t* tb = vbuf + (tok >> 5) * VTB + (tok & 31) * 16;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) ib[tk][w] = 0u;
+#pragma unroll
+      for (int p = 0; p < VKB; ++p) {
+        const uint4 v = *reinterpret_cast<const uint4*>(tb + p * TILE * 16);
+        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) ib[tk][w] |= ((wd[w] >> g) & 0x01010101u) << p;
+      }
     }
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      int idx = 0;
-#pragma unroll
-      for (int p = 0; p < VKB; ++p) idx |= ((wd[p][w] >> lane) & 1u) << p;
-      const float cv = vc[idx];
-      acc[0][w] = fmaf(ww.x, cv, acc[0][w]);
-      acc[1][w] = fmaf(ww.y, cv, acc[1][w]);
-      acc[2][w] = fmaf(ww.z, cv, acc[2][w]);
-      acc[3][w] = fmaf(ww.w, cv, acc[3][w]);
+    for (int j = 0; j < 8; ++j) {
+      const int w = j >> 1, k0 = 2 * (j & 1);  // rows g and g + 8: bytes k0 and k0 + 1 of word w
+      auto val = [&](int tk, int k) { return vch[(ib[tk][w] >> (8 * k)) & 0xFFu]; };
+      const __half2 h0 = __halves2half2(val(0, k0), val(1, k0));
+      const __half2 h1 = __halves2half2(val(0, k0 + 1), val(1, k0 + 1));
+      const __half2 h2 = __halves2half2(val(2, k0), val(3, k0));
+      const __half2 h3 = __halves2half2(val(2, k0 + 1), val(3, k0 + 1));
+      const uint32_t af[4] = {*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
+                              *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3)};
+      mma_f16_16816(acc[j], af, b0, b1);
     }
-  };
-  if (a.veps > 0.f) {  // Sparse V: dropped tokens (all four weights zero) are skipped, uniformly over the warp
-    for (int j = warp; j < ntok; j += 4) {
-      const float4 ww = wv[j];
-      if (ww.x != 0.f || ww.y != 0.f || ww.z != 0.f || ww.w != 0.f) vstep(j, ww);
-    }
-  } else {
-#pragma unroll 2
-    for (int j = warp; j < ntok; j += 4) vstep(j, wv[j]);
   }
   float* red = reinterpret_cast<float*>(kbuf + CH * 16);  // [4 warps][QCHUNK][DP]
+  if (2 * t4 < QCHUNK) {  // D: rows g, g + 8 of block j; columns (query heads) 2 t4, 2 t4 + 1
 #pragma unroll
-  for (int qq = 0; qq < QCHUNK; ++qq)
-#pragma unroll
-    for (int w = 0; w < 4; ++w) red[(warp * QCHUNK + qq) * DP + 32 * w + lane] = acc[qq][w];
+    for (int j = 0; j < 8; ++j) {
+      float* r0 = red + (warp * QCHUNK + 2 * t4) * DP + 16 * j + g;
+      r0[0] = acc[j][0];
+      r0[DP] = acc[j][1];
+      r0[8] = acc[j][2];
+      r0[DP + 8] = acc[j][3];
+    }
+  }
   __syncthreads();
   const int c = threadIdx.x;
   float accs[4];
