@@ -4,7 +4,7 @@ tq_decode_attn; with v_eps > 0 the output lies within the Sparse V bound
 v_eps * sum_{p_t < v_eps} |v_hat_t| of both the oracle's full output and its
 Sparse V output (the kernel drops a subset of the oracle's tokens), plus the
 decode tolerance 2e-3 |o|.  Shapes cover the staged kernel (max_tokens a
-multiple of 32) and the plain one, several 512-token splits, ragged lengths
+multiple of 32) and the plain one, several 256-token splits, ragged lengths
 and GQA groups; a large softmax scale makes the attention peaked so that
 many tokens fall below v_eps."""
 import numpy as np

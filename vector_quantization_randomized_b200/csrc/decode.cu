@@ -7,7 +7,7 @@
 //   v_hat_t = n_v D H c_v[idx_t] / sqrt(d_pad).
 //
 // Split-K over tokens ("flash-decoding"): CTA (b, kv head, query chunk,
-// token chunk of 512) computes the logits of its 4 query heads with the
+// token chunk of 256) computes the logits of its 4 query heads with the
 // tensor-core code scan (scan.cuh), the chunk's softmax statistics, and the
 // value sum in the *rotated* domain, o_rot = sum_t p_t n_v,t c_v[idx_t]
 // (the rotation is linear, so it is applied once per output row instead of
@@ -25,7 +25,7 @@
 namespace {
 using namespace tqd;
 
-constexpr int CH = 512;  // tokens per split-K chunk
+constexpr int CH = 256;  // tokens per split-K chunk
 
 struct DArgs {
   const uint8_t* kcodes;
@@ -377,7 +377,8 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const DArgs a) {
       mma_f16_16816(acc[j], af, b0, b1);
     }
   }
-  float* red = reinterpret_cast<float*>(kbuf + CH * 16);  // [4 warps][QCHUNK][DP]
+  __syncthreads();  // every warp is done with the weights and the V tiles
+  float* red = reinterpret_cast<float*>(kbuf);  // [4 warps][QCHUNK][DP], over the weights
   if (2 * t4 < QCHUNK) {  // D: rows g, g + 8 of block j; columns (query heads) 2 t4, 2 t4 + 1
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -423,7 +424,7 @@ struct CArgs {
 
 __global__ void __launch_bounds__(128) combine_kernel(const CArgs a) {
   __shared__ float o[256];
-  __shared__ float wts[1024];
+  __shared__ float wts[2048];
   __shared__ float tot;
   const int64_t h = blockIdx.x;  // b * hq + head
   const int b = (int)(h / a.hq);
@@ -481,7 +482,9 @@ int launch_decode(const DArgs& a, int blocks, cudaStream_t st) {
   cudaError_t e;
   if (staged) {
     constexpr int smem = staged_smem<KB, SI, VKB>();
-    static_assert((CH / TILE) * TILE * (KB * 16 + 16 * SI) >= 2 * CH * 16, "weights and warp sums alias the K tiles");
+    static_assert((CH / TILE) * TILE * (KB * 16 + 16 * SI) >= CH * 16 &&
+                      (CH / TILE) * TILE * (KB * 16 + 16 * SI) >= 4 * QCHUNK * 128 * 4,
+                  "the weights and, after them, the warp sums alias the K tiles");
     e = cudaFuncSetAttribute(decode_staged_kernel<KB, SI, VKB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_decode_attn: %s", cudaGetErrorString(e));
     cfg.dynamicSmemBytes = smem;
@@ -577,7 +580,7 @@ int decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int ba
   int64_t prep_total = (int64_t)batch * n_kv_heads * nqc * tqd::prep_chunk_bytes(sh.fr);
   prep_total = (prep_total + 255) & ~(int64_t)255;
   const int nch = (int)std::max<int64_t>(1, (max_tokens + CH - 1) / CH);
-  if (nch > 1024) return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: max_tokens above 524288 is not supported");
+  if (nch > 2048) return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: max_tokens above 524288 is not supported");
   DArgs a;
   a.kcodes = static_cast<const uint8_t*>(kcodes);
   a.knorms = knorms;
