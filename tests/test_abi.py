@@ -151,3 +151,49 @@ def test_polar_sizes_and_validation():
     assert tq._lib.tq_polar_table_floats(128, 4) == -1
     bad = tq.tq_polar_params(128, 128, 4, 0, None, None)
     assert tq._lib.tq_polar_quantize(ctypes.byref(bad), None, 2, 1, 128, None, None, None) == tq.TQ_EINVAL
+
+
+def _fake_polar(**kw):
+    p = dict(d=128, d_pad=128, w=2)
+    p.update(kw)
+    buf = np.zeros(256, np.float32)
+    ptr = buf.ctypes.data
+    return tq.tq_polar_params(p["d"], p["d_pad"], p["w"], 0, ptr, ptr), buf
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d_pad=64), tq.TQ_EUNSUPPORTED),
+    (dict(d=0), tq.TQ_EINVAL),
+    (dict(d=129), tq.TQ_EINVAL),
+    (dict(w=0), tq.TQ_EINVAL),
+    (dict(w=4), tq.TQ_EINVAL),
+])
+def test_polar_validation_rejects_bad_params(kw, code):
+    st, keep = _fake_polar(**kw)
+    lib = tq._lib
+    p = ctypes.byref(st)
+    assert lib.tq_polar_quantize(p, keep.ctypes.data, tq.TQ_BF16, 10, 128, keep.ctypes.data, keep.ctypes.data,
+                                 None) == code
+    assert lib.tq_polar_dequantize(p, keep.ctypes.data, keep.ctypes.data, 10, keep.ctypes.data, 128, None) == code
+    assert lib.tq_polar_logits(p, keep.ctypes.data, 4, keep.ctypes.data, keep.ctypes.data, 10, 1,
+                               keep.ctypes.data, None) == code
+    assert tq.tq_last_error()
+
+
+def test_polar_validation_rejects_null_misaligned_and_sizes():
+    st, keep = _fake_polar()
+    lib = tq._lib
+    p = ctypes.byref(st)
+    ok = keep.ctypes.data  # 16-byte aligned host buffer: never dereferenced before validation fails
+    assert lib.tq_polar_quantize(p, None, tq.TQ_BF16, 10, 128, ok, ok, None) == tq.TQ_EINVAL
+    assert lib.tq_polar_quantize(p, ok, 9, 10, 128, ok, ok, None) == tq.TQ_EINVAL
+    assert lib.tq_polar_quantize(p, ok, tq.TQ_BF16, 10, 100, ok, ok, None) == tq.TQ_EINVAL  # ld < d
+    assert lib.tq_polar_quantize(p, ok + 4, tq.TQ_BF16, 10, 128, ok, ok, None) == tq.TQ_EINVAL
+    assert lib.tq_polar_quantize(p, ok, tq.TQ_BF16, -1, 128, ok, ok, None) == tq.TQ_EINVAL
+    assert lib.tq_polar_quantize(p, None, tq.TQ_BF16, 0, 128, None, None, None) == tq.TQ_OK  # nothing to do
+    assert lib.tq_polar_dequantize(p, ok + 8, ok, 10, ok, 128, None) == tq.TQ_EINVAL
+    assert lib.tq_polar_logits(p, ok, 0, ok, ok, 10, 1, ok, None) == tq.TQ_EINVAL
+    assert lib.tq_polar_logits(p, ok, 9, ok, ok, 10, 1, ok, None) == tq.TQ_EINVAL
+    assert lib.tq_polar_logits(p, ok, 4, ok, ok, 0, 1, ok, None) == tq.TQ_OK
+    null = tq.tq_polar_params(128, 128, 2, 0, None, None)
+    assert lib.tq_polar_logits(ctypes.byref(null), ok, 4, ok, ok, 10, 1, ok, None) == tq.TQ_EINVAL
