@@ -9,6 +9,8 @@
 * tq_polar_logits on oracle-made records: |l - l_oracle| <= 1e-4 |l| +
   1e-5 n ||q||, every group size 1..8, several KV heads, key counts that are
   not multiples of the 128-key block.
+* The bench's full launch (8 KV heads x 32768 keys, 32 query heads) at
+  w = 2 and 3: sampled keys' indices and norms, and their logits.
 """
 import numpy as np
 import pytest
@@ -122,3 +124,45 @@ def test_logits_d200():
     ref = polar.logits(q, D, enc["i1"], enc["ihi"], enc["norm_f16"], 2, tabs)
     tol = logit_tolerance(ref, enc["norm_f16"], q)
     assert np.all(np.abs(out.cpu().numpy() - ref) <= tol)
+
+
+@pytest.mark.parametrize("w", [2, 3])
+def test_layer_full_size_sampled(w):
+    """The bench's polar launch (8 KV heads x 32768 bf16 keys, 32 query heads,
+    GQA 4): indices and norms of 3000 sampled keys and of the last 64 against
+    the oracle, and every query head's logits of those keys against the
+    oracle's logits from its own encoding wherever the two encodings agree."""
+    H, T, d, G = 8, 32768, 128, 4
+    n = H * T
+    x = wl.kv_block(1, H, T, d, seed=wl.SEED_KEYS).reshape(n, d)
+    p = tq.PolarParams(d, w, seed=42)
+    D, tabs, d_pad = _oracle(d, w)
+    codes = torch.empty(p.code_bytes(n), dtype=torch.uint8, device="cuda")
+    norms = torch.empty(n, dtype=torch.int16, device="cuda")
+    tq.tq_polar_quantize(p, torch.from_numpy(x).to(torch.bfloat16).cuda(), codes, norms)
+    q = wl.queries(H * G, d, seed=wl.SEED_QUERIES)
+    lg = torch.empty((H * G, T), dtype=torch.float32, device="cuda")
+    tq.tq_polar_logits(p, dev(q.astype(np.float32)), G, codes, norms, T, H, lg)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([np.random.default_rng(w).integers(0, n, 3000), np.arange(n - 64, n)]))
+    rb = polar.record_bytes(d_pad, w)
+    recs = codes.cpu().numpy().reshape(n, rb)[rows]
+    i1, ihi = polar.unpack(recs.ravel(), rows.size, w, d_pad)
+    nn = norms.cpu().numpy().view(np.float16)[rows]
+    xin = torch.from_numpy(x[rows]).to(torch.bfloat16).float().numpy().astype(np.float64)
+    enc = polar.encode(xin, D, w, tabs)
+    f1, fl = polar.boundary_flags(enc, w, d_pad, tabs)
+    same = np.all(i1 == enc["i1"], axis=1)
+    assert not np.any((i1 != enc["i1"]) & ~f1)
+    for a, b, f in zip(ihi, enc["ihi"], fl):
+        assert not np.any((a != b) & ~f)
+        same &= np.all(a == b, axis=1)
+    assert np.all((nn == enc["norm_f16"]) | f16_neighbours(nn, enc["norm_f16"]))
+    same &= nn == enc["norm_f16"]
+    got = lg.cpu().numpy().astype(np.float64)
+    for h in range(H * G):
+        sel = np.flatnonzero((rows // T == h // G) & same)
+        ref = polar.logits(q[h:h + 1], D, enc["i1"][sel], [a[sel] for a in enc["ihi"]], enc["norm_f16"][sel], w,
+                           tabs)[0]
+        tol = logit_tolerance(ref[None, :], enc["norm_f16"][sel], q[h:h + 1])[0]
+        assert np.all(np.abs(got[h, rows[sel] % T] - ref) <= tol), h
