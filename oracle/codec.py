@@ -102,7 +102,7 @@ def encode(x, D, centroids, thresholds, S=None):
 
 
 def boundary_flags(enc, thresholds, S=None, rel=1e-6):
-    """Decisions that lie within `rel` of a boundary (spec tolerance band).
+    """Decisions that lie within `rel` of a boundary (the parity tolerance band).
 
     * index j of a vector: |y_j - t_l| <= rel * max(|t_l|, 1/sqrt(d_pad)) for some l
       (the scale is floored at the coordinate standard deviation because every

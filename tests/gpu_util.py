@@ -53,7 +53,7 @@ def f16_neighbours(a, b):
 def compare_codes(op, x, codes, norms, rnorms):
     """Compare GPU codes with the oracle's encoding of the same inputs.
 
-    Bit-exact except decisions inside the spec band (flags); a vector
+    Bit-exact except decisions inside the tolerance band (flags); a vector
     whose index decision was flagged *and* differs has a different residual,
     so its signs and residual norm are not comparable and are counted instead.
     Returns a dict of counts; raises AssertionError on any unflagged mismatch.

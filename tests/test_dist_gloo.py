@@ -2,7 +2,7 @@
 
 * the plumbing each rank runs around the timed region — barrier, maximum of
   the per-rank times over the ranks, whole-job weak-scaling throughput;
-* the reference arm launched the way the driver launches every arm
+* the reference arm launched as a multi-GPU run is launched
   (torch.distributed.run, 2 processes, 127.0.0.1): rank 0 alone runs and
   prints one JSON line, the other rank exits 0 without work.
 """
