@@ -337,8 +337,9 @@ int64_t tq_polar_code_bytes(int d_pad, int w, int64_t n_vec);
 
 /*
  * tq_polar_quantize - encode n_vec vectors (x: device, rows of d elements of
- *   dtype, stride ld elements; 16-byte alignment as tq_quantize).  codes:
- *   device, tq_polar_code_bytes bytes, 16-byte aligned; norms: device fp16.
+ *   dtype, stride ld elements; x, ld*elem_size and d*elem_size 16-byte
+ *   aligned, as tq_quantize).  codes: device, tq_polar_code_bytes bytes,
+ *   16-byte aligned; norms: device fp16.
  */
 int tq_polar_quantize(const tq_polar_params* p, const void* x, int dtype, int64_t n_vec, int64_t ld,
                       void* codes, uint16_t* norms, tq_stream_t stream);

@@ -197,3 +197,12 @@ def test_polar_validation_rejects_null_misaligned_and_sizes():
     assert lib.tq_polar_logits(p, ok, 4, ok, ok, 0, 1, ok, None) == tq.TQ_OK
     null = tq.tq_polar_params(128, 128, 2, 0, None, None)
     assert lib.tq_polar_logits(ctypes.byref(null), ok, 4, ok, ok, 10, 1, ok, None) == tq.TQ_EINVAL
+
+
+def test_polar_quantize_rejects_row_length_off_16_bytes():
+    """d * element size must be a multiple of 16 bytes (the kernel loads groups of 4 elements)."""
+    lib = tq._lib
+    for d, dtype, code in ((6, tq.TQ_F32, tq.TQ_EINVAL), (100, tq.TQ_BF16, tq.TQ_EINVAL), (10, tq.TQ_F32, tq.TQ_EINVAL)):
+        st, keep = _fake_polar(d=d)
+        ok = keep.ctypes.data
+        assert lib.tq_polar_quantize(ctypes.byref(st), ok, dtype, 10, 128, ok, ok, None) == code, (d, dtype)

@@ -454,8 +454,9 @@ extern "C" int tq_polar_quantize(const tq_polar_params* p, const void* x, int dt
   if (!x || !codes || !norms) return set_error(TQ_EINVAL, "tq_polar_quantize: NULL pointer argument");
   if (ld < p->d) return set_error(TQ_EINVAL, "tq_polar_quantize: ld < d");
   const int es = dtype == TQ_F32 ? 4 : 2;
-  if (!aligned(x, 16) || ((ld * es) % 16) != 0 || !aligned(codes, 16) || !aligned(norms, 2))
-    return set_error(TQ_EINVAL, "tq_polar_quantize: x, ld*elem and codes must be 16-byte aligned");
+  if (!aligned(x, 16) || ((ld * es) % 16) != 0 || ((int64_t)p->d * es) % 16 != 0 || !aligned(codes, 16) ||
+      !aligned(norms, 2))
+    return set_error(TQ_EINVAL, "tq_polar_quantize: x, ld*elem, d*elem and codes must be 16-byte aligned");
   PArgs a{};
   a.x = static_cast<const uint8_t*>(x);
   a.n_vec = n_vec;
