@@ -2,7 +2,8 @@
 not come from it: the transform's exact inverse, the level-2 angle law's
 Lloyd-Max fixed point in closed form, Monte-Carlo angle laws of rotated
 Gaussian vectors against the Beta law, nearest-centroid decisions by brute
-force, the bit layout on a hand-made example, and <q, x_hat> = logit."""
+force, the bit layout on a hand-made example, <q, x_hat> = logit, and the
+stored angle tables against a 30-digit Newton solution (mpmath)."""
 import math
 
 import numpy as np
@@ -137,3 +138,33 @@ def test_distortion_falls_with_bits_and_zero_vector():
         assert np.all(xr[0] == 0) and enc["norm"][0] == 0
         errs.append(np.mean(np.sum((xr[1:] - x[1:]) ** 2, 1) / np.sum(x[1:] ** 2, 1)))
     assert errs[0] > errs[1] > errs[2] and errs[2] < 0.05
+
+
+def _mp_angle_fixed_point(level, L, start):
+    """Lloyd-Max on (sin psi cos psi)^(k-1) over [0, pi/2] by Newton in 30 digits, mpmath quadrature."""
+    import mpmath as mp
+    mp.mp.dps = 30
+    k = 1 << (level - 1)
+    f = lambda t: (mp.sin(t) * mp.cos(t)) ** (k - 1)
+    half = L // 2
+    q = mp.pi / 4
+
+    def residual(*up):  # centroids above pi/4; the law is symmetric about pi/4
+        c = [2 * q - x for x in reversed(up)] + list(up)
+        e = [mp.mpf(0)] + [(c[j] + c[j + 1]) / 2 for j in range(L - 1)] + [2 * q]
+        return [c[j] - mp.quad(lambda t: t * f(t), [e[j], e[j + 1]]) / mp.quad(f, [e[j], e[j + 1]])
+                for j in range(half, L)]
+
+    sol = mp.findroot(residual, [mp.mpf(x) for x in start[half:]], tol=mp.mpf(10) ** -26)
+    up = np.array([float(x) for x in (sol if hasattr(sol, "__len__") else [sol])])
+    return np.concatenate([math.pi / 2 - up[::-1], up])
+
+
+@pytest.mark.parametrize("level,L", [(2, 2), (2, 4), (4, 4), (7, 2), (7, 4)])
+def test_angle_tables_match_high_precision(level, L):
+    """The stored fp32 angle centroids are the fp32 rounding of a 30-digit Newton
+    solution of the level's Lloyd-Max conditions (mpmath quadrature of the density)."""
+    c, _ = polar.lloyd_max_angle(level, L)
+    ref = _mp_angle_fixed_point(level, L, c)
+    assert np.max(np.abs(c - ref)) < 1e-11
+    assert np.array_equal(c.astype(np.float32), ref.astype(np.float32))
