@@ -268,3 +268,31 @@ def unpack(buf, n, w, d_pad):
         ihi.append(ix)
         cnt //= 2
     return i1, ihi
+
+
+# ---- QJL stage on the polar residual --------------------------------------------
+# "TurboQuant explainer" (m.163.com), "第二步：QJL" and "合起来": the residual of
+# stage 1 is JL-projected and kept as sign bits, and the estimator
+# E[<y, Q^-1(Q(x))>] = <y, x> is unbiased; b - 1 bits of stage 1 plus 1 bit.
+# Here stage 1 is the polar code: r = y - y_hat with y_hat the unit-radius
+# reconstruction from the stored tables.
+
+def encode_prod(x, D, w, S, tabs=None):
+    """Polar stage 1 plus the QJL stage: adds y_hat, r, gamma (fp64 and fp16), z = S r, signs [z >= 0]."""
+    enc = encode(x, D, w, tabs)
+    yh = decode_unit(enc["i1"], enc["ihi"], w, D.shape[0], tabs)
+    r = enc["y"] - yh
+    gamma = np.sqrt(np.sum(r * r, axis=1))
+    z = r @ np.asarray(S, dtype=np.float64).T
+    enc.update(yhat=yh, r=r, gamma=gamma, rnorm_f16=gamma.astype(np.float16), z=z, signs=(z >= 0).astype(np.uint8))
+    return enc
+
+
+def logits_prod(q, D, S, yhat, signs, norm, gamma, m):
+    """l[h, k] = n_k (<q~_h, y_hat_k> + gamma_k sqrt(pi/2)/m <S q~_h, 2 s_k - 1>), q~ = H D q / sqrt(d_pad)."""
+    d_pad = D.shape[0]
+    qt = codec.rotate(codec.pad(q, d_pad), D)
+    u = qt @ np.asarray(S, dtype=np.float64).T
+    pm = 2.0 * np.asarray(signs, dtype=np.float64) - 1.0
+    corr = (u @ pm.T) * (math.sqrt(math.pi / 2.0) / m) * np.asarray(gamma, dtype=np.float64)[None, :]
+    return (qt @ np.asarray(yhat, dtype=np.float64).T + corr) * np.asarray(norm, dtype=np.float64)[None, :]

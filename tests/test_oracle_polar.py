@@ -168,3 +168,50 @@ def test_angle_tables_match_high_precision(level, L):
     ref = _mp_angle_fixed_point(level, L, c)
     assert np.max(np.abs(c - ref)) < 1e-11
     assert np.array_equal(c.astype(np.float32), ref.astype(np.float32))
+
+
+@pytest.mark.parametrize("w", [1, 2])
+def test_prod_stage_unbiased_over_S_with_its_variance(w):
+    """QJL on the polar residual: over Gaussian S the estimate averages to <q, x>
+    with variance n^2 ((pi/2) gamma^2 ||q~||^2 - <q~, r>^2) / m."""
+    from oracle.params import gaussian_normals_f64
+    d, m, N = 128, 128, 3000
+    rng = np.random.default_rng(20 + w)
+    x = rng.standard_normal((1, d)) * 2.0
+    q = rng.standard_normal((1, d))
+    D = params.sign_flips(13, d)
+    tabs = polar.tables(d, w)
+    vals = []
+    for s in range(N):
+        S = gaussian_normals_f64(3000 + s, m, d)
+        enc = polar.encode_prod(x, D, w, S, tabs)
+        vals.append(polar.logits_prod(q, D, S, enc["yhat"], enc["signs"], enc["norm"], enc["gamma"], m)[0, 0])
+    vals = np.array(vals)
+    qt = codec.rotate(q, D)[0]
+    n, g, r = enc["norm"][0], enc["gamma"][0], enc["r"][0]
+    var = n * n * ((math.pi / 2) * g * g * (qt @ qt) - (qt @ r) ** 2) / m
+    assert abs(vals.mean() - float(q[0] @ x[0])) < 4 * math.sqrt(var / N)
+    assert abs(vals.var() / var - 1) < 4 * math.sqrt(2.0 / N)
+
+
+def test_prod_stage_removes_the_stage1_shrinkage():
+    """Over random rotations the polar stage-1 estimate alone shrinks <q, x> (its
+    reconstruction is shorter on average than y along y); adding the QJL stage
+    makes the estimate unbiased over (D, S)."""
+    from oracle.params import gaussian_normals_f64
+    d, m, N, w = 128, 128, 1500, 1
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((1, d))
+    q = x + 0.3 * rng.standard_normal((1, d))
+    tabs = polar.tables(d, w)
+    s1, s2 = [], []
+    for s in range(N):
+        D = params.sign_flips(5000 + s, d)
+        S = gaussian_normals_f64(7000 + s, m, d)
+        enc = polar.encode_prod(x, D, w, S, tabs)
+        s1.append(polar.logits(q, D, enc["i1"], enc["ihi"], enc["norm"], w, tabs)[0, 0])
+        s2.append(polar.logits_prod(q, D, S, enc["yhat"], enc["signs"], enc["norm"], enc["gamma"], m)[0, 0])
+    truth = float(q[0] @ x[0])
+    s1, s2 = np.array(s1), np.array(s2)
+    assert s1.mean() < truth - 8 * s1.std() / math.sqrt(N)              # biased low
+    assert abs(s2.mean() - truth) < 4 * s2.std() / math.sqrt(N)           # unbiased
