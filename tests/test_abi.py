@@ -122,7 +122,7 @@ def test_validation_rejects_null_and_misaligned():
     assert lib.tq_code_bytes(-1, 1, 1, 1) == -1
 
 
-@pytest.mark.parametrize("d_pad", [128, 256])
+@pytest.mark.parametrize("d_pad", [128, 256, 1024, 4096])
 @pytest.mark.parametrize("w", [1, 2, 3])
 def test_polar_tables_match_oracle(d_pad, w):
     """The library's angle tables (C++ Gauss-Legendre Lloyd iteration) equal the oracle's
