@@ -392,7 +392,7 @@ def logits_isolated(torch, tq, wk, reps_min=8):
 def cpu_oracle_layer(sample_tokens=16384):
     """The oracle (fp64 numpy, as it stands) on a bounded sample of the layer workload:
     all 8 heads x `sample_tokens` tokens, b = 3 and 4, quantize K and V + logits."""
-    from vector_quantization_randomized_b200 import workloads as wl
+    import workloads as wl
     from oracle import codec, estimate
     from oracle.codebook import stored_codebook
     from oracle.params import sign_flips, qjl_matrix
@@ -656,7 +656,7 @@ def main():
     import torch
     world, rank, local = dist_setup(args)
     import vector_quantization_randomized_b200 as tq
-    from vector_quantization_randomized_b200 import workloads as wl
+    import workloads as wl
     if args.workload != "layer":
         return run_secondary(args, world, rank, local, torch, tq, wl)
     peak, peak_kind = measured_peaks()

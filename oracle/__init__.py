@@ -7,7 +7,7 @@ leg of ``bench.py`` may import or run it.
 
 It shares no code with ``vector_quantization_randomized_b200`` (no kernels,
 headers, helpers, tables or constant generators).  The seeded *input*
-generators (``vector_quantization_randomized_b200.workloads``) hold none of the
+generators (the top-level ``workloads`` module) hold none of the
 method's arithmetic and are the only thing both sides use.
 
 Sources, by page and section (the pages are web articles about Google's

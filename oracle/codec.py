@@ -117,16 +117,18 @@ def boundary_flags(enc, thresholds, S=None, rel=1e-6):
     scale = np.maximum(np.abs(t), 1.0 / np.sqrt(d_pad))
     idx_flag = np.any(np.abs(y[:, :, None] - t[None, None, :]) <= rel * scale[None, None, :], axis=2)
 
-    def f16_tie(v):
-        lo = (v * (1 - rel)).astype(np.float16)
-        hi = (v * (1 + rel)).astype(np.float16)
-        return lo != hi
-
-    flags = dict(idx=idx_flag, norm=f16_tie(enc["norm"]), rnorm=f16_tie(enc["gamma"]))
+    flags = dict(idx=idx_flag, norm=f16_tie_flags(enc["norm"], rel), rnorm=f16_tie_flags(enc["gamma"], rel))
     if S is not None:
         Sn = np.sqrt(np.sum(np.asarray(S, dtype=np.float64) ** 2, axis=1))
         flags["signs"] = np.abs(enc["z"]) <= rel * Sn[None, :] * enc["gamma"][:, None]
     return flags
+
+
+def f16_tie_flags(v, rel=1e-6):
+    """Values within `rel` (relative) of a half-precision rounding tie:
+    fp16(v(1-rel)) != fp16(v(1+rel)), so either rounding of v is acceptable."""
+    v = np.asarray(v, dtype=np.float64)
+    return (v * (1 - rel)).astype(np.float16) != (v * (1 + rel)).astype(np.float16)
 
 
 def code_bytes(d_pad, kb, m, n_vec):

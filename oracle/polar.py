@@ -6,7 +6,7 @@ rotation the vector is rewritten in polar form, a radius and angles; in high
 dimension the angles follow a known, highly concentrated Beta law, so they are
 coded with fixed, precomputed tables and no normalisation constant is stored.
 
-The pages give no formulas.  Readings taken here (each listed in the design doc):
+The pages give no formulas.  Readings taken here:
 
 * Rotation: the same sign flips and Walsh-Hadamard rotation as the scalar code
   (codec.rotate) of the unit vector x/||x||; the radius kept is ||x|| (fp16),

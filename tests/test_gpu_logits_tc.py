@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import vector_quantization_randomized_b200 as tq
-from vector_quantization_randomized_b200 import workloads as wl
+import workloads as wl
 from oracle import estimate
 from gpu_util import make_pair, oracle_codes, logit_tolerance
 

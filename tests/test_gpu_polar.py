@@ -17,8 +17,8 @@ import pytest
 import torch
 
 import vector_quantization_randomized_b200 as tq
-from vector_quantization_randomized_b200 import workloads as wl
-from oracle import polar
+import workloads as wl
+from oracle import codec, polar
 from oracle.params import sign_flips
 from gpu_util import f16_neighbours, logit_tolerance
 
@@ -52,7 +52,8 @@ def _quantize_check(x_host, dtype, d, w):
         flagged += int(f.sum())
         mismatched += int((a != b).sum())
     nn = norms.cpu().numpy().view(np.float16)
-    assert np.all((nn == enc["norm_f16"]) | f16_neighbours(nn, enc["norm_f16"]))
+    tie = codec.f16_tie_flags(enc["norm"])
+    assert np.all((nn == enc["norm_f16"]) | (tie & f16_neighbours(nn, enc["norm_f16"])))
     assert mismatched <= flagged
     return mismatched, flagged
 
@@ -157,7 +158,8 @@ def test_layer_full_size_sampled(w):
     for a, b, f in zip(ihi, enc["ihi"], fl):
         assert not np.any((a != b) & ~f)
         same &= np.all(a == b, axis=1)
-    assert np.all((nn == enc["norm_f16"]) | f16_neighbours(nn, enc["norm_f16"]))
+    tie = codec.f16_tie_flags(enc["norm"])
+    assert np.all((nn == enc["norm_f16"]) | (tie & f16_neighbours(nn, enc["norm_f16"])))
     same &= nn == enc["norm_f16"]
     got = lg.cpu().numpy().astype(np.float64)
     for h in range(H * G):

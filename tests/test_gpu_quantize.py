@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import vector_quantization_randomized_b200 as tq
-from vector_quantization_randomized_b200 import workloads as wl
+import workloads as wl
 from gpu_util import make_pair, gpu_quantize, compare_codes
 
 pytestmark = pytest.mark.gpu

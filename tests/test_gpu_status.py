@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import vector_quantization_randomized_b200 as tq
-from vector_quantization_randomized_b200 import workloads as wl
+import workloads as wl
 
 pytestmark = pytest.mark.gpu
 
