@@ -87,3 +87,10 @@ def test_ring_wraps_many_items_per_cta():
         got = out[h * G:(h + 1) * G].cpu().numpy().astype(np.float64)
         tol = logit_tolerance(ref, norms[h * T:(h + 1) * T], qh)
         assert np.all(np.abs(got - ref) <= tol), h
+
+
+@pytest.mark.parametrize("bits,n_heads,n_keys", [(4, 700, 64), (3, 600, 128)])
+def test_many_heads_per_cta(bits, n_heads, n_keys):
+    """Short sequences over many KV heads: a CTA's item range crosses several heads,
+    so the in-kernel query preparation refills its two B-image slots in turn."""
+    _check(bits, tq.TQ_MODE_PROD, n_heads, 4, n_keys, seed=5)

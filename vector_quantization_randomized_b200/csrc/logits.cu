@@ -276,9 +276,7 @@ bool scan_supported(int dp, int kb) { return (dp == 128 && kb >= 1 && kb <= 3) |
 
 int64_t prep_chunk_bytes_max(int dp, int kb, int m) {
   const tqd::ScanShape sh(dp, kb, m);
-  int64_t b = tqd::prep_chunk_bytes(sh.fr);
-  if (dp == 128) b = std::max<int64_t>(b, tqd::prep_chunk_bytes_tc(tqd::tc_kchunks(kb, m)));
-  return b;
+  return tqd::prep_chunk_bytes(sh.fr);
 }
 }  // namespace tq
 
@@ -317,14 +315,18 @@ extern "C" int tq_logits_ld(const tq_params* p, const float* q, int n_q, int gro
   const tqd::ScanShape sh(p->d_pad, kb, m);
   const int nqc = (group + tqd::QCHUNK - 1) / tqd::QCHUNK;
   const int chunks = n_kv_heads * nqc;
-  const bool tc = logits_tc_supported(p->d_pad, kb, m, group, n_keys, norms, rnorms);
-  const int kc = tqd::tc_kchunks(kb, m);
-  const int64_t chunk_bytes = tc ? tqd::prep_chunk_bytes_tc(kc) : tqd::prep_chunk_bytes(sh.fr);
-  const int64_t need = (int64_t)chunks * chunk_bytes;
+  const int64_t need = (int64_t)chunks * tqd::prep_chunk_bytes(sh.fr);
   if (workspace_bytes < need)
     return set_error(TQ_EINVAL, "tq_logits: workspace too small (%lld < %lld bytes)", (long long)workspace_bytes,
                      (long long)need);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (logits_tc_supported(p->d_pad, kb, m, group, n_keys, norms, rnorms)) {
+    // tensor-memory scan with the query preparation inside the kernel: the workspace is not used
+    rc = launch_logits_tc(kb, m, q, p->d, p->centroids, p->signs_D, p->S, codes, norms, rnorms, n_keys, n_kv_heads,
+                          group, logits, ld_logits, st);
+    if (rc == TQ_OK) clear_error();
+    return rc;
+  }
   tqd::PrepArgs pa;
   pa.q = q;
   pa.d = p->d;
@@ -339,16 +341,8 @@ extern "C" int tq_logits_ld(const tq_params* p, const float* q, int n_q, int gro
   pa.S = p->S;
   pa.out = static_cast<uint8_t*>(workspace);
   pa.fr = sh.fr;
-  pa.layout = tc ? 1 : 0;
-  pa.kc = kc;
   rc = launch_prep(pa, st);
   if (rc) return rc;
-  if (tc) {
-    rc = launch_logits_tc(kb, m, codes, norms, rnorms, n_keys, n_kv_heads, group, pa.out, chunk_bytes, logits,
-                          ld_logits, st);
-    if (rc == TQ_OK) clear_error();
-    return rc;
-  }
 
   LArgs a;
   a.codes = static_cast<const uint8_t*>(codes);

@@ -2,32 +2,38 @@
 // query heads per KV head ("TurboQuant explainer" (m.163.com), "第二步：QJL"
 // estimator; "速度": logits straight from the compressed keys).
 //
-// The integer form of the estimator is the one in scan.cuh: every product is
-// "integer weight x code bit", the weights split into signed base-256 digits.
-// Here the code bits are the A operand of tcgen05.mma kind::i8 (u8 x s8 ->
-// s32), held in tensor memory, and the prepared query digits are the B operand
-// in shared memory:
+// Integer form of the estimator (scan.cuh): every product is "integer weight x
+// code bit".  Weights 2 alpha_T q_rot_j (Walsh plane T of the codebook) and
+// 2 u_i (u = S q_rot) are scaled by a per-query power of two to integers below
+// 2^23, shifted left by 7 - c for bit class c = coordinate % 8 and split into
+// four signed base-256 digits.  The code bits are the A operand of
+// tcgen05.mma kind::i8 (u8 x s8 -> s32), held in tensor memory:
 //
-//   A[key][chunk 8P + c][4w + b] = byte b of (plane word w of plane P) & (1 << c)
-//                                = 2^c * bit(coordinate 32w + 8b + c),
+//   A[key][K = 128P + 16c + 4w + b] = byte b of (word w of plane P) & (1 << c)
+//                                   = 2^c * bit(coordinate 32w + 8b + c),
 //
-// i.e. bit class c of a plane is the plane's four words masked with
-// 0x01010101 << c, one 32-bit tensor-memory column per masked word; the B
-// image (prep.cu) holds at the same K position the digit of the weight of
-// that coordinate, pre-shifted by 7 - c.  One MMA of M = 128 keys, N = 32
-// (4 queries x 4 digits x {centroid, sign}), K = 32 bytes.
+// one 32-bit tensor-memory column per masked word.  The digits are the B
+// operand in shared memory, 16 rows = 4 queries x 4 digits.  Centroid planes
+// and the sign plane go to separate N = 16 MMAs with their own accumulator
+// columns, so no MMA multiplies a zero block.  Per 128-key item: 4 NT centroid
+// MMAs and 4 sign MMAs (M = 128, N = 16, K = 32 bytes).
 //
-// Warp-specialised pipeline, one persistent CTA per SM over (KV head, 128-key
-// tile) items, all hand-offs on mbarriers (waits bounded):
-//   warp 0      bulk copies of the code tiles and norms into a ring of shared-memory stages;
-//   warps 1-4   tcgen05.mma issue: two pairs take alternate items, each warp of a
-//               pair every other K step into its own partial accumulator of a ring
-//               of accumulator sets (one thread issues an MMA only every ~50
-//               cycles and waits for them to be taken before its next item); the
-//               pair that meets a new KV head first loads its B image (bulk copy);
-//   8 warps     expansion: stage -> masked words -> tcgen05.st into one of two or
-//               three A buffers in tensor memory (warp = lane quadrant x 4 bit classes);
-//   8 warps     epilogue: tcgen05.ld of the partial accumulators, digit
+// The query preparation (rotation, projection, scaling, digit split) runs
+// inside this kernel: each CTA builds the B image of the KV heads it scans, so
+// tq_logits is one launch and needs no workspace on this path.
+//
+// Warp roles, one persistent CTA per SM over a contiguous range of
+// (KV head, 128-key tile) items, all hand-offs on mbarriers with bounded waits:
+//   warp 0      bulk copies of code tiles and norms into a ring of stages;
+//   warps 1-4   MMA issue: two pairs take alternate items; each warp of a pair
+//               issues every other K step of the item into its own partial
+//               accumulator.  The loops are warp-uniform and one lane, chosen
+//               by elect.sync, issues, with the descriptors of a whole item
+//               unrolled from two base values;
+//   warps 5-12  expansion: stage -> masked words -> tcgen05.st into one of two
+//               or three A buffers (warp = lane quadrant x 4 bit classes);
+//   warps 13-20 query preparation into a ring of two B images, then the
+//               epilogue: tcgen05.ld of the partial accumulators, digit
 //               combination, norms, logits (warp = lane quadrant x 2 queries).
 #include <cuda_runtime.h>
 
@@ -43,77 +49,261 @@ namespace {
 using namespace tqd;
 
 constexpr int TK = 128;  // keys per item (MMA M)
-constexpr int MAX_STAGES = 16;
-constexpr int HDR = 1024;  // barriers + tensor-memory base, ahead of the B image
+constexpr int DP = 128;
+constexpr int MAX_STAGES = 12;
 
 struct TArgs {
   const uint8_t* codes;
   const uint16_t* norms;
   const uint16_t* rnorms;
-  int64_t n_keys;        // keys per KV head, a multiple of 32
-  int group;             // query heads per KV head, 1..4
-  int tb;                // bytes of one 32-key code tile
-  int tiles_per_head;    // ceil(n_keys / 128)
-  int64_t n_items;       // n_kv_heads * tiles_per_head
-  const uint8_t* prep;   // per KV head: B image + per-query scalars
-  int64_t prep_bytes;
+  int64_t n_keys;      // keys per KV head, a multiple of 32
+  int group;           // query heads per KV head, 1..4
+  int tb;              // bytes of one 32-key code tile
+  int tiles_per_head;  // ceil(n_keys / 128)
+  int64_t n_items;     // n_kv_heads * tiles_per_head
+  const float* q;      // [n_kv_heads * group][d] fp32
+  int d;
+  int kb;
+  int m;
+  const float* cent;   // codebook centroids (2^kb)
+  const int8_t* D;     // sign flips [128]
+  const uint16_t* S;   // QJL matrix, fp16 [m][128]
   float* logits;
-  int64_t ld;            // logits row stride
-  float kappa;           // sqrt(pi/2) / m
-  int stages;            // ring stages (<= MAX_STAGES)
+  int64_t ld;          // logits row stride
+  float kappa;         // sqrt(pi/2) / m
+  int stages;          // ring stages (<= MAX_STAGES)
 };
 
 template <int KB, int SI>
 struct TL {
   static constexpr int NT = KB == 1 ? 1 : (KB == 2 ? 2 : 4);  // Walsh planes
   static constexpr int NP = NT + SI;                          // planes in A
-  static constexpr int KC = 8 * NP;                           // 16-byte K chunks
-  static constexpr int ACOLS = 4 * KC;                        // tensor-memory columns of one A buffer
-  static constexpr int KSTEPS = ACOLS / 8;                    // MMAs per item (K = 32 bytes each)
-  static constexpr int BBYTES = 512 * KC;                     // B image
-  static constexpr int TILEB = 32 * 16 * (KB + SI);           // one 32-key code tile
-  static constexpr int NORMB = 256 * (1 + SI);                // fp16 norms (+ residual norms) of 128 keys
-  static constexpr int STAGE = 4 * TILEB + NORMB;             // one item: code tiles, then norms
-  // Two partial accumulators per item, one per MMA-issuing warp: a thread issues a
-  // tcgen05.mma only every ~50 cycles while the tensor pipe finishes one of these
-  // in ~17, so two warps issue in parallel (K steps j, j + 2, ...) and the epilogue
-  // adds the two partial sums (exact int32).  NB accumulator sets in a ring, so the
-  // MMAs of item i wait for the epilogue of item i - NB, not i - 2.
-  static constexpr int NACC = 2;
-  static constexpr int NISS = 2 * NACC;  // two pairs of issuing warps, alternate items
-  static constexpr int COLS = 512;
-  // A buffers: three where they fit beside three accumulator sets (b <= 3), else two;
-  // the expansion of item i then waits for the MMAs of item i - NA
-  static constexpr int NA = 3 * ACOLS + 3 * 32 * NACC <= COLS ? 3 : 2;
-  static constexpr int NB = (COLS - NA * ACOLS) / (32 * NACC) < 4 ? (COLS - NA * ACOLS) / (32 * NACC) : 4;
-  static_assert(NB >= 2 && 32 * NACC * NB + NA * ACOLS <= COLS, "tensor-memory budget");
-  static constexpr int W_EXP0 = 1 + NISS, W_EPI0 = W_EXP0 + 8;  // first expansion / epilogue warp
-  static constexpr int NTHREADS = (W_EPI0 + 8) * 32;
-  static_assert(KSTEPS >= NACC, "every accumulator is written by each item");
-  static constexpr int smem(int stages) { return HDR + BBYTES + stages * STAGE; }
+  static constexpr int ACOLS = 32 * NP;                       // tensor-memory columns of one A buffer
+  static constexpr int CSTEPS = 4 * NT;                       // centroid MMAs per item (K = 32 bytes each)
+  static constexpr int SSTEPS = 4 * SI;                       // sign MMAs per item
+  // B image of one KV head: 4 per-query float4 scalars, then the centroid digits
+  // (16 rows x NT*128 bytes) and the sign digits (16 rows x 128 bytes), each in the
+  // canonical K-major layout: 16-byte K chunk kc at kc*256, 8-row group g at g*128.
+  static constexpr int IMG_C = 64;
+  static constexpr int IMG_S = 64 + NT * 2048;
+  static constexpr int IMG = (64 + NP * 2048 + 127) / 128 * 128;
+  static constexpr int TILEB = 32 * 16 * (KB + SI);  // one 32-key code tile
+  static constexpr int NORMB = 256 * (1 + SI);       // fp16 norms (+ residual norms) of 128 keys
+  static constexpr int STAGE = 4 * TILEB + NORMB;    // one item: code tiles, then norms
+  static constexpr int ACC = 64;                     // accumulator set: 2 partials x (16 centroid + 16 sign)
+  static constexpr int NA = (3 * ACOLS + 3 * ACC <= 512) ? 3 : 2;
+  static constexpr int NB0 = (512 - NA * ACOLS) / ACC;
+  static constexpr int NB = NB0 < 4 ? NB0 : 4;
+  static_assert(NB >= 2 && NA * ACOLS + NB * ACC <= 512, "tensor-memory budget");
+  static constexpr int W_EXP0 = 5, W_EPI0 = 13;
+  static constexpr int NTHREADS = 21 * 32;
+  static constexpr int OFF_IMG = 1024;
+  static constexpr int OFF_PREP = OFF_IMG + 2 * IMG;      // q_rot float4[128], u float4[128], partial u [2][128]
+  static constexpr int OFF_RING = OFF_PREP + 4 * 128 * 16;
+  static constexpr int smem(int stages) { return OFF_RING + stages * STAGE; }
 };
+
+// frexpf's exponent (x = f 2^e, 0.5 <= f < 1) and 2^k from the fp32 bit pattern
+// for normal values (exact), the library calls otherwise.
+__device__ __forceinline__ int exponent_of(float x) {
+  const uint32_t b = __float_as_uint(x) & 0x7FFFFFFFu;
+  if (b >= 0x00800000u && b < 0x7F800000u) return (int)(b >> 23) - 126;
+  int e;
+  frexpf(x, &e);
+  return e;
+}
+__device__ __forceinline__ float pow2(int k) {
+  return (k >= -126 && k <= 127) ? __uint_as_float((uint32_t)(127 + k) << 23) : ldexpf(1.f, k);
+}
+
+// Barrier over the 8 query-prep / epilogue warps on an mbarrier (8 arrivals):
+// unlike bar.sync its wait has an iteration limit, so a stalled partner sets the
+// fault word instead of hanging the CTA.
+struct GroupSync {
+  uint64_t* bar;
+  uint32_t phase;
+  __device__ __forceinline__ void sync(int lane) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+    mbar_wait(bar, phase);
+    phase ^= 1u;
+  }
+};
+
+// B image of KV head `head` into `img`, by the 256 threads of warps 13-20
+// (et = 0..255).  Steps: q_rot = H D q / sqrt(128) (warp per query);
+// u = S q_rot (thread = row of S x half of the coordinates); per-query scales
+// 2^F, 2^G putting the largest weight just below 2^23; digits into the image.
+template <int KB, int SI>
+__device__ void make_image(const TArgs& a, int64_t head, uint8_t* img, float4* qT, float4* uT, float4* up,
+                           const float* alpha, float* red, int et, GroupSync& gs) {
+  using L = TL<KB, SI>;
+  const int ew = et >> 5, lane = et & 31;
+  float* qTf = reinterpret_cast<float*>(qT);
+  float* uTf = reinterpret_cast<float*>(uT);
+  if (ew < 4) {  // warp = query ew; lane holds coordinates lane + 32 i
+    const bool valid = ew < a.group;
+    const int64_t row = head * a.group + ew;
+    float y[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = 32 * i + lane;
+      y[i] = (valid && j < a.d) ? __ldg(a.q + row * a.d + j) * (float)__ldg(a.D + j) : 0.f;
+    }
+#pragma unroll
+    for (int h = 1; h < 4; h <<= 1)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if ((i & h) == 0) {
+          const float u = y[i], w = y[i + h];
+          y[i] = u + w;
+          y[i + h] = u - w;
+        }
+#pragma unroll
+    for (int sft = 1; sft < 32; sft <<= 1)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float o = __shfl_xor_sync(FULL, y[i], sft);
+        y[i] = (lane & sft) ? (o - y[i]) : (y[i] + o);
+      }
+    float sum = 0.f, mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float v = y[i] * 0.08838834764831845f;  // 1/sqrt(128)
+      qTf[4 * (32 * i + lane) + ew] = v;
+      sum += v;
+      mx = fmaxf(mx, fabsf(v));
+    }
+    sum = warp_sum(sum);
+    mx = warp_max(mx);
+    if (lane == 0) {
+      red[4 * ew] = sum;
+      red[4 * ew + 1] = mx;
+    }
+  }
+  gs.sync(lane);
+  if constexpr (SI) {  // u = S q_rot: row i = et % 128, coordinates 64h .. 64h + 63 (h = et / 128)
+    const int i = et & 127, h = et >> 7;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), acc2 = acc;
+    if (i < a.m) {
+      const uint4* srow = reinterpret_cast<const uint4*>(a.S + (size_t)i * DP) + 8 * h;
+      uint4 sv[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sv[k] = __ldg(srow + k);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t wv[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w};
+#pragma unroll
+        for (int h2 = 0; h2 < 4; ++h2) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[h2]));
+          const int j = 64 * h + 8 * k + 2 * h2;
+          const float4 q0 = qT[j], q1 = qT[j + 1];
+          acc.x = fmaf(f.x, q0.x, acc.x);
+          acc.y = fmaf(f.x, q0.y, acc.y);
+          acc.z = fmaf(f.x, q0.z, acc.z);
+          acc.w = fmaf(f.x, q0.w, acc.w);
+          acc2.x = fmaf(f.y, q1.x, acc2.x);
+          acc2.y = fmaf(f.y, q1.y, acc2.y);
+          acc2.z = fmaf(f.y, q1.z, acc2.z);
+          acc2.w = fmaf(f.y, q1.w, acc2.w);
+        }
+      }
+    }
+    up[128 * h + i] = make_float4(acc.x + acc2.x, acc.y + acc2.y, acc.z + acc2.z, acc.w + acc2.w);
+    gs.sync(lane);
+    if (et < 128) {
+      const float4 p0 = up[et], p1 = up[128 + et];
+      uT[et] = make_float4(p0.x + p1.x, p0.y + p1.y, p0.z + p1.z, p0.w + p1.w);
+    }
+    gs.sync(lane);
+  }
+  if (ew < 4) {  // scales and per-query scalars: warp = query ew
+    float su = 0.f, mu = 0.f;
+    if constexpr (SI) {
+      for (int i = lane; i < a.m; i += 32) {
+        const float v = uTf[4 * i + ew];
+        su += v;
+        mu = fmaxf(mu, fabsf(v));
+      }
+      su = warp_sum(su);
+      mu = warp_max(mu);
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int T = 0; T < L::NT; ++T) amax = fmaxf(amax, fabsf(alpha[T]));
+    const float mc = 2.f * amax * red[4 * ew + 1], ms = 2.f * mu;
+    const int F = mc > 0.f ? 23 - exponent_of(mc) : 0;
+    const int G = ms > 0.f ? 23 - exponent_of(ms) : 0;
+    if (lane == 0) {
+      red[4 * ew + 2] = pow2(F);
+      red[4 * ew + 3] = pow2(G);
+      // sum_T alpha_T = c[L-1] (all index bits set)
+      reinterpret_cast<float4*>(img)[ew] =
+          make_float4(pow2(-(F + 7)), alpha[4] * red[4 * ew], pow2(-(G + 7)), su);
+    }
+  }
+  gs.sync(lane);
+  // Digit words, one thread per (query q, plane P, bit class c, word w): the weights of
+  // coordinates 32w + 8b + c (b = 0..3) give word w of K chunk c of plane P in the 4
+  // digit rows 4q + d.  Scaling by 2^F (2^G) is exact.
+  for (int e = et; e < 4 * L::NP * 32; e += 256) {
+    const int w = e & 3, c = (e >> 2) & 7, pq = e >> 5;
+    const int q = pq / L::NP, P = pq - q * L::NP;
+    const bool cen = P < L::NT;
+    const float scale = cen ? 2.f * alpha[P] * red[4 * q + 2] : 2.f * red[4 * q + 3];
+    const float* src = cen ? qTf : uTf;
+    uint32_t W[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int j = 32 * w + 8 * b + c;
+      int X = (cen || j < a.m) ? __float2int_rn(src[4 * j + q] * scale) * (1 << (7 - c)) : 0;
+#pragma unroll
+      for (int dd = 0; dd < 3; ++dd) {
+        const int lowb = (int)(int8_t)(X & 0xFF);
+        W[dd] |= (uint32_t)(uint8_t)lowb << (8 * b);
+        X = (X - lowb) >> 8;
+      }
+      W[3] |= (uint32_t)(uint8_t)X << (8 * b);
+    }
+    const int kc = cen ? 8 * P + c : c;
+    uint8_t* base = img + (cen ? L::IMG_C : L::IMG_S) + kc * 256 + (q >> 1) * 128 + 4 * w;
+#pragma unroll
+    for (int dd = 0; dd < 4; ++dd) *reinterpret_cast<uint32_t*>(base + (4 * (q & 1) + dd) * 16) = W[dd];
+  }
+  fence_async_smem();  // the image is read by the tensor core (async proxy)
+  gs.sync(lane);
+}
 
 template <int KB, int SI>
 __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(const TArgs a) {
   using L = TL<KB, SI>;
   constexpr int W_EXP0 = L::W_EXP0, W_EPI0 = L::W_EPI0;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // [MAX_STAGES] stage loaded
-  uint64_t* empty = full + MAX_STAGES;                  // [MAX_STAGES] stage read by the expansion and epilogue warps
-  uint64_t* afull = empty + MAX_STAGES;                 // [3] A buffer written (8 arrivals)
-  uint64_t* mdone = afull + 3;                          // [3] MMAs of the item done: its A buffer is free
-  uint64_t* cfull = mdone + 3;                          // [4] MMAs done: accumulator set full
-  uint64_t* accfree = cfull + 4;                        // [4] accumulator set read (8 arrivals)
-  uint64_t* bfull = accfree + 4;                        // B image loaded
-  uint32_t* tbase = reinterpret_cast<uint32_t*>(bfull + 1);
-  uint8_t* Bsm = smem + HDR;
-  uint8_t* ring = Bsm + L::BBYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // [MAX_STAGES] stage loaded
+  uint64_t* empty = full + MAX_STAGES;                 // [MAX_STAGES] stage read by expansion and epilogue
+  uint64_t* afull = empty + MAX_STAGES;                // [3] A buffer written (8 arrivals)
+  uint64_t* mdone = afull + 3;                         // [3] MMAs of the item done: its A buffer is free (2)
+  uint64_t* cfull = mdone + 3;                         // [4] accumulator set full (2)
+  uint64_t* accfree = cfull + 4;                       // [4] accumulator set read (8)
+  uint64_t* imgfull = accfree + 4;                     // [2] B image ready (1)
+  uint64_t* imgfree = imgfull + 2;                     // [2] no MMA reads the B image any more (4)
+  uint64_t* gbar = imgfree + 2;                        // barrier of the 8 prep / epilogue warps (8)
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(gbar + 1);
+  float* alpha = reinterpret_cast<float*>(tbase + 4);  // [5] Walsh coefficients, then c[L-1]
+  float* red = alpha + 8;                              // [16] per query: sum, max, 2^F, 2^G
+  uint8_t* imgs = smem + L::OFF_IMG;
+  float4* qT = reinterpret_cast<float4*>(smem + L::OFF_PREP);
+  float4* uT = qT + 128;
+  float4* up = uT + 128;
+  uint8_t* ring = smem + L::OFF_RING;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.stages;
   const int64_t i0 = (int64_t)blockIdx.x * a.n_items / gridDim.x;
   const int64_t i1 = (int64_t)(blockIdx.x + 1) * a.n_items / gridDim.x;
   const int n = (int)(i1 - i0);
+  const int64_t h_first = i0 / a.tiles_per_head;
+  const int n_img = n > 0 ? (int)((i1 - 1) / a.tiles_per_head - h_first) + 1 : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < MAX_STAGES; ++s) {
@@ -122,29 +312,33 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
     }
     for (int b = 0; b < 3; ++b) {
       mbar_init(&afull[b], 8);
-      mbar_init(&mdone[b], L::NACC);
+      mbar_init(&mdone[b], 2);
     }
     for (int c = 0; c < 4; ++c) {
-      mbar_init(&cfull[c], L::NACC);
+      mbar_init(&cfull[c], 2);
       mbar_init(&accfree[c], 8);
     }
-    mbar_init(bfull, 1);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&imgfull[k], 1);
+      mbar_init(&imgfree[k], 4);
+    }
+    mbar_init(gbar, 8);
   }
-  if (warp == 0) tmem_alloc(tbase, L::COLS);
+  if (warp == 0) tmem_alloc(tbase, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tbase;
-  // tensor-memory columns: accumulator set c = NACC x 32 columns from c * NACC * 32,
-  // then the two A buffers
-  auto acc_col = [&](int c, int k) { return tmem + (uint32_t)(32 * (c * L::NACC + k)); };
-  auto a_col = [&](int b) { return tmem + (uint32_t)(32 * L::NACC * L::NB + b * L::ACOLS); };
+  // tensor-memory columns: accumulator sets (64 each), then the A buffers
+  auto acc_col = [&](int c) { return tmem + (uint32_t)(L::ACC * c); };
+  auto a_col = [&](int b) { return tmem + (uint32_t)(L::ACC * L::NB + b * L::ACOLS); };
 
   if (warp == 0) {
-    // ---------------- producer: code tiles into the ring ----------------
+    // ---------------- producer: code tiles and norms into the ring ----------------
+    grid_dependency_wait();  // codes may come from the preceding kernel in the stream
     if (lane == 0) {
       int issued = 0;
-      int64_t head = i0 / a.tiles_per_head;  // (head, t) advance by one item per iteration: no division in the loop
+      int64_t head = h_first;
       int t = (int)(i0 % a.tiles_per_head);
       for (int i = 0, s = 0, use = 0; i < n; ++i) {
         if (i >= S && !mbar_wait(&empty[s], (use - 1) & 1)) break;
@@ -165,57 +359,50 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       for (int i = (issued > S ? issued - S : 0); i < issued; ++i) mbar_wait(&full[i % S], (i / S) & 1);
     }
   } else if (warp < W_EXP0) {
-    // ---------------- B image + MMA issue ----------------
-    // Two pairs of issuing warps take alternate items (pair p: items i with i % 2 == p),
-    // each warp of a pair every other K step into its own partial accumulator.  A
-    // thread cannot go on to its next item until the tensor core has taken its MMAs,
-    // so the other pair keeps the tensor pipe busy meanwhile.
+    // ---------------- MMA issue (warp-uniform, elected lane) ----------------
     const int j = warp - 1, par = j >> 1, k = j & 1;
-    if (lane == 0) {
-      grid_dependency_wait();  // the B image comes from the query-prep kernel
-      constexpr uint32_t idesc = idesc_u8s8_s32(TK, 32);
-      const uint32_t sB = smem_u32(Bsm);
-      int64_t cur = -1, head = i0 / a.tiles_per_head;
-      int t = (int)(i0 % a.tiles_per_head);
-      uint32_t loads = 0, waited = 0;  // B images requested so far / waited for
-      int done = -1;
-      bool ok = true;
-      for (int i = 0, c = 0, cu = 0; i < n && ok; ++i, ++t, (++c == L::NB ? (c = 0, ++cu) : 0)) {
-        const int b = i % L::NA, ua = i / L::NA;  // A buffer and its use count
-        if (t == a.tiles_per_head) t = 0, ++head;
-        const bool mine = (i & 1) == par;
-        if (head != cur) {
-          if (mine && k == 0) {  // reload B once no MMA of either pair still reads the old one
-            if (i >= 1 && !mbar_wait(&mdone[(i - 1) % L::NA], ((i - 1) / L::NA) & 1)) break;
-            if (i >= 2 && !mbar_wait(&mdone[(i - 2) % L::NA], ((i - 2) / L::NA) & 1)) break;
-            mbar_expect_tx(bfull, L::BBYTES);
-            bulk_g2s(Bsm, a.prep + head * a.prep_bytes, L::BBYTES, bfull);
-          }
-          ++loads;
-          cur = head;
-        }
-        if (!mine) continue;
-        if (waited != loads) {  // the latest B image (load number loads - 1) has landed
-          if (!mbar_wait(bfull, (loads - 1) & 1)) break;
-          waited = loads;
-        }
-        if (!mbar_wait(&afull[b], ua & 1)) break;
-        if (cu >= 1 && !mbar_wait(&accfree[c], (cu - 1) & 1)) break;
-        tc_fence_after();
-        for (int ks = k; ks < L::KSTEPS; ks += 2)
-          umma_i8_ts(acc_col(c, k), a_col(b) + 8 * ks, smem_desc(sB + ks * 256, 128, L::KC * 128), idesc,
-                     ks >= 2 ? 1u : 0u);
-        umma_commit(&mdone[b]);
-        umma_commit(&cfull[c]);
-        done = i;
+    constexpr uint32_t idesc = idesc_u8s8_s32(TK, 16);
+    int t = (int)(i0 % a.tiles_per_head);
+    int kimg = 0;
+    bool ok = n > 0 && mbar_wait(&imgfull[0], 0);
+    uint32_t simg = smem_u32(imgs);
+    for (int i = 0; i < n && ok; ++i, ++t) {
+      if (t == a.tiles_per_head) {  // next KV head: release the old image, wait for the next one
+        t = 0;
+        __syncwarp();
+        umma_commit_elect(&imgfree[kimg & 1]);
+        ++kimg;
+        if (!mbar_wait(&imgfull[kimg & 1], (kimg >> 1) & 1)) break;
+        simg = smem_u32(imgs + (kimg & 1) * L::IMG);
       }
-      if (done >= 0) mbar_wait(&mdone[done % L::NA], (done / L::NA) & 1);  // no MMA left in flight
+      if ((i & 1) != par) continue;
+      const int b = i % L::NA, ua = i / L::NA, c = i % L::NB, cu = i / L::NB;
+      if (!mbar_wait(&afull[b], ua & 1)) break;
+      if (cu >= 1 && !mbar_wait(&accfree[c], (cu - 1) & 1)) break;
+      __syncwarp();  // elect.sync needs the whole warp converged
+      tc_fence_after();
+      const uint32_t dacc = acc_col(c) + 32u * (uint32_t)k;
+      const uint32_t abuf = a_col(b) + 8u * (uint32_t)k;
+      const uint64_t dc = smem_desc(simg + L::IMG_C + 512 * k, 256, 128);
+#pragma unroll
+      for (int u = 0; u < L::CSTEPS / 2; ++u)  // K steps k, k+2, ...: 1024 bytes of image apart
+        umma_i8_ts_elect(dacc, abuf + 16u * u, dc + (uint64_t)(64 * u), idesc, u > 0 ? 1u : 0u);
+      if constexpr (SI) {
+        const uint64_t ds = smem_desc(simg + L::IMG_S + 512 * k, 256, 128);
+#pragma unroll
+        for (int u = 0; u < L::SSTEPS / 2; ++u)
+          umma_i8_ts_elect(dacc + 16u, abuf + 32u * L::NT + 16u * u, ds + (uint64_t)(64 * u), idesc,
+                           u > 0 ? 1u : 0u);
+      }
+      umma_commit_elect(&mdone[b]);
+      umma_commit_elect(&cfull[c]);
     }
+    __syncwarp();
   } else if (warp < W_EPI0) {
     // ---------------- expansion: code bits -> A in tensor memory ----------------
     const int ew = warp - W_EXP0;
-    const int qd = warp & 3;   // tensor-memory lane quadrant = 32-key code tile within the item
-    const int cg = ew >> 2;    // bit classes 4cg .. 4cg+3
+    const int qd = warp & 3;  // tensor-memory lane quadrant = 32-key code tile within the item
+    const int cg = ew >> 2;   // bit classes 4cg .. 4cg+3
     for (int i = 0, s = 0, use = 0; i < n; ++i, (++s == S ? (s = 0, ++use) : 0)) {
       const int b = i % L::NA, ua = i / L::NA;
       if (!mbar_wait(&full[s], use & 1)) break;
@@ -228,7 +415,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       if (lane == 0) mbar_arrive(&empty[s]);
       uint4 it[L::NP];
 #pragma unroll
-      for (int T = 0; T < L::NT; ++T) it[T] = pw[T];
+      for (int T = 0; T < L::NT; ++T) it[T] = pw[T < KB ? T : 0];
       if constexpr (KB == 3)
         it[3] = make_uint4(pw[0].x ^ pw[1].x ^ pw[2].x, pw[0].y ^ pw[1].y ^ pw[2].y, pw[0].z ^ pw[1].z ^ pw[2].z,
                            pw[0].w ^ pw[1].w ^ pw[2].w);
@@ -253,21 +440,47 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       if (lane == 0) mbar_arrive(&afull[b]);
     }
   } else {
-    // ---------------- epilogue: accumulators -> logits ----------------
-    grid_dependency_wait();  // per-query scalars come from the query-prep kernel
+    // ---------------- query preparation, then the epilogue ----------------
+    const int et = threadIdx.x - 32 * W_EPI0;
     const int ew = warp - W_EPI0;
     const int qd = warp & 3, qp = ew >> 2;  // keys 32qd + lane; queries 2qp, 2qp+1
-    int64_t cur = -1, head = i0 / a.tiles_per_head;
+    grid_dependency_wait();                // queries may come from the preceding kernel in the stream
+    if (et < L::NT + 1) {                  // Walsh coefficients of the odd-symmetric codebook (fp64), c[L-1]
+      const int Lv = 1 << KB;
+      double s = 0.0;
+      if (et < L::NT) {
+        const int mask = walsh_mask(KB, et);
+        for (int l = 0; l < Lv; ++l) s += (double)__ldg(a.cent + l) * ((__popc(l & mask) & 1) ? 1.0 : -1.0);
+        alpha[et] = (float)(s / Lv);
+      } else {
+        alpha[4] = __ldg(a.cent + Lv - 1);
+      }
+    }
+    GroupSync gs{gbar, 0u};
+    gs.sync(lane);
+    for (int k = 0; k < n_img && k < 2; ++k) {
+      make_image<KB, SI>(a, h_first + k, imgs + k * L::IMG, qT, uT, up, alpha, red, et, gs);
+      if (et == 0) mbar_arrive(&imgfull[k]);
+    }
+    int64_t head = h_first;
     int t = (int)(i0 % a.tiles_per_head);
+    int kimg = 0;
     float4 sc[2] = {};
+    bool fresh = true;
     for (int i = 0, s = 0, use = 0, c = 0, cu = 0; i < n;
          ++i, ++t, (++s == S ? (s = 0, ++use) : 0), (++c == L::NB ? (c = 0, ++cu) : 0)) {
-      if (t == a.tiles_per_head) t = 0, ++head;
-      if (head != cur) {
-        const float4* qs = reinterpret_cast<const float4*>(a.prep + head * a.prep_bytes + L::BBYTES);
+      if (t == a.tiles_per_head) t = 0, ++head, ++kimg, fresh = true;
+      if (fresh) {
+        fresh = false;
+        const float4* qs = reinterpret_cast<const float4*>(imgs + (kimg & 1) * L::IMG);
         sc[0] = qs[2 * qp];
         sc[1] = qs[2 * qp + 1];
-        cur = head;
+        const int kn = kimg + 1;  // the next head's image, into the slot image kimg - 1 used
+        if (kn >= 2 && kn < n_img) {
+          mbar_wait(&imgfree[kn & 1], ((kn - 2) >> 1) & 1);  // on a time-out the fault word is set; go on
+          make_image<KB, SI>(a, head + 1, imgs + (kn & 1) * L::IMG, qT, uT, up, alpha, red, et, gs);
+          if (et == 0) mbar_arrive(&imgfull[kn & 1]);
+        }
       }
       const int64_t key = (int64_t)t * TK + 32 * qd + lane;
       const bool kvalid = key < a.n_keys;
@@ -279,33 +492,41 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       if (lane == 0) mbar_arrive(&empty[s]);
       if (!mbar_wait(&cfull[c], cu & 1)) break;
       tc_fence_after();
-      uint32_t r[16], rp[16];
-      const uint32_t lrow = ((uint32_t)(32 * qd) << 16) + 16 * qp;
-      tmem_ld16_issue(acc_col(c, 0) + lrow, r);
-      tmem_ld16_issue(acc_col(c, 1) + lrow, rp);
-      tmem_ld_wait16(r);
-      tmem_ld_wait16(rp);
+      uint32_t c0[8], c1[8], s0[8], s1[8];
+      const uint32_t lrow = acc_col(c) + ((uint32_t)(32 * qd) << 16) + 8 * qp;
+      tmem_ld8_issue(lrow, c0);
+      tmem_ld8_issue(lrow + 32, c1);
+      if constexpr (SI) {
+        tmem_ld8_issue(lrow + 16, s0);
+        tmem_ld8_issue(lrow + 48, s1);
+      } else {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) r[e] += rp[e];  // exact: the full sums stay below 2^24
+        for (int e = 0; e < 8; ++e) s0[e] = s1[e] = 0u;
+      }
+      tmem_ld_wait8x4(c0, c1, s0, s1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&accfree[c]);
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int q = 2 * qp + j;
-        if (q < a.group && kvalid) {
+      for (int jj = 0; jj < 2; ++jj) {
+        const int qi = 2 * qp + jj;
+        if (qi < a.group && kvalid) {
           // sum_d 256^d C[d]: each C[d] an exact int32 below 2^24; one fp32 rounding per step
-          const float cen = fmaf((float)(int)r[8 * j + 3], 16777216.f,
-                                 fmaf((float)(int)r[8 * j + 2], 65536.f,
-                                      fmaf((float)(int)r[8 * j + 1], 256.f, (float)(int)r[8 * j])));
-          float l = fmaf(cen, sc[j].x, -sc[j].y);
-          if constexpr (SI) {
-            const float sg = fmaf((float)(int)r[8 * j + 7], 16777216.f,
-                                  fmaf((float)(int)r[8 * j + 6], 65536.f,
-                                       fmaf((float)(int)r[8 * j + 5], 256.f, (float)(int)r[8 * j + 4])));
-            l = fmaf(gam * a.kappa, fmaf(sg, sc[j].z, -sc[j].w), l);
+          int C[4], Z[4];
+#pragma unroll
+          for (int dd = 0; dd < 4; ++dd) {
+            C[dd] = (int)(c0[4 * jj + dd] + c1[4 * jj + dd]);
+            Z[dd] = (int)(s0[4 * jj + dd] + s1[4 * jj + dd]);
           }
-          a.logits[(head * a.group + q) * a.ld + key] = nrm * l;
+          const float cen =
+              fmaf((float)C[3], 16777216.f, fmaf((float)C[2], 65536.f, fmaf((float)C[1], 256.f, (float)C[0])));
+          float l = fmaf(cen, sc[jj].x, -sc[jj].y);
+          if constexpr (SI) {
+            const float sg =
+                fmaf((float)Z[3], 16777216.f, fmaf((float)Z[2], 65536.f, fmaf((float)Z[1], 256.f, (float)Z[0])));
+            l = fmaf(gam * a.kappa, fmaf(sg, sc[jj].z, -sc[jj].w), l);
+          }
+          a.logits[(head * a.group + qi) * a.ld + key] = nrm * l;
         }
       }
     }
@@ -313,7 +534,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, L::COLS);
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 template <int KB, int SI>
@@ -321,7 +542,7 @@ int launch_tc(const TArgs& a0, int sm, cudaStream_t st) {
   using L = TL<KB, SI>;
   TArgs a = a0;
   a.stages = MAX_STAGES;
-  while (a.stages > 4 && L::smem(a.stages) > 227 * 1024) --a.stages;
+  while (a.stages > 4 && L::smem(a.stages) > 200 * 1024) --a.stages;
   // at least 120 KB: one CTA per SM, so no second CTA waits for the SM's tensor memory
   const int bytes = std::max(L::smem(a.stages), 120 * 1024);
   auto kern = logits_tc_kernel<KB, SI>;
@@ -351,10 +572,10 @@ bool logits_tc_supported(int dp, int kb, int m, int group, int64_t n_keys, const
          aligned(norms, 16) && (m == 0 || aligned(rnorms, 16));
 }
 
-// Scan with the query-prep output `prep` (layout 1, one chunk per KV head).
-int launch_logits_tc(int kb, int m, const void* codes, const uint16_t* norms, const uint16_t* rnorms,
-                     int64_t n_keys, int n_kv_heads, int group, const uint8_t* prep, int64_t prep_bytes,
-                     float* logits, int64_t ld, cudaStream_t st) {
+// The fused scan: query preparation inside the kernel, no workspace.
+int launch_logits_tc(int kb, int m, const float* q, int d, const float* cent, const int8_t* D, const uint16_t* S,
+                     const void* codes, const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys,
+                     int n_kv_heads, int group, float* logits, int64_t ld, cudaStream_t st) {
   TArgs a;
   a.codes = static_cast<const uint8_t*>(codes);
   a.norms = norms;
@@ -364,8 +585,13 @@ int launch_logits_tc(int kb, int m, const void* codes, const uint16_t* norms, co
   a.tb = tqd::tile_bytes(128, kb, m);
   a.tiles_per_head = (int)((n_keys + TK - 1) / TK);
   a.n_items = (int64_t)n_kv_heads * a.tiles_per_head;
-  a.prep = prep;
-  a.prep_bytes = prep_bytes;
+  a.q = q;
+  a.d = d;
+  a.kb = kb;
+  a.m = m;
+  a.cent = cent;
+  a.D = D;
+  a.S = S;
   a.logits = logits;
   a.ld = ld;
   a.kappa = (float)(std::sqrt(M_PI / 2.0) / (m > 0 ? m : 1));

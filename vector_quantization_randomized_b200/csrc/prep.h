@@ -12,11 +12,11 @@ int launch_prep(const tqd::PrepArgs& a, cudaStream_t st);
 // Number of SMs of the current device.
 int sm_count();
 // The tensor-memory logits scan (logits_tc.cu): supported shapes, and the launch
-// over query-prep output of layout 1 (one chunk per KV head).
+// (query preparation inside the kernel, no workspace).
 bool logits_tc_supported(int dp, int kb, int m, int group, int64_t n_keys, const void* norms, const void* rnorms);
-int launch_logits_tc(int kb, int m, const void* codes, const uint16_t* norms, const uint16_t* rnorms,
-                     int64_t n_keys, int n_kv_heads, int group, const uint8_t* prep, int64_t prep_bytes,
-                     float* logits, int64_t ld, cudaStream_t st);
+int launch_logits_tc(int kb, int m, const float* q, int d, const float* cent, const int8_t* D, const uint16_t* S,
+                     const void* codes, const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys,
+                     int n_kv_heads, int group, float* logits, int64_t ld, cudaStream_t st);
 // Bytes of query-prep scratch per chunk of 4 queries, the larger of both layouts.
 int64_t prep_chunk_bytes_max(int dp, int kb, int m);
 }  // namespace tq

@@ -64,17 +64,6 @@ struct ScanShape {
 // 2^-(G+7), sum u).
 __host__ __device__ __forceinline__ int64_t prep_chunk_bytes(int fr) { return (int64_t)fr * 32 * 4 + 4 * 16; }
 
-// Query-prep output for the tensor-memory scan (d_pad 128): the B operand
-// image of one chunk, 32 rows x kc 16-byte K chunks in the canonical K-major
-// no-swizzle layout (8-row groups kc*128 bytes apart, K chunks 128 bytes
-// apart, 16 bytes per row), then the same per-query scalars.  Row 8j + r holds,
-// for query j, digit r of the centroid weights (r < 4) or digit r-4 of the
-// sign weights (r >= 4); K chunk 8P + c holds bit class c of plane P (Walsh
-// planes, then the sign plane), byte 4w + b of a chunk is coordinate
-// 32w + 8b + c.
-__host__ __device__ __forceinline__ int64_t prep_chunk_bytes_tc(int kc) { return (int64_t)kc * 512 + 4 * 16; }
-__host__ __device__ __forceinline__ int tc_kchunks(int kb, int m) { return 8 * (walsh_planes(kb) + (m > 0 ? 1 : 0)); }
-
 struct PrepArgs {
   const float* q;       // query rows, stride d
   int d, dp, kb, m;
@@ -82,10 +71,8 @@ struct PrepArgs {
   const float* cent;
   const int8_t* D;
   const uint16_t* S;
-  uint8_t* out;         // n_outer*nqc chunks of prep_chunk_bytes(fr) (layout 0) or prep_chunk_bytes_tc(kc) (layout 1)
+  uint8_t* out;         // n_outer*nqc chunks of prep_chunk_bytes(fr)
   int fr;
-  int layout = 0;       // 0: mma.sync A fragments; 1: tcgen05 B image (d_pad 128)
-  int kc = 0;           // K chunks of the B image (layout 1)
 };
 
 // Compile-time scan over one 8-key subtile.
