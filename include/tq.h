@@ -163,6 +163,10 @@ int tq_dequantize(const tq_params* p, const void* codes, const uint16_t* norms,
  *      l = n*( <q_rot, c[idx]> + gamma*sqrt(pi/2)/m*<S q_rot, 2s-1> ),
  *      q_rot = H D q / sqrt(d_pad).  MSE-mode codes give n*<q_rot, c[idx]>.
  *   workspace: device, >= tq_logits_workspace(p, n_q) bytes, 16-byte aligned.
+ *      The tensor-core path (d_pad 128, group <= 4, n_keys a multiple of 32,
+ *      16-byte aligned norms) prepares the queries inside its kernel and does
+ *      not touch the workspace; the other shapes keep their query
+ *      preparation there.
  * Supported: d_pad 128 with kb <= 3, d_pad 256 with kb <= 2.
  */
 int64_t tq_logits_workspace(const tq_params* p, int n_q);
@@ -231,7 +235,7 @@ int tq_decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int
 /*
  * tq_decode_attn_sparse - tq_decode_attn with Sparse V [Z1 "Sparse V": skip
  *   the value work of tokens whose attention weight is negligible].  Same
- *   arguments plus v_eps >= 0.  Inside each 512-token split of a sequence, a
+ *   arguments plus v_eps >= 0.  Inside each 256-token split of a sequence, a
  *   token is dropped when its weight within the split, p_t / (split sum), is
  *   below v_eps for every query head sharing the KV head; since that bounds its
  *   final softmax weight from above, only tokens with final weight < v_eps are
@@ -251,7 +255,8 @@ int tq_decode_attn_sparse(const tq_params* kp, const tq_params* vp, const float*
  *   q: device fp32 [n_q][d]; codes/norms/rnorms: n_db vectors.
  *   ids: device int32 [n_q][k], scores: device fp32 [n_q][k]: the k largest
  *   logit estimates (as tq_logits with group 1) per query, in descending
- *   order, ties to the lower id.  1 <= k <= 32.
+ *   order, ties to the lower id.  1 <= k <= 16.  When n_db < k the trailing
+ *   slots hold id INT32_MAX and score -inf.
  *   workspace: device, >= tq_search_workspace(...) bytes, 16-byte aligned.
  */
 int64_t tq_search_workspace(const tq_params* p, int n_q, int64_t n_db, int k);
@@ -259,6 +264,57 @@ int tq_search_topk(const tq_params* p, const float* q, int n_q, const void* code
                    const uint16_t* norms, const uint16_t* rnorms, int64_t n_db, int k,
                    int32_t* ids, float* scores, void* workspace, int64_t workspace_bytes,
                    tq_stream_t stream);
+
+/*
+ * Sharded forms: one process per GPU, each holding one shard; the only
+ * exchange is one all-gather of the small per-shard results (the caller's,
+ * e.g. torch.distributed over NCCL; see parallel.py of the Python package).
+ *
+ * tq_search_merge - global top-k of a database split across devices [E5:
+ *   inner-product search over very large sets].  Each device runs
+ *   tq_search_topk on its shard; the lists are gathered and merged here.
+ *   ids, scores: device [n_parts][n_q][k], int32 shard-local ids and fp32
+ *     estimates as tq_search_topk returns them (id < 0 or INT32_MAX, or
+ *     score -inf: empty slot).
+ *   id_offsets: HOST int64 [n_parts], the global id of each shard's first
+ *     vector (0 <= offset < INT32_MAX); added to that shard's ids.
+ *   out_ids / out_scores: device [n_q][k]: the k best by estimate, ties to the
+ *     lower global id.  This equals tq_search_topk over the whole database
+ *     when every shard returned its exact top-k.
+ *   1 <= n_parts <= 64, 1 <= k <= 16, n_parts * k <= 1024.
+ */
+int tq_search_merge(const int32_t* ids, const float* scores, int n_parts, const int64_t* id_offsets, int n_q,
+                    int k, int32_t* out_ids, float* out_scores, tq_stream_t stream);
+
+/*
+ * tq_decode_attn_partial - tq_decode_attn over the tokens this caller holds
+ *   (a token range of every sequence, laid out as a KV cache of its own with
+ *   max_tokens and per-sequence counts seq_lens of that range), returning the
+ *   unnormalised partial instead of the output [E4, split over devices].
+ *   partial: device fp32 [batch][n_q_heads][d_pad + 2], per row
+ *     o_rot[0..d_pad) = sum_t 2^(s_t - m) n_v,t c_v[idx_t]  (rotated domain),
+ *     then m = max_t s_t with s_t = scale * l_t * log2(e) (-inf: no token),
+ *     then l = sum_t 2^(s_t - m) (0: no token).
+ *   Other arguments and the workspace as tq_decode_attn;
+ *   tq_decode_attn_partial_bytes gives the size of `partial`.
+ */
+int64_t tq_decode_attn_partial_bytes(const tq_params* vp, int batch, int n_q_heads);
+int tq_decode_attn_partial(const tq_params* kp, const tq_params* vp, const float* q, int batch,
+                           int n_q_heads, int n_kv_heads, const void* kcodes, const uint16_t* knorms,
+                           const uint16_t* krnorms, const void* vcodes, const uint16_t* vnorms,
+                           const int32_t* seq_lens, int64_t max_tokens, float scale, float* partial,
+                           void* workspace, int64_t workspace_bytes, tq_stream_t stream);
+
+/*
+ * tq_decode_attn_merge - log-sum-exp merge of n_parts partials (device fp32
+ *   [n_parts][batch][n_q_heads][d_pad + 2], e.g. all-gathered from the
+ *   devices) and the inverse rotation: with M = max_k m_k and w_k = 2^(m_k - M),
+ *   out[b][h] = D H (sum_k w_k o_k) / (sum_k w_k l_k) / sqrt(d_pad), first d
+ *   coordinates; rows empty in every part are zero.  vp: the value
+ *   parameters (MSE code, d_pad 128).  1 <= n_parts <= 2048.
+ */
+int tq_decode_attn_merge(const tq_params* vp, const float* partials, int n_parts, int batch, int n_q_heads,
+                         float* out, tq_stream_t stream);
 
 /*
  * tq_device_status - report (and optionally clear) device-side wait timeouts.

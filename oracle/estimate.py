@@ -27,6 +27,11 @@ attention and top-k search (TEST INFRASTRUCTURE).
   |o - o_full| <= v_eps * sum over skipped tokens of |v_hat_j|.
 * Search ("TurboQuant explainer", "向量搜索"): the k database ids with the
   largest estimate, ties to the lower id.
+* Sharded forms (a database or a sequence split across devices): the global
+  top-k is the top-k of the union of per-shard top-k lists (ids offset to
+  global), and decode attention over a token split is the log-sum-exp merge
+  of per-shard partials (m = max score, l = sum exp(score - m),
+  o = sum exp(score - m) v_hat).
 
 All arithmetic in fp64; the stored fp16 norms are used as stored.
 """
@@ -163,3 +168,64 @@ def recall_at_k(found, truth):
     """Mean over rows of |found_row ∩ truth_row| / k."""
     k = truth.shape[1]
     return float(np.mean([len(set(f) & set(t)) / k for f, t in zip(found, truth)]))
+
+
+def decode_partial(q, kD, kS, k_idx, k_signs, k_norm, k_rnorm, k_cent, km,
+                   vD, v_idx, v_norm, v_cent, d, seq_lens, Hq, Hkv, max_tokens, scale=0.0):
+    """Unnormalised decode attention over the tokens given (one shard of every sequence),
+    same arguments and indexing as decode_attention.  Per (b, h): m = max_t scale*l_t,
+    l = sum_t exp(scale*l_t - m), o = sum_t exp(scale*l_t - m) v_hat_t.  A row without
+    tokens has m = -inf, l = 0, o = 0.  Returns (m [B, Hq], l [B, Hq], o [B, Hq, d])."""
+    B = q.shape[0]
+    group = Hq // Hkv
+    if scale == 0.0:
+        scale = 1.0 / np.sqrt(d)
+    m = np.full((B, Hq), -np.inf)
+    lsum = np.zeros((B, Hq))
+    o = np.zeros((B, Hq, d))
+    for b in range(B):
+        L = int(seq_lens[b])
+        if L == 0:
+            continue
+        for h in range(Hq):
+            g = h // group
+            base = (b * Hkv + g) * max_tokens
+            sl = slice(base, base + L)
+            q_rot, u = prep_queries(q[b, h][None, :], kD, kS)
+            s = scale * logits_from_codes(q_rot, u, k_idx[sl], k_signs[sl], k_norm[sl], k_rnorm[sl], k_cent, km)[0]
+            m[b, h] = np.max(s)
+            w = np.exp(s - m[b, h])
+            lsum[b, h] = np.sum(w)
+            o[b, h] = w @ dequant_mse(v_idx[sl], v_norm[sl], v_cent, vD, d)
+    return m, lsum, o
+
+
+def merge_partials(parts):
+    """Log-sum-exp merge of decode partials [(m, l, o), ...]: with M = max_k m_k and
+    w_k = exp(m_k - M) (0 for an empty part), out = sum_k w_k o_k / sum_k w_k l_k;
+    rows that are empty in every part are 0."""
+    M = np.max(np.stack([p[0] for p in parts]), axis=0)
+    num = np.zeros_like(parts[0][2])
+    den = np.zeros_like(parts[0][1])
+    for m, lsum, o in parts:
+        w = np.where(np.isfinite(m), np.exp(np.where(np.isfinite(m), m - np.where(np.isfinite(M), M, 0.0), 0.0)),
+                     0.0)
+        num += w[..., None] * o
+        den += w * lsum
+    safe = np.where(den > 0, den, 1.0)
+    return np.where(den[..., None] > 0, num / safe[..., None], 0.0)
+
+
+def merge_topk(ids_parts, score_parts, offsets, k):
+    """Global top-k from per-shard top-k lists: ids_parts[p] [n_q, k_p] shard-local ids
+    (an id < 0 marks an empty slot), score_parts[p] their estimates, offsets[p] the first
+    global id of shard p.  Ties go to the lower global id.  Returns (ids, scores) [n_q, k]."""
+    ids = np.concatenate([np.where(np.asarray(i) >= 0, np.asarray(i, dtype=np.int64) + int(o), -1)
+                          for i, o in zip(ids_parts, offsets)], axis=1)
+    sc = np.concatenate([np.asarray(s, dtype=np.float64) for s in score_parts], axis=1)
+    sc = np.where(ids >= 0, sc, -np.inf)
+    big = np.where(ids >= 0, ids, np.iinfo(np.int64).max)
+    order = np.lexsort((big, -sc), axis=1)[:, :k]
+    out_i = np.take_along_axis(ids, order, axis=1)
+    out_s = np.take_along_axis(sc, order, axis=1)
+    return out_i, out_s

@@ -57,6 +57,11 @@ _SIGS = {
                                      _f32, _vp, _vp, _i64, _vp]),
     "tq_search_workspace": (_i64, [_P, _i32, _i64, _i32]),
     "tq_search_topk": (_i32, [_P, _vp, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _vp, _i64, _vp]),
+    "tq_decode_attn_partial_bytes": (_i64, [_P, _i32, _i32]),
+    "tq_decode_attn_partial": (_i32, [_P, _P, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _f32, _vp,
+                                      _vp, _i64, _vp]),
+    "tq_decode_attn_merge": (_i32, [_P, _vp, _i32, _i32, _i32, _vp, _vp]),
+    "tq_search_merge": (_i32, [_vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _vp]),
     "tq_device_status": (_i32, [_i32]),
     "tq_diag_bounded_wait": (_i32, [_i64, _vp]),
     "tq_polar_table_floats": (_i64, [_i32, _i32]),
@@ -246,6 +251,38 @@ def tq_search_topk(p, q, codes, norms, rnorms, n_db, k, ids, scores, workspace, 
     return _check(_lib.tq_search_topk(p.ref, _ptr(q), q.shape[0], _ptr(codes), _ptr(norms), _ptr(rnorms), n_db,
                                       k, _ptr(ids), _ptr(scores), _ptr(workspace), workspace.numel(),
                                       _stream(stream)))
+
+
+# ---- sharded forms (one device per shard, see parallel.py) ---------------------
+def tq_decode_attn_partial_bytes(vp, batch, n_q_heads):
+    return _lib.tq_decode_attn_partial_bytes(vp.ref, batch, n_q_heads)
+
+
+def tq_decode_attn_partial(kp, vp, q, n_kv_heads, kcodes, knorms, krnorms, vcodes, vnorms, seq_lens, max_tokens,
+                           partial, workspace, scale=0.0, stream=None):
+    """Decode attention over the tokens this caller holds, as an unnormalised partial
+    (device fp32 [batch, n_q_heads, d_pad + 2]: o_rot, m, l) for tq_decode_attn_merge."""
+    batch, n_q_heads = q.shape[0], q.shape[1]
+    return _check(_lib.tq_decode_attn_partial(kp.ref, vp.ref, _ptr(q), batch, n_q_heads, n_kv_heads, _ptr(kcodes),
+                                              _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms),
+                                              _ptr(seq_lens), max_tokens, scale, _ptr(partial), _ptr(workspace),
+                                              workspace.numel(), _stream(stream)))
+
+
+def tq_decode_attn_merge(vp, partials, out, stream=None):
+    """Log-sum-exp merge of partials (device fp32 [n_parts, batch, n_q_heads, d_pad + 2]) into out [batch, n_q_heads, d]."""
+    n_parts, batch, n_q_heads = partials.shape[0], partials.shape[1], partials.shape[2]
+    return _check(_lib.tq_decode_attn_merge(vp.ref, _ptr(partials), n_parts, batch, n_q_heads, _ptr(out),
+                                            _stream(stream)))
+
+
+def tq_search_merge(ids, scores, id_offsets, k, out_ids, out_scores, stream=None):
+    """Global top-k from per-shard lists ids/scores (device [n_parts, n_q, k]); id_offsets: the
+    first global id of each shard (host sequence of n_parts ints)."""
+    n_parts, n_q = ids.shape[0], ids.shape[1]
+    offs = np.ascontiguousarray(np.asarray(id_offsets, dtype=np.int64))
+    return _check(_lib.tq_search_merge(_ptr(ids), _ptr(scores), n_parts, offs.ctypes.data, n_q, k, _ptr(out_ids),
+                                       _ptr(out_scores), _stream(stream)))
 
 
 # ---- polar-coordinate stage 1 -------------------------------------------------

@@ -415,45 +415,64 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const DArgs a) {
 }
 
 struct CArgs {
-  const float* part;
+  const float* part;       // partial rows: o_rot[dp], m, l
+  int64_t row_stride;      // floats between consecutive output rows' first partial
+  int64_t chunk_stride;    // floats between the partials of one row
   const int8_t* vD;
-  const int32_t* seq_lens;
-  float* out;
+  const int32_t* seq_lens;  // NULL: a row is empty when no partial has weight
+  float* out;              // final mode: [rows][d]
+  float* part_out;         // partial mode (non-NULL): [rows][dp + 2], unnormalised, no rotation
   int nch, d, dp, hq;
 };
 
+// Log-sum-exp merge of the partials of one output row (b, h): weights
+// 2^(m_k - M) over the partials k, then either the normalised output with the
+// inverse rotation D H / sqrt(dp) (final mode), or the merged partial itself.
 __global__ void __launch_bounds__(128) combine_kernel(const CArgs a) {
   __shared__ float o[256];
   __shared__ float wts[2048];
   __shared__ float tot;
+  __shared__ float red[4];
   const int64_t h = blockIdx.x;  // b * hq + head
   const int b = (int)(h / a.hq);
-  const float* src = a.part + h * a.nch * (a.dp + 2);
+  const float* src = a.part + h * a.row_stride;
   // chunk weights 2^(m_k - M)
   float mx = -INFINITY;
-  for (int k = threadIdx.x; k < a.nch; k += blockDim.x) mx = fmaxf(mx, src[(int64_t)k * (a.dp + 2) + a.dp]);
+  for (int k = threadIdx.x; k < a.nch; k += blockDim.x) mx = fmaxf(mx, src[(int64_t)k * a.chunk_stride + a.dp]);
   mx = warp_max(mx);
-  __shared__ float red[4];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
   __syncthreads();
   mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
   __syncthreads();
   float lsum = 0.f;
   for (int k = threadIdx.x; k < a.nch; k += blockDim.x) {
-    const float mk = src[(int64_t)k * (a.dp + 2) + a.dp];
+    const float mk = src[(int64_t)k * a.chunk_stride + a.dp];
     const float wk = (mk == -INFINITY) ? 0.f : exp2f(mk - mx);
     wts[k] = wk;
-    lsum += wk * src[(int64_t)k * (a.dp + 2) + a.dp + 1];
+    lsum += wk * src[(int64_t)k * a.chunk_stride + a.dp + 1];
   }
   lsum = warp_sum(lsum);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = lsum;
   __syncthreads();
   if (threadIdx.x == 0) tot = red[0] + red[1] + red[2] + red[3];
   __syncthreads();
-  const bool empty = (a.seq_lens[b] <= 0) || !(tot > 0.f);
+  const bool empty = (a.seq_lens != nullptr && a.seq_lens[b] <= 0) || !(tot > 0.f);
+  if (a.part_out) {
+    float* dst = a.part_out + h * (a.dp + 2);
+    for (int c = threadIdx.x; c < a.dp; c += blockDim.x) {
+      float s = 0.f;
+      for (int k = 0; k < a.nch; ++k) s = fmaf(wts[k], src[(int64_t)k * a.chunk_stride + c], s);
+      dst[c] = empty ? 0.f : s;
+    }
+    if (threadIdx.x == 0) {
+      dst[a.dp] = empty ? -INFINITY : mx;
+      dst[a.dp + 1] = empty ? 0.f : tot;
+    }
+    return;
+  }
   for (int c = threadIdx.x; c < a.dp; c += blockDim.x) {
     float s = 0.f;
-    for (int k = 0; k < a.nch; ++k) s = fmaf(wts[k], src[(int64_t)k * (a.dp + 2) + c], s);
+    for (int k = 0; k < a.nch; ++k) s = fmaf(wts[k], src[(int64_t)k * a.chunk_stride + c], s);
     o[c] = empty ? 0.f : s / tot;
   }
   __syncthreads();
@@ -530,7 +549,7 @@ namespace {
 int decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int batch, int n_q_heads, int n_kv_heads,
                 const void* kcodes, const uint16_t* knorms, const uint16_t* krnorms, const void* vcodes,
                 const uint16_t* vnorms, const int32_t* seq_lens, int64_t max_tokens, float scale, float v_eps,
-                float* out, void* workspace, int64_t workspace_bytes, tq_stream_t stream) {
+                float* out, float* partial_out, void* workspace, int64_t workspace_bytes, tq_stream_t stream) {
   using namespace tq;
   int rc = check_params(kp, "tq_decode_attn(kp)");
   if (rc) return rc;
@@ -549,7 +568,7 @@ int decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int ba
     clear_error();
     return TQ_OK;
   }
-  if (!q || !kcodes || !knorms || !krnorms || !vcodes || !vnorms || !seq_lens || !out || !workspace)
+  if (!q || !kcodes || !knorms || !krnorms || !vcodes || !vnorms || !seq_lens || (!out && !partial_out) || !workspace)
     return set_error(TQ_EINVAL, "tq_decode_attn: NULL pointer argument");
   if (!aligned(kcodes, 16) || !aligned(vcodes, 16) || !aligned(workspace, 16))
     return set_error(TQ_EINVAL, "tq_decode_attn: codes and workspace must be 16-byte aligned");
@@ -618,9 +637,12 @@ int decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int ba
   if (rc) return rc;
   CArgs ca;
   ca.part = a.part;
+  ca.row_stride = (int64_t)nch * (128 + 2);
+  ca.chunk_stride = 128 + 2;
   ca.vD = vp->signs_D;
   ca.seq_lens = seq_lens;
   ca.out = out;
+  ca.part_out = partial_out;
   ca.nch = nch;
   ca.d = kp->d;
   ca.dp = 128;
@@ -639,7 +661,7 @@ extern "C" int tq_decode_attn(const tq_params* kp, const tq_params* vp, const fl
                               int64_t max_tokens, float scale, float* out, void* workspace,
                               int64_t workspace_bytes, tq_stream_t stream) {
   return decode_attn(kp, vp, q, batch, n_q_heads, n_kv_heads, kcodes, knorms, krnorms, vcodes, vnorms, seq_lens,
-                     max_tokens, scale, 0.f, out, workspace, workspace_bytes, stream);
+                     max_tokens, scale, 0.f, out, nullptr, workspace, workspace_bytes, stream);
 }
 
 extern "C" int tq_decode_attn_sparse(const tq_params* kp, const tq_params* vp, const float* q, int batch,
@@ -650,5 +672,58 @@ extern "C" int tq_decode_attn_sparse(const tq_params* kp, const tq_params* vp, c
   if (!(v_eps >= 0.f) || !std::isfinite(v_eps))
     return tq::set_error(TQ_EINVAL, "tq_decode_attn_sparse: v_eps must be finite and >= 0");
   return decode_attn(kp, vp, q, batch, n_q_heads, n_kv_heads, kcodes, knorms, krnorms, vcodes, vnorms, seq_lens,
-                     max_tokens, scale, v_eps, out, workspace, workspace_bytes, stream);
+                     max_tokens, scale, v_eps, out, nullptr, workspace, workspace_bytes, stream);
+}
+
+extern "C" int64_t tq_decode_attn_partial_bytes(const tq_params* vp, int batch, int n_q_heads) {
+  if (!vp || batch < 0 || n_q_heads < 1) return -1;
+  return (int64_t)batch * n_q_heads * (vp->d_pad + 2) * 4;
+}
+
+extern "C" int tq_decode_attn_partial(const tq_params* kp, const tq_params* vp, const float* q, int batch,
+                                      int n_q_heads, int n_kv_heads, const void* kcodes, const uint16_t* knorms,
+                                      const uint16_t* krnorms, const void* vcodes, const uint16_t* vnorms,
+                                      const int32_t* seq_lens, int64_t max_tokens, float scale, float* partial,
+                                      void* workspace, int64_t workspace_bytes, tq_stream_t stream) {
+  if (!partial) return tq::set_error(TQ_EINVAL, "tq_decode_attn_partial: NULL partial");
+  if (!tq::aligned(partial, 4)) return tq::set_error(TQ_EINVAL, "tq_decode_attn_partial: misaligned partial");
+  return decode_attn(kp, vp, q, batch, n_q_heads, n_kv_heads, kcodes, knorms, krnorms, vcodes, vnorms, seq_lens,
+                     max_tokens, scale, 0.f, nullptr, partial, workspace, workspace_bytes, stream);
+}
+
+extern "C" int tq_decode_attn_merge(const tq_params* vp, const float* partials, int n_parts, int batch,
+                                    int n_q_heads, float* out, tq_stream_t stream) {
+  using namespace tq;
+  int rc = check_params(vp, "tq_decode_attn_merge");
+  if (rc) return rc;
+  if (vp->mode != TQ_MODE_MSE || vp->d_pad != 128)
+    return set_error(TQ_EUNSUPPORTED, "tq_decode_attn_merge: needs the MSE-code value parameters with d_pad 128");
+  if (n_parts < 1 || n_parts > 2048 || batch < 0 || n_q_heads < 1)
+    return set_error(TQ_EINVAL, "tq_decode_attn_merge: need 1 <= n_parts <= 2048, batch >= 0, n_q_heads >= 1");
+  if (batch == 0) {
+    clear_error();
+    return TQ_OK;
+  }
+  if (!partials || !out) return set_error(TQ_EINVAL, "tq_decode_attn_merge: NULL pointer argument");
+  if (!aligned(partials, 4) || !aligned(out, 4)) return set_error(TQ_EINVAL, "tq_decode_attn_merge: misaligned pointer");
+  const int64_t rows = (int64_t)batch * n_q_heads;
+  if (rows > 0x7fffffff) return set_error(TQ_EUNSUPPORTED, "tq_decode_attn_merge: too many rows");
+  CArgs ca;
+  ca.part = partials;
+  ca.row_stride = 128 + 2;
+  ca.chunk_stride = rows * (128 + 2);
+  ca.vD = vp->signs_D;
+  ca.seq_lens = nullptr;
+  ca.out = out;
+  ca.part_out = nullptr;
+  ca.nch = n_parts;
+  ca.d = vp->d;
+  ca.dp = 128;
+  ca.hq = n_q_heads;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  combine_kernel<<<(unsigned)rows, 128, 0, st>>>(ca);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(TQ_ECUDA, "tq_decode_attn_merge: launch failed: %s", cudaGetErrorString(e));
+  clear_error();
+  return TQ_OK;
 }

@@ -249,6 +249,45 @@ __global__ void __launch_bounds__(32) merge_kernel(const MArgs a) {
   }
 }
 
+// Merge of per-shard top-k lists (a database split across devices, "TurboQuant
+// explainer" (m.163.com), "向量搜索"): one warp per query gathers the n_parts x k
+// candidates with their shard offsets and selects the k best, ties to the lower id.
+constexpr int MAX_SHARDS = 64;
+struct ShardMergeArgs {
+  const int32_t* ids;    // [n_parts][n_q][k] shard-local
+  const float* scores;   // [n_parts][n_q][k]
+  int n_parts, n_q, k;
+  int64_t offs[MAX_SHARDS];
+  int32_t* out_ids;
+  float* out_scores;
+};
+
+__global__ void __launch_bounds__(32) shard_merge_kernel(const ShardMergeArgs a) {
+  extern __shared__ float sbuf[];
+  const int q = blockIdx.x, lane = threadIdx.x;
+  const int n = a.n_parts * a.k;
+  float* cs = sbuf;
+  int* ci = reinterpret_cast<int*>(sbuf + n);
+  float* os = reinterpret_cast<float*>(ci + n);
+  int* oi = reinterpret_cast<int*>(os + KM);
+  for (int j = lane; j < n; j += 32) {
+    const int part = j / a.k, r = j - part * a.k;
+    const int64_t src = ((int64_t)part * a.n_q + q) * a.k + r;
+    const int id = a.ids[src];
+    const float sc = a.scores[src];
+    const bool empty = id < 0 || id == INT_MAX || !(sc > -INFINITY);
+    cs[j] = empty ? -INFINITY : sc;
+    ci[j] = empty ? INT_MAX : (int)(id + a.offs[part]);
+  }
+  __syncwarp();
+  warp_select(cs, ci, n, a.k, os, oi, lane);
+  __syncwarp();
+  if (lane < a.k) {
+    a.out_ids[(int64_t)q * a.k + lane] = oi[lane];
+    a.out_scores[(int64_t)q * a.k + lane] = os[lane];
+  }
+}
+
 int search_nsplit(int64_t n_db) {
   // each split should give every warp a few hundred keys; at most 32 splits (merge handles 1024 candidates)
   const int64_t per = 8192;
@@ -386,6 +425,44 @@ extern "C" int tq_search_topk(const tq_params* p, const float* q, int n_q, const
   merge_kernel<<<n_q, 32, msmem, st>>>(ma);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(TQ_ECUDA, "tq_search_topk: merge launch failed: %s", cudaGetErrorString(e));
+  clear_error();
+  return TQ_OK;
+}
+
+extern "C" int tq_search_merge(const int32_t* ids, const float* scores, int n_parts, const int64_t* id_offsets,
+                               int n_q, int k, int32_t* out_ids, float* out_scores, tq_stream_t stream) {
+  using namespace tq;
+  if (n_parts < 1 || n_parts > MAX_SHARDS || k < 1 || k > KM || n_parts * k > 1024 || n_q < 0)
+    return set_error(TQ_EINVAL, "tq_search_merge: need 1 <= n_parts <= %d, 1 <= k <= %d, n_parts * k <= 1024",
+                     MAX_SHARDS, KM);
+  if (n_q == 0) {
+    clear_error();
+    return TQ_OK;
+  }
+  if (!ids || !scores || !id_offsets || !out_ids || !out_scores)
+    return set_error(TQ_EINVAL, "tq_search_merge: NULL pointer argument");
+  if (!aligned(ids, 4) || !aligned(scores, 4) || !aligned(out_ids, 4) || !aligned(out_scores, 4))
+    return set_error(TQ_EINVAL, "tq_search_merge: misaligned pointer");
+  ShardMergeArgs a;
+  a.ids = ids;
+  a.scores = scores;
+  a.n_parts = n_parts;
+  a.n_q = n_q;
+  a.k = k;
+  for (int p = 0; p < MAX_SHARDS; ++p) a.offs[p] = 0;
+  for (int p = 0; p < n_parts; ++p) {
+    if (id_offsets[p] < 0 || id_offsets[p] >= INT_MAX)
+      return set_error(TQ_EINVAL, "tq_search_merge: id offset %lld out of range", (long long)id_offsets[p]);
+    a.offs[p] = id_offsets[p];
+  }
+  a.out_ids = out_ids;
+  a.out_scores = out_scores;
+  const int n = n_parts * k;
+  const int smem = (2 * n + 2 * KM) * 4;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  shard_merge_kernel<<<n_q, 32, smem, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(TQ_ECUDA, "tq_search_merge: launch failed: %s", cudaGetErrorString(e));
   clear_error();
   return TQ_OK;
 }
