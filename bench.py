@@ -34,6 +34,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 HBM_NOMINAL_GBS = 8000.0
+METRIC = "compressed-key logits keys/s and HBM GB/s (frac of 8 TB/s) at b=3,4"
+VALUE_DEF = ("keys per second through the whole step (tq_quantize of K and V, tq_logits of the 32 decode "
+             "queries), b=3 and b=4; tq_logits alone, with GB/s and fractions of 8 TB/s, under 'logits'")
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -47,6 +50,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-kernels", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
     return ap.parse_args()
 
 
@@ -422,6 +426,44 @@ def cpu_oracle_layer(sample_tokens=16384):
     return keys / dt, cores, dt, f"8 heads x {T} tokens (of 32768), b=3 and b=4: quantize K and V + logits"
 
 
+def cpu_oracle_one_core():
+    """The oracle on one host core (BLAS limited to one thread): config 0 whole (4096 fp32 keys,
+    16 queries, b = 4: quantize + logits) and a 16384-vector sample of config 3 (bf16, product
+    code at b = 2, 3, 4)."""
+    import workloads as wl
+    from oracle import codec, estimate
+    from oracle.codebook import stored_codebook
+    from oracle.params import sign_flips, qjl_matrix
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:
+        return None
+    with threadpool_limits(limits=1):
+        Dk, S = sign_flips(wl.SEED_PARAMS, 128), qjl_matrix(wl.SEED_PARAMS, 128, 128)
+        x = wl.head_vectors(4096, 128, seed=wl.SEED_KEYS, token_scale=False)
+        q = wl.queries(16, 128)
+        c, t = stored_codebook(128, 3)
+        t0 = time.perf_counter()
+        e = codec.encode(x, Dk, c, t, S)
+        buf = codec.pack(e["idx"], e["signs"], 3, 128)
+        idx, sg = codec.unpack(buf, 4096, 128, 3, 128)
+        estimate.logits_gqa(q, Dk, S, idx, sg, e["norm_f16"], e["rnorm_f16"], c, 128, 1, 16, 4096)
+        cfg0 = time.perf_counter() - t0
+        n3 = 16384
+        x3 = wl.to_bf16(wl.head_vectors(n3, 128, seed=wl.SEED_KEYS))
+        per = {}
+        for b in (2, 3, 4):
+            c, t = stored_codebook(128, b - 1)
+            t0 = time.perf_counter()
+            e = codec.encode(x3, Dk, c, t, S)
+            codec.pack(e["idx"], e["signs"], b - 1, 128)
+            per[f"b{b}"] = n3 / (time.perf_counter() - t0)
+    return {"cores": 1, "config0_seconds": round(cfg0, 3),
+            "config0": "4096 fp32 keys x 16 queries, b=4: quantize + logits",
+            "config3_vectors_per_s": {k: round(v, 1) for k, v in per.items()},
+            "config3_sample": f"{n3} of 2^20 bf16 vectors, product code m=128"}
+
+
 # --------------------------------------------------------------------------- traffic record
 def traffic_record(kernel_file_label):
     """ncu-derived DRAM bytes per launch from profiles/traffic.json, or None if the
@@ -454,6 +496,124 @@ def gpu_kv(torch, n_seq, n_heads, n_tokens, d, seed):
     return out.reshape(-1, d)
 
 
+def measure_decode(torch, tq, wl, steps, warmup, peak, sparse=True):
+    """Decode attention, 64 sequences x 8 KV heads x 16384 tokens, d 128, 32 query heads:
+    K product code b = 3, V MSE code b = 3 (inputs drawn on the GPU, then quantized)."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    B, Hkv, T, d, Hq = 64, 8, 16384, 128, 32
+    kp = tq.Params(d, 3, tq.TQ_MODE_PROD, 128, wl.SEED_PARAMS)
+    vp = tq.Params(d, 3, tq.TQ_MODE_MSE, 0, wl.SEED_PARAMS + 1)
+    n = B * Hkv * T
+    bufs = {}
+    for name, p, seed in (("k", kp, wl.SEED_KEYS), ("v", vp, wl.SEED_VALUES)):
+        x = gpu_kv(torch, B, Hkv, T, d, seed)
+        c = torch.empty(p.code_bytes(n), dtype=torch.uint8, device="cuda")
+        nn = torch.empty(n, dtype=torch.int16, device="cuda")
+        rn = torch.empty(n, dtype=torch.int16, device="cuda") if p.mode == tq.TQ_MODE_PROD else None
+        tq.tq_quantize(p, x, c, nn, rn)
+        torch.cuda.synchronize()
+        del x
+        bufs[name] = (c, nn, rn)
+    q = torch.randn((B, Hq, d), device="cuda")
+    out = torch.empty((B, Hq, d), device="cuda")
+    ws = torch.empty(tq.tq_decode_attn_workspace(kp, B, Hq, Hkv, T), dtype=torch.uint8, device="cuda")
+    sl = torch.full((B,), T, dtype=torch.int32, device="cuda")
+
+    def timed(run):
+        for _ in range(warmup):
+            run()
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record()
+        for _ in range(steps):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    ms = timed(lambda: tq.tq_decode_attn(kp, vp, q, Hkv, bufs["k"][0], bufs["k"][1], bufs["k"][2], bufs["v"][0],
+                                         bufs["v"][1], sl, T, out, ws))
+    mbytes = bufs["k"][0].numel() + 4 * n + bufs["v"][0].numel() + 2 * n + q.numel() * 4
+    gbs = mbytes / (ms / 1e3) / 1e9
+    res = {"us": round(ms * 1000, 2), "tokens_per_s": n / (ms / 1e3), "metric_bytes": mbytes, "gbs": round(gbs, 1),
+           "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4), "frac_measured": round(gbs / peak, 4),
+           "workload": "decode-64x8x16384-Kprod3-Vmse3-hq32", "inputs": "> L2 (856 MB of codes)"}
+    if sparse:
+        sp = {}
+        for eps in (1e-4, 1e-3):
+            ms_s = timed(lambda: tq.tq_decode_attn_sparse(kp, vp, q, Hkv, bufs["k"][0], bufs["k"][1], bufs["k"][2],
+                                                          bufs["v"][0], bufs["v"][1], sl, T, out, ws, v_eps=eps))
+            sp[f"v_eps={eps:g}"] = {"us": round(ms_s * 1000, 2), "tokens_per_s": n / (ms_s / 1e3)}
+        res["sparse_v"] = sp
+    del bufs, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_quantize(torch, tq, wl, steps, warmup, peak):
+    """tq_quantize on 2^20 bf16 vectors, d 128, product code m = 128, at b = 2, 3, 4
+    (268 MB of input per call: larger than L2)."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    n, d = 1 << 20, 128
+    x = gpu_kv(torch, 1, 8, n // 8, d, wl.SEED_KEYS)
+    res = {}
+    for b in (2, 3, 4):
+        p = tq.Params(d, b, tq.TQ_MODE_PROD, 128, wl.SEED_PARAMS)
+        c = torch.empty(p.code_bytes(n), dtype=torch.uint8, device="cuda")
+        nn = torch.empty(n, dtype=torch.int16, device="cuda")
+        rn = torch.empty(n, dtype=torch.int16, device="cuda")
+        run = lambda: tq.tq_quantize(p, x, c, nn, rn)
+        for _ in range(warmup):
+            run()
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record()
+        for _ in range(steps):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        byts = n * d * 2 + c.numel() + 4 * n
+        gbs = byts / (ms / 1e3) / 1e9
+        res[f"b{b}"] = {"us": round(ms * 1000, 2), "vectors_per_s": n / (ms / 1e3), "gbs": round(gbs, 1),
+                        "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4), "frac_measured": round(gbs / peak, 4)}
+    del x
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_config0(torch, tq, wl, reps=50):
+    """Single head, d 128: 4096 fp32 keys (per-channel law, no per-token scale), 16 queries,
+    b = 4 product code: absolute latency of tq_quantize and tq_logits (median of `reps`)."""
+    d, n, nq = 128, 4096, 16
+    x = torch.from_numpy(wl.head_vectors(n, d, seed=wl.SEED_KEYS, token_scale=False)).cuda()
+    q = torch.from_numpy(wl.queries(nq, d)).cuda()
+    p = tq.Params(d, 4, tq.TQ_MODE_PROD, 128, wl.SEED_PARAMS)
+    c = torch.empty(p.code_bytes(n), dtype=torch.uint8, device="cuda")
+    nn = torch.empty(n, dtype=torch.int16, device="cuda")
+    rn = torch.empty(n, dtype=torch.int16, device="cuda")
+    lg = torch.empty((nq, n), device="cuda")
+    ws = torch.empty(tq.tq_logits_workspace(p, nq), dtype=torch.uint8, device="cuda")
+    calls = {"tq_quantize": lambda: tq.tq_quantize(p, x, c, nn, rn),
+             "tq_logits": lambda: tq.tq_logits(p, q, nq, c, nn, rn, n, 1, lg, ws)}
+    res = {}
+    for name, f in calls.items():
+        for _ in range(5):
+            f()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1000)
+        res[name + "_us"] = round(statistics.median(ts), 2)
+    res["workload"] = "single-head-4096x128-fp32-16q-b4"
+    return res
+
+
 def run_secondary(args, world, rank, local, torch, tq, wl):
     """Other workloads (their own JSON line): 'decode' = 64 sequences x 8 KV heads x 16384 tokens
     (K product b=3, V MSE b=3, 32 query heads); 'quantize' = 2^20 bf16 vectors at b=2,3,4;
@@ -462,82 +622,12 @@ def run_secondary(args, world, rank, local, torch, tq, wl):
     peak, peak_kind = measured_peaks()
     ev = lambda: torch.cuda.Event(enable_timing=True)
     if args.workload == "decode":
-        B, Hkv, T, d, Hq = 64, 8, 16384, 128, 32
-        kp = tq.Params(d, 3, tq.TQ_MODE_PROD, 128, wl.SEED_PARAMS)
-        vp = tq.Params(d, 3, tq.TQ_MODE_MSE, 0, wl.SEED_PARAMS + 1)
-        n = B * Hkv * T
-        bufs = {}
-        for name, p, seed in (("k", kp, wl.SEED_KEYS), ("v", vp, wl.SEED_VALUES)):
-            x = gpu_kv(torch, B, Hkv, T, d, seed)
-            c = torch.empty(p.code_bytes(n), dtype=torch.uint8, device="cuda")
-            nn = torch.empty(n, dtype=torch.int16, device="cuda")
-            rn = torch.empty(n, dtype=torch.int16, device="cuda") if p.mode == tq.TQ_MODE_PROD else None
-            tq.tq_quantize(p, x, c, nn, rn)
-            torch.cuda.synchronize()
-            del x
-            bufs[name] = (c, nn, rn)
-        q = torch.randn((B, Hq, d), device="cuda")
-        out = torch.empty((B, Hq, d), device="cuda")
-        ws = torch.empty(tq.tq_decode_attn_workspace(kp, B, Hq, Hkv, T), dtype=torch.uint8, device="cuda")
-        sl = torch.full((B,), T, dtype=torch.int32, device="cuda")
-        run = lambda: tq.tq_decode_attn(kp, vp, q, Hkv, bufs["k"][0], bufs["k"][1], bufs["k"][2], bufs["v"][0],
-                                        bufs["v"][1], sl, T, out, ws)
-        for _ in range(args.warmup):
-            run()
-        torch.cuda.synchronize()
-        e0, e1 = ev(), ev()
-        e0.record()
-        for _ in range(args.steps):
-            run()
-        e1.record()
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / args.steps
-        mbytes = bufs["k"][0].numel() + 4 * n + bufs["v"][0].numel() + 2 * n + q.numel() * 4
-        gbs = mbytes / (ms / 1e3) / 1e9
-        line = {"metric": "decode attention tokens/s", "value": n / (ms / 1e3), "unit": "tokens/s",
-                "ms_per_step": ms, "config": {"workload": "decode-64x8x16384-Kprod3-Vmse3-hq32"},
-                "metric_bytes": mbytes, "gbs": round(gbs, 1), "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4),
-                "frac_measured": round(gbs / peak, 4)}
-        # Sparse V: same step, tokens whose attention weight is below v_eps add no value
-        sparse = {}
-        for eps in (1e-4, 1e-3):
-            run_s = lambda: tq.tq_decode_attn_sparse(kp, vp, q, Hkv, bufs["k"][0], bufs["k"][1], bufs["k"][2],
-                                                     bufs["v"][0], bufs["v"][1], sl, T, out, ws, v_eps=eps)
-            for _ in range(args.warmup):
-                run_s()
-            torch.cuda.synchronize()
-            e0.record()
-            for _ in range(args.steps):
-                run_s()
-            e1.record()
-            torch.cuda.synchronize()
-            ms_s = e0.elapsed_time(e1) / args.steps
-            sparse[f"v_eps={eps:g}"] = {"ms_per_step": round(ms_s, 4), "tokens_per_s": n / (ms_s / 1e3)}
-        line["sparse_v"] = sparse
+        r = measure_decode(torch, tq, wl, args.steps, args.warmup, peak)
+        n = 64 * 8 * 16384
+        line = {"metric": "decode attention tokens/s", "value": r["tokens_per_s"], "unit": "tokens/s",
+                "ms_per_step": r["us"] / 1000, "config": {"workload": r["workload"]}, "decode": r}
     elif args.workload == "quantize":
-        n, d = 1 << 20, 128
-        x = gpu_kv(torch, 1, 8, n // 8, d, wl.SEED_KEYS)
-        res = {}
-        for b in (2, 3, 4):
-            p = tq.Params(d, b, tq.TQ_MODE_PROD, 128, wl.SEED_PARAMS)
-            c = torch.empty(p.code_bytes(n), dtype=torch.uint8, device="cuda")
-            nn = torch.empty(n, dtype=torch.int16, device="cuda")
-            rn = torch.empty(n, dtype=torch.int16, device="cuda")
-            run = lambda: tq.tq_quantize(p, x, c, nn, rn)
-            for _ in range(args.warmup):
-                run()
-            torch.cuda.synchronize()
-            e0, e1 = ev(), ev()
-            e0.record()
-            for _ in range(args.steps):
-                run()
-            e1.record()
-            torch.cuda.synchronize()
-            ms = e0.elapsed_time(e1) / args.steps
-            byts = n * d * 2 + c.numel() + 4 * n
-            gbs = byts / (ms / 1e3) / 1e9
-            res[f"b{b}"] = {"us": round(ms * 1000, 2), "vectors_per_s": n / (ms / 1e3), "gbs": round(gbs, 1),
-                            "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4), "frac_measured": round(gbs / peak, 4)}
+        res = measure_quantize(torch, tq, wl, args.steps, args.warmup, peak)
         line = {"metric": "quantize vectors/s", "value": res["b4"]["vectors_per_s"], "unit": "vectors/s",
                 "config": {"workload": "quantize-2^20x128-bf16-prod-m128"}, "per_bits": res}
     elif args.workload == "polar":
@@ -594,11 +684,16 @@ def run_secondary(args, world, rank, local, torch, tq, wl):
             nn = torch.empty(n_db, dtype=torch.int16, device="cuda")
             rn = torch.empty(n_db, dtype=torch.int16, device="cuda")
             e0, e1 = ev(), ev()
+            for _ in range(3):  # warm-up
+                tq.tq_quantize(p, db, c, nn, rn)
+            torch.cuda.synchronize()
+            q_reps = 10
             e0.record()
-            tq.tq_quantize(p, db, c, nn, rn)
+            for _ in range(q_reps):
+                tq.tq_quantize(p, db, c, nn, rn)
             e1.record()
             torch.cuda.synchronize()
-            q_ms = e0.elapsed_time(e1)
+            q_ms = e0.elapsed_time(e1) / q_reps
             ids = torch.empty((n_q, k), dtype=torch.int32, device="cuda")
             scs = torch.empty((n_q, k), dtype=torch.float32, device="cuda")
             ws = torch.empty(tq.tq_search_workspace(p, n_q, n_db, k), dtype=torch.uint8, device="cuda")
@@ -614,8 +709,11 @@ def run_secondary(args, world, rank, local, torch, tq, wl):
             ms = e0.elapsed_time(e1) / args.steps
             got = ids.cpu().numpy()
             recall = float(np.mean([len(set(got[i]) & set(truth[i])) / k for i in range(n_q)]))
+            q_bytes = n_db * d * 2 + c.numel() + 4 * n_db
             res[f"b{b}"] = {"search_ms": round(ms, 3), "estimates_per_s": n_q * n_db / (ms / 1e3),
-                            "recall_at_10": round(recall, 4), "quantize_db_ms": round(q_ms, 3)}
+                            "recall_at_10": round(recall, 4), "quantize_db_ms": round(q_ms, 3),
+                            "quantize_db_gbs": round(q_bytes / (q_ms / 1e3) / 1e9, 1),
+                            "quantize_db": "warm, mean of 10 calls after 3 warm-up calls"}
         line = {"metric": "search estimates/s", "value": res["b4"]["estimates_per_s"], "unit": "estimates/s",
                 "config": {"workload": "search-1e6x200-1e4q-top10"}, "per_bits": res}
     else:
@@ -626,6 +724,12 @@ def run_secondary(args, world, rank, local, torch, tq, wl):
 
 
 # --------------------------------------------------------------------------- main
+def layer_config(world):
+    return {"workload": "llama3.1-8b-layer-kv8x32768-gqa4-d128", "kv_heads": 8, "tokens": 32768, "q_heads": 32,
+            "d": 128, "bits": [3, 4], "kv_dtype": "bf16", "value": VALUE_DEF,
+            "l2": "flushed between steps (256 MB write)", "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -638,11 +742,10 @@ def run_reference(args):
         v, cores, dt, sample = cpu_oracle_layer(sample_tokens=2048)
         vals.append(v)
     v = statistics.median(vals)
-    line = {"impl": "reference", "metric": "compressed-key logits keys/s (whole step, b=3 and b=4)",
+    line = {"impl": "reference", "metric": METRIC,
             "value": v, "unit": "keys/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "llama3.1-8b-layer-kv8x32768-gqa4-d128", "kv_heads": 8, "tokens": 32768,
-                       "q_heads": 32, "d": 128, "bits": [3, 4]},
+            "config": layer_config(world),
             "cpu_baseline": {"value": v, "unit": "keys/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -691,14 +794,27 @@ def main():
         avg = statistics.mean(times)
         gbs = wk.bytes_of(label) / (avg / 1e3) / 1e9
         kernels[label] = {"us": round(avg * 1000, 2), "gbs": round(gbs, 1), "frac_measured": round(gbs / peak, 4)}
+    logits = None
     if not args.no_kernels:
         iso = logits_isolated(torch, tq, wk)
+        logits = {}
         for b, (us, mb, lat) in iso.items():
             gbs = mb / (us / 1e6) / 1e9
             kernels[f"tq_logits_b{b}_l2cold"] = {
                 "us": round(us, 2), "keys_per_s": round(wk.n / (us / 1e6)), "gbs": round(gbs, 1),
                 "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4), "frac_measured": round(gbs / peak, 4),
                 "single_launch_us": round(lat, 2)}
+            logits[f"b{b}"] = {"keys_per_s": round(wk.n / (us / 1e6)), "gbs": round(gbs, 1),
+                               "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4), "frac_measured": round(gbs / peak, 4),
+                               "us_per_call": round(us, 2), "metric_bytes": int(mb)}
+        logits["how"] = ("tq_logits alone (query preparation included), one call per distinct copy of the codes; "
+                         f"copies total > 4x L2, launches captured in a CUDA graph")
+
+    configs = None
+    if not args.no_configs:
+        configs = {"config0_latency": measure_config0(torch, tq, wl),
+                   "quantize_2^20": measure_quantize(torch, tq, wl, max(5, args.steps // 2), 3, peak),
+                   "decode": measure_decode(torch, tq, wl, max(5, args.steps // 2), 3, peak, sparse=False)}
 
     e2e = None
     if not args.no_e2e:
@@ -710,16 +826,15 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu:
         v, cores, dt, sample = cpu_oracle_layer()
         cpu = {"value": v, "unit": "keys/s", "cores": cores, "kind": "oracle", "sample": sample,
-               "seconds": round(dt, 2)}
+               "seconds": round(dt, 2), "one_core": cpu_oracle_one_core()}
     if rank == 0:
-        line = {"metric": "compressed-key logits keys/s (whole step, b=3 and b=4)", "value": value, "unit": "keys/s",
+        line = {"metric": METRIC, "value": value, "unit": "keys/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 4),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32+s8",
                 "data": "synthetic",
-                "config": {"workload": "llama3.1-8b-layer-kv8x32768-gqa4-d128", "kv_heads": 8, "tokens": 32768,
-                           "q_heads": 32, "d": 128, "bits": [3, 4], "kv_dtype": "bf16",
-                           "l2": "flushed between steps (256 MB write)", "parallelism": f"replicas x{world}"},
-                "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+                "config": layer_config(world),
+                "roofline": roofline, "logits": logits, "kernels": kernels, "configs": configs,
+                "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": wk.launches_per_step * args.steps, "clocks": clocks}
         print(json.dumps(line), flush=True)
     if world > 1:
