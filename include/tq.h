@@ -193,14 +193,21 @@ int tq_logits_ld(const tq_params* p, const float* q, int n_q, int group, const v
  * allocate device memory when they call (for example code that runs while a
  * CUDA graph is being captured, or a plugin whose host framework owns every
  * device buffer and passes only inputs and outputs).  Same arguments and
- * results as tq_logits minus the workspace; the query-prep scratch is a
- * static device array of tq_logits_noalloc_max_scratch() bytes (1 MiB) that
- * every device loading the library keeps until the process exits.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current) and caches it; make
- *    that first call before any stream capture.
- *  - Calls needing more scratch than the array (more than about 300 query
- *    heads at d_pad 128) return TQ_EINVAL with a message; nothing is launched.
+ * results as tq_logits minus the workspace.  Shapes that tq_logits serves on
+ * its tensor-core path need no scratch at all; the others keep their query
+ * preparation in a static device array of tq_logits_noalloc_max_scratch()
+ * bytes (1 MiB) that every device loading the library keeps until the
+ * process exits.
+ *  - The array's device address is looked up (cudaGetSymbolAddress, with the
+ *    device current) on the first call on a device, and again whenever the
+ *    current driver context differs from the one of the last lookup (after a
+ *    cudaDeviceReset, or under a non-primary context); make the first call on
+ *    a device before any stream capture.
+ *  - Scratch needed on the other shapes: n_kv_heads * ceil(group / 4) chunks
+ *    of 128*fr + 64 bytes, fr = 8 * 4 * (mma slots per bit class); at d_pad 128
+ *    a chunk is 12352 bytes at b = 4 (product code, m = 128) and 8256 bytes at
+ *    b = 3, so 1 MiB holds 84 and 127 chunks.  Calls needing more return
+ *    TQ_EINVAL with a message; nothing is launched.
  *  - All calls share the one array: calls that may overlap on the GPU (other
  *    streams, other host threads) race and must be serialised by the caller.
  *    The scratch is fully rewritten by each call, so nothing needs clearing.
@@ -388,7 +395,8 @@ int64_t tq_polar_table_floats(int d_pad, int w);
  * quadrature in fp64; centroids rounded to fp32.  TQ_EINVAL on bad arguments. */
 int tq_polar_make_tables(int d_pad, int w, float* tables);
 
-/* Bytes of a polar code buffer holding n_vec records. */
+/* Bytes of a polar code buffer holding n_vec records of w * d_pad / 8 bytes
+ * (d_pad a power of two >= 8; -1 for other arguments). */
 int64_t tq_polar_code_bytes(int d_pad, int w, int64_t n_vec);
 
 /*

@@ -223,7 +223,8 @@ def boundary_flags(enc, w, d_pad, tabs=None, rel=1e-6):
 
 
 def record_bytes(d_pad, w):
-    return int(w) * int(d_pad) // 8
+    """Bytes of one record: w * d_pad bits, rounded up to whole bytes (exact for d_pad >= 8)."""
+    return (int(w) * int(d_pad) + 7) // 8
 
 
 def pack(i1, ihi, w, d_pad):

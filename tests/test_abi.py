@@ -147,6 +147,11 @@ def test_polar_tables_match_oracle(d_pad, w):
 
 def test_polar_sizes_and_validation():
     assert tq.tq_polar_code_bytes(128, 2, 10) == 10 * 32
+    # a record is w * d_pad / 8 whole bytes: d_pad 8 is the smallest (w = 1: one byte)
+    assert tq.tq_polar_code_bytes(8, 1, 3) == 3
+    assert tq.tq_polar_code_bytes(8, 3, 3) == 9
+    for w in (1, 2, 3):
+        assert tq.tq_polar_code_bytes(4, w, 1) == -1
     assert tq._lib.tq_polar_table_floats(100, 2) == -1
     assert tq._lib.tq_polar_table_floats(128, 4) == -1
     bad = tq.tq_polar_params(128, 128, 4, 0, None, None)

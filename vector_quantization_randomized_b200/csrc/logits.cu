@@ -404,20 +404,42 @@ __device__ __align__(256) uint8_t g_logits_scratch[kNoAllocScratchBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
+void* g_scratch_ctx[kMaxDevices] = {};  // the driver context the address was looked up in
 
-// Device address of the static scratch on the current device, looked up once per device.
+// The current driver context (cuCtxGetCurrent through the runtime's driver entry point, so
+// the library does not link the driver library itself); nullptr when unavailable.
+void* current_context() {
+  using GetCtx = int (*)(void**);
+  static GetCtx fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<GetCtx>(f);
+  }();
+  void* ctx = nullptr;
+  if (fn && fn(&ctx) != 0) ctx = nullptr;
+  return ctx;
+}
+
+// Device address of the static scratch on the current device.  It is looked up once per
+// device and looked up again when the current driver context is not the one it was found
+// in (after cudaDeviceReset, or under a context other than the device's primary one).
 int scratch_on_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_logits_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return tq::set_error(TQ_EUNSUPPORTED, "tq_logits_noalloc: device index %d", dev);
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_logits_scratch);
     if (e != cudaSuccess || !ptr)
       return tq::set_error(TQ_ECUDA, "tq_logits_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
     g_scratch_ptr[dev] = ptr;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return TQ_OK;
@@ -436,8 +458,11 @@ extern "C" int tq_logits_noalloc(const tq_params* p, const float* q, int n_q, in
   if (group < 1 || n_kv_heads < 1 || (int64_t)n_kv_heads * group != n_q)
     return set_error(TQ_EINVAL, "tq_logits_noalloc: need n_q == n_kv_heads * group");
   const int kb = index_bits(p);
-  const int64_t need = (int64_t)n_kv_heads * ((group + tqd::QCHUNK - 1) / tqd::QCHUNK) *
-                       prep_chunk_bytes_max(p->d_pad, kb, p->mode == TQ_MODE_PROD ? p->m : 0);
+  const int m = p->mode == TQ_MODE_PROD ? p->m : 0;
+  // the tensor-core path prepares its queries inside the kernel; the other shapes use the scratch
+  const bool tc = logits_tc_supported(p->d_pad, kb, m, group, n_keys, norms, rnorms);
+  const int64_t need =
+      tc ? 0 : (int64_t)n_kv_heads * ((group + tqd::QCHUNK - 1) / tqd::QCHUNK) * prep_chunk_bytes_max(p->d_pad, kb, m);
   if (need > kNoAllocScratchBytes)
     return set_error(TQ_EINVAL,
                      "tq_logits_noalloc: %d query heads need %lld bytes of scratch, above the static %lld; "

@@ -120,7 +120,8 @@ extern "C" int64_t tq_polar_table_floats(int d_pad, int w) {
 }
 
 extern "C" int64_t tq_polar_code_bytes(int d_pad, int w, int64_t n_vec) {
-  if (!tq::is_pow2(d_pad) || d_pad < 4 || w < 1 || w > 3 || n_vec < 0) return -1;
+  // a record is w * d_pad / 8 whole bytes, so d_pad >= 8 (d_pad 4 at w = 1 would be half a byte)
+  if (!tq::is_pow2(d_pad) || d_pad < 8 || w < 1 || w > 3 || n_vec < 0) return -1;
   return n_vec * (int64_t)w * d_pad / 8;
 }
 
