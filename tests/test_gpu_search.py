@@ -15,19 +15,19 @@ from gpu_util import make_pair, oracle_codes
 pytestmark = pytest.mark.gpu
 
 
-def _check(d, bits, n_db, n_q, k, seed=0):
-    p, op = make_pair(d, bits, tq.TQ_MODE_PROD, seed=42)
+def _check(d, bits, n_db, n_q, k, seed=0, mode=tq.TQ_MODE_PROD):
+    p, op = make_pair(d, bits, mode, seed=42)
     db = wl.to_bf16(wl.search_set(n_db, d, seed=seed))
     q = wl.search_set(n_q, d, seed=seed + 1)
     codes, norms, rnorms, enc = oracle_codes(op, db)
     q_rot, u = estimate.prep_queries(q, op.D, op.S)
-    ref = estimate.logits_from_codes(q_rot, u, enc["idx"], enc["signs"], norms, rnorms, op.c, op.m)
+    ref = estimate.logits_from_codes(q_rot, u, enc["idx"], enc.get("signs"), norms, rnorms, op.c, op.m)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     ids = torch.full((n_q, k), -7, dtype=torch.int32, device="cuda")
     sc = torch.full((n_q, k), float("nan"), dtype=torch.float32, device="cuda")
     ws = torch.empty(tq.tq_search_workspace(p, n_q, n_db, k), dtype=torch.uint8, device="cuda")
-    tq.tq_search_topk(p, dev(q), dev(codes), dev(norms.view(np.int16)), dev(rnorms.view(np.int16)), n_db, k, ids,
-                      sc, ws)
+    tq.tq_search_topk(p, dev(q), dev(codes), dev(norms.view(np.int16)),
+                      dev(rnorms.view(np.int16)) if rnorms is not None else None, n_db, k, ids, sc, ws)
     gi = ids.cpu().numpy().astype(np.int64)
     gs = sc.cpu().numpy().astype(np.float64)
     qn = np.linalg.norm(q.astype(np.float64), axis=1)
@@ -47,9 +47,15 @@ def _check(d, bits, n_db, n_q, k, seed=0):
         assert must <= got <= may, (r, sorted(must - got), sorted(got - may))
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 def test_search_d200(bits):
     _check(200, bits, n_db=20000, n_q=37, k=10)
+
+
+def test_search_d200_mse_codes_many_splits():
+    """MSE-only codes (no sign plane); 40000 vectors make three database splits whose last
+    item is ragged, and 33 queries three chunks of 16 (the last one with one query)."""
+    _check(200, 3, n_db=40003, n_q=33, k=16, seed=3, mode=tq.TQ_MODE_MSE)
 
 
 def test_search_d128_b4():

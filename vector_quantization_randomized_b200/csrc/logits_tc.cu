@@ -116,20 +116,6 @@ __device__ __forceinline__ float pow2(int k) {
   return (k >= -126 && k <= 127) ? __uint_as_float((uint32_t)(127 + k) << 23) : ldexpf(1.f, k);
 }
 
-// Barrier over the 8 query-prep / epilogue warps on an mbarrier (8 arrivals):
-// unlike bar.sync its wait has an iteration limit, so a stalled partner sets the
-// fault word instead of hanging the CTA.
-struct GroupSync {
-  uint64_t* bar;
-  uint32_t phase;
-  __device__ __forceinline__ void sync(int lane) {
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar);
-    mbar_wait(bar, phase);
-    phase ^= 1u;
-  }
-};
-
 // B image of KV head `head` into `img`, by the 256 threads of warps 13-20
 // (et = 0..255).  Steps: q_rot = H D q / sqrt(128) (warp per query);
 // u = S q_rot (thread = row of S x half of the coordinates); per-query scales

@@ -17,6 +17,13 @@ bool logits_tc_supported(int dp, int kb, int m, int group, int64_t n_keys, const
 int launch_logits_tc(int kb, int m, const float* q, int d, const float* cent, const int8_t* D, const uint16_t* S,
                      const void* codes, const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys,
                      int n_kv_heads, int group, float* logits, int64_t ld, cudaStream_t st);
+// The tensor-memory search (search_tc.cu): supported shapes, workspace, and the
+// prep + scan launch that leaves [n_q][*nsplit][16] candidates for the split merge.
+bool search_tc_supported(int dp, int kb, int m);
+int64_t search_tc_workspace(int kb, int m, int n_q, int64_t n_db);
+int launch_search_tc(const tq_params* p, int kb, const float* q, int n_q, const void* codes, const uint16_t* norms,
+                     const uint16_t* rnorms, int64_t n_db, void* workspace, float2** cand, int* nsplit,
+                     cudaStream_t st);
 // Bytes of query-prep scratch per chunk of 4 queries, the larger of both layouts.
 int64_t prep_chunk_bytes_max(int dp, int kb, int m);
 }  // namespace tq

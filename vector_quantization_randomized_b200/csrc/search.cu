@@ -338,6 +338,8 @@ extern "C" int64_t tq_search_workspace(const tq_params* p, int n_q, int64_t n_db
   if (!p || n_q < 0 || n_db < 0 || k < 1) return -1;
   const int kb = p->mode == TQ_MODE_PROD ? p->bits - 1 : p->bits;
   if (kb < 1 || kb > 4 || (p->d_pad != 128 && p->d_pad != 256)) return -1;
+  const int m = p->mode == TQ_MODE_PROD ? p->m : 0;
+  if (tq::search_tc_supported(p->d_pad, kb, m)) return tq::search_tc_workspace(kb, m, n_q, n_db);
   return prep_bytes_for(p, n_q) + (int64_t)n_q * search_nsplit(n_db) * KM * 8;
 }
 
@@ -369,6 +371,25 @@ extern "C" int tq_search_topk(const tq_params* p, const float* q, int n_q, const
   const tqd::ScanShape sh(p->d_pad, kb, m);
   const int nqc = (n_q + tqd::QCHUNK - 1) / tqd::QCHUNK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (search_tc_supported(p->d_pad, kb, m)) {  // tensor-memory scan, then the split merge
+    float2* cand = nullptr;
+    int nsplit = 0;
+    rc = launch_search_tc(p, kb, q, n_q, codes, norms, rnorms, n_db, workspace, &cand, &nsplit, st);
+    if (rc) return rc;
+    MArgs ma;
+    ma.cand = cand;
+    ma.n_q = n_q;
+    ma.nsplit = nsplit;
+    ma.k = k;
+    ma.ids = ids;
+    ma.scores = scores;
+    const int msmem = (2 * nsplit * KM + 2 * KM) * 4;
+    merge_kernel<<<n_q, 32, msmem, st>>>(ma);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(TQ_ECUDA, "tq_search_topk: merge launch failed: %s", cudaGetErrorString(e));
+    clear_error();
+    return TQ_OK;
+  }
   tqd::PrepArgs pa;
   pa.q = q;
   pa.d = p->d;

@@ -236,4 +236,19 @@ __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
 }
 
+// Barrier over `count` warps on an mbarrier initialised with that count: unlike
+// bar.sync its wait has an iteration limit, so a stalled partner sets the fault
+// word instead of hanging the CTA.  Every participating warp calls sync() the
+// same number of times.
+struct GroupSync {
+  uint64_t* bar;
+  uint32_t phase;
+  __device__ __forceinline__ void sync(int lane) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+    mbar_wait(bar, phase);
+    phase ^= 1u;
+  }
+};
+
 }  // namespace tqd
