@@ -425,6 +425,34 @@ int tq_polar_dequantize(const tq_polar_params* p, const void* codes, const uint1
 int tq_polar_logits(const tq_polar_params* p, const float* q, int group, const void* codes,
                     const uint16_t* norms, int64_t n_keys, int n_kv_heads, float* logits, tq_stream_t stream);
 
+/*
+ * tq_polar_qjl - the QJL stage on the polar code's residual [E 第二步 applied
+ *   to the polar stage 1 of E 第一步]: after tq_polar_quantize of the same x,
+ *   r = y - y_hat (y the rotated unit vector, y_hat rebuilt from the records
+ *   with unit radius), gamma = ||r||, and the sign bits of S r.  Together with
+ *   the polar record this is the product code of the polar stage: w bits per
+ *   coordinate plus one bit per projection.
+ *   S: device fp16 [m][d_pad] (tq_make_params with the same d_pad), m a
+ *      multiple of 32 in [32, d_pad].
+ *   x, dtype, ld: as tq_polar_quantize; codes: its records (read).
+ *   signs: device, n_vec * m / 8 bytes, 4-byte aligned: vector v's bits at
+ *      byte v*m/8, bit i at bit i%32 of little-endian word i/32, bit = [(S r)_i >= 0].
+ *   rnorms: device fp16 [n_vec], gamma.
+ */
+int tq_polar_qjl(const tq_polar_params* p, const uint16_t* S, int m, const void* x, int dtype, int64_t n_vec,
+                 int64_t ld, const void* codes, void* signs, uint16_t* rnorms, tq_stream_t stream);
+
+/*
+ * tq_polar_logits_prod - logits of the polar product code, unbiased over S:
+ *   l[h][k] = n_k ( <q~_h, y_hat_k> + gamma_k sqrt(pi/2)/m <S q~_h, 2 s_k - 1> ).
+ *   Arguments as tq_polar_logits plus S, m (as tq_polar_qjl), signs and
+ *   rnorms (from tq_polar_qjl).  Writes the stage-1 logits, then adds the QJL
+ *   term in a second kernel.
+ */
+int tq_polar_logits_prod(const tq_polar_params* p, const uint16_t* S, int m, const float* q, int group,
+                         const void* codes, const uint16_t* norms, const void* signs, const uint16_t* rnorms,
+                         int64_t n_keys, int n_kv_heads, float* logits, tq_stream_t stream);
+
 /* Message for the last failed call on this thread ("" if none). */
 const char* tq_last_error(void);
 

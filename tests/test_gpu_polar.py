@@ -168,3 +168,74 @@ def test_layer_full_size_sampled(w):
                            tabs)[0]
         tol = logit_tolerance(ref[None, :], enc["norm_f16"][sel], q[h:h + 1])[0]
         assert np.all(np.abs(got[h, rows[sel] % T] - ref) <= tol), h
+
+
+# ---- QJL stage on the polar residual (product code of the polar stage) -----------------
+def _qjl_S(d_pad, m):
+    from oracle.params import qjl_matrix
+    kp = tq.Params(d_pad, 4, tq.TQ_MODE_PROD, m, 42, d_pad)   # the library's S for this seed (device fp16)
+    return kp.S, qjl_matrix(42, m, d_pad)
+
+
+@pytest.mark.parametrize("w,d,dtype", [(1, 128, torch.bfloat16), (2, 128, torch.bfloat16), (3, 128, torch.float16),
+                                       (2, 200, torch.float32)])
+def test_qjl_encode(w, d, dtype):
+    """tq_polar_qjl after tq_polar_quantize against polar.encode_prod: sign bits exact except
+    projections within 1e-6 ||S_i|| gamma of zero (codec.boundary_flags' rule), gamma exact
+    except fp16 ties, on every vector whose angle indices equal the oracle's."""
+    n = 777
+    x = wl.to_bf16(wl.head_vectors(n, 128, seed=11)) if d == 128 else wl.search_set(n, d, seed=11).astype(np.float32)
+    p = tq.PolarParams(d, w, seed=42)
+    D, tabs, d_pad = _oracle(d, w)
+    m = d_pad
+    S_dev, S_or = _qjl_S(d_pad, m)
+    xt = torch.from_numpy(x).to(dtype)
+    xin = xt.float().numpy().astype(np.float64)
+    codes = torch.zeros(p.code_bytes(n), dtype=torch.uint8, device="cuda")
+    norms = torch.zeros(n, dtype=torch.int16, device="cuda")
+    signs = torch.full((n * m // 8,), 0xAB, dtype=torch.uint8, device="cuda")
+    rn = torch.zeros(n, dtype=torch.int16, device="cuda")
+    tq.tq_polar_quantize(p, xt.cuda(), codes, norms)
+    tq.tq_polar_qjl(p, S_dev, m, xt.cuda(), codes, signs, rn)
+    torch.cuda.synchronize()
+    enc = polar.encode_prod(xin, D, w, S_or, tabs)
+    i1, ihi = polar.unpack(codes.cpu().numpy(), n, w, d_pad)
+    same = np.all(i1 == enc["i1"], axis=1)
+    for a, b in zip(ihi, enc["ihi"]):
+        same &= np.all(a == b, axis=1)
+    assert same.mean() > 0.99
+    got = np.unpackbits(signs.cpu().numpy().reshape(n, m // 8), axis=1, bitorder="little")
+    fl = codec.boundary_flags(dict(y=enc["y"], norm=enc["norm"], gamma=enc["gamma"], z=enc["z"]),
+                              np.zeros(0, np.float32), S_or)["signs"]
+    bad = (got != enc["signs"]) & ~fl & same[:, None]
+    assert not np.any(bad), np.argwhere(bad)[:5]
+    g = rn.cpu().numpy().view(np.float16)
+    tie = codec.f16_tie_flags(enc["gamma"])
+    ok = (g == enc["rnorm_f16"]) | (tie & f16_neighbours(g, enc["rnorm_f16"])) | ~same
+    assert np.all(ok)
+
+
+@pytest.mark.parametrize("w,group,heads,n_keys", [(2, 4, 3, 1000), (3, 1, 2, 300), (1, 8, 1, 129)])
+def test_qjl_logits(w, group, heads, n_keys):
+    """tq_polar_logits_prod on oracle-made records, signs and gamma against polar.logits_prod."""
+    x = np.concatenate([wl.head_vectors(n_keys, 128, seed=12, head=h) for h in range(heads)])
+    D, tabs, d_pad = _oracle(128, w)
+    m = 128
+    S_dev, S_or = _qjl_S(d_pad, m)
+    enc = polar.encode_prod(x, D, w, S_or, tabs)
+    buf = polar.pack(enc["i1"], enc["ihi"], w, d_pad).ravel()
+    sbytes = np.packbits(enc["signs"], axis=1, bitorder="little").ravel()
+    q = wl.queries(heads * group, 128, seed=13)
+    p = tq.PolarParams(128, w, seed=42)
+    out = torch.full((heads * group, n_keys), float("nan"), device="cuda")
+    tq.tq_polar_logits_prod(p, S_dev, m, dev(q.astype(np.float32)), group, dev(buf),
+                            dev(enc["norm_f16"].view(np.int16)), dev(sbytes), dev(enc["rnorm_f16"].view(np.int16)),
+                            n_keys, heads, out)
+    got = out.cpu().numpy().astype(np.float64)
+    for h in range(heads * group):
+        gk = h // group
+        sl = slice(gk * n_keys, (gk + 1) * n_keys)
+        ref = polar.logits_prod(q[h:h + 1], D, S_or, enc["yhat"][sl], enc["signs"][sl], enc["norm_f16"][sl],
+                                enc["rnorm_f16"][sl], m)
+        tol = logit_tolerance(ref, enc["norm_f16"][sl], q[h:h + 1])
+        assert np.all(np.abs(got[h] - ref[0]) <= tol[0]), h

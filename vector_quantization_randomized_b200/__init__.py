@@ -70,6 +70,8 @@ _SIGS = {
     "tq_polar_quantize": (_i32, [_PP, _vp, _i32, _i64, _i64, _vp, _vp, _vp]),
     "tq_polar_dequantize": (_i32, [_PP, _vp, _vp, _i64, _vp, _i64, _vp]),
     "tq_polar_logits": (_i32, [_PP, _vp, _i32, _vp, _vp, _i64, _i32, _vp, _vp]),
+    "tq_polar_qjl": (_i32, [_PP, _vp, _i32, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "tq_polar_logits_prod": (_i32, [_PP, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _i64, _i32, _vp, _vp]),
     "tq_last_error": (ctypes.c_char_p, []),
     "tq_version": (_i32, []),
 }
@@ -338,3 +340,16 @@ def tq_polar_dequantize(p, codes, norms, n_vec, out, ld=None, stream=None):
 def tq_polar_logits(p, q, group, codes, norms, n_keys, n_kv_heads, logits, stream=None):
     return _check(_lib.tq_polar_logits(p.ref, _ptr(q), group, _ptr(codes), _ptr(norms), n_keys, n_kv_heads,
                                        _ptr(logits), _stream(stream)))
+
+
+def tq_polar_qjl(p, S, m, x, codes, signs, rnorms, n_vec=None, ld=None, stream=None):
+    """QJL stage on the polar residual: sign bits of S r (device uint8 [n_vec * m / 8]) and gamma (fp16)."""
+    n_vec = x.shape[0] if n_vec is None else n_vec
+    ld = x.stride(0) if ld is None else ld
+    return _check(_lib.tq_polar_qjl(p.ref, _ptr(S), m, _ptr(x), _dtype_code(x), n_vec, ld, _ptr(codes), _ptr(signs),
+                                    _ptr(rnorms), _stream(stream)))
+
+
+def tq_polar_logits_prod(p, S, m, q, group, codes, norms, signs, rnorms, n_keys, n_kv_heads, logits, stream=None):
+    return _check(_lib.tq_polar_logits_prod(p.ref, _ptr(S), m, _ptr(q), group, _ptr(codes), _ptr(norms), _ptr(signs),
+                                            _ptr(rnorms), n_keys, n_kv_heads, _ptr(logits), _stream(stream)))

@@ -383,6 +383,203 @@ __global__ void __launch_bounds__(128) polar_logits_kernel(const PArgs a) {
     if (g < a.group) a.logits[((int64_t)kv * a.group + g) * a.n_keys + key] = acc[g] * n;
 }
 
+// ---- QJL stage on the polar residual ---------------------------------------------
+// "TurboQuant explainer" (m.163.com), "第二步：QJL" applied to the polar stage 1:
+// r = y - y_hat (y the rotated unit vector, y_hat the unit-radius reconstruction
+// from the stored tables), gamma = ||r||, sign bits of S r.  A warp per vector:
+// the rotation as in the quantize kernel, y_hat as in the dequantize kernel, r
+// staged in shared memory, then lane l computes the projections l + 32 j in
+// fp64 (exact products of fp16 S and fp32 r) from S stored transposed in shared
+// memory, and a ballot per 32 projections packs the sign words.
+template <int DP, int W, int DT>
+__global__ void __launch_bounds__(256) polar_qjl_kernel(const PArgs a, const uint16_t* S, int m, uint32_t* signs,
+                                                        uint16_t* rnorms) {
+  using P = PL<DP, W>;
+  constexpr int NI = P::NI;
+  extern __shared__ __align__(16) uint8_t qsm[];
+  __half* St = reinterpret_cast<__half*>(qsm);                      // [DP][m]: St[k][i] = S[i][k]
+  float* rw = reinterpret_cast<float*>(qsm + (size_t)DP * m * 2);   // [8][DP] residual of each warp's vector
+  float* tab = rw + 8 * DP;                                         // the tables
+  uint32_t* rec = reinterpret_cast<uint32_t*>(tab + P::T1 + (P::LV - 1) * P::TL);  // [8][NW + 1]
+  for (int e = threadIdx.x; e < m * DP; e += blockDim.x) {
+    const int i = e / DP, k = e % DP;
+    St[k * m + i] = __ushort_as_half(__ldg(S + e));
+  }
+  for (int i = threadIdx.x; i < P::T1 + (P::LV - 1) * P::TL; i += blockDim.x) tab[i] = a.tables[i];
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  float dsg[NI];
+#pragma unroll
+  for (int k = 0; k < NI; ++k) dsg[k] = (float)a.D[NI * lane + k];
+  uint32_t* r = rec + wib * (P::NW + 1);
+  if (lane == 0) r[P::NW] = 0u;
+  float* rv = rw + wib * DP;
+  const float rs = rsqrtf((float)DP);
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t v = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib; v < a.n_vec; v += warps) {
+    // ---- y: rotation of the unit vector (as polar_quantize_kernel)
+    const uint8_t* row = a.x + v * a.ld * (DT == TQ_F32 ? 4 : 2);
+    float y[NI];
+    float ss = 0.f;
+#pragma unroll
+    for (int g4 = 0; g4 < NI / 4; ++g4) {
+      const int j = NI * lane + 4 * g4;
+      float e[4] = {0.f, 0.f, 0.f, 0.f};
+      if (j < a.d) {
+        if constexpr (DT == TQ_F32) {
+          const float4 f = __ldg(reinterpret_cast<const float4*>(row) + (j >> 2));
+          e[0] = f.x, e[1] = f.y, e[2] = f.z, e[3] = f.w;
+        } else {
+          const uint2 u = __ldg(reinterpret_cast<const uint2*>(row) + (j >> 2));
+          const uint32_t wd[2] = {u.x, u.y};
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if constexpr (DT == TQ_BF16) {
+              e[2 * h] = __uint_as_float(wd[h] << 16);
+              e[2 * h + 1] = __uint_as_float(wd[h] & 0xFFFF0000u);
+            } else {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wd[h]));
+              e[2 * h] = f.x, e[2 * h + 1] = f.y;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        y[4 * g4 + k] = e[k] * dsg[4 * g4 + k];
+        ss = fmaf(y[4 * g4 + k], y[4 * g4 + k], ss);
+      }
+    }
+    ss = warp_sum(ss);
+    const float n = sqrtf(ss);
+#pragma unroll
+    for (int hs = 1; hs < NI; hs <<= 1)
+#pragma unroll
+      for (int k = 0; k < NI; ++k)
+        if ((k & hs) == 0) {
+          const float u = y[k], w = y[k + hs];
+          y[k] = u + w;
+          y[k + hs] = u - w;
+        }
+#pragma unroll
+    for (int sft = 1; sft < 32; sft <<= 1)
+#pragma unroll
+      for (int k = 0; k < NI; ++k) {
+        const float o = __shfl_xor_sync(FULL, y[k], sft);
+        y[k] = (lane & sft) ? (o - y[k]) : (y[k] + o);
+      }
+    const float sc = n > 0.f ? rs / n : 0.f;
+    // ---- y_hat from the record (as polar_dequantize_kernel, without the inverse rotation)
+    if (lane < P::NW) r[lane] = __ldg(reinterpret_cast<const uint32_t*>(a.ccodes + v * (P::NW * 4)) + lane);
+    __syncwarp();
+    auto get = [&](int p, int width) {
+      const uint64_t w64 = (uint64_t)r[p >> 5] | ((uint64_t)r[(p >> 5) + 1] << 32);
+      return (int)((w64 >> (p & 31)) & ((1u << width) - 1u));
+    };
+    auto cs = [&](int l, int ix) {
+      const float* t = tab + P::T1 + (l - 2) * P::TL + 2 * P::L2 - 1;
+      return make_float2(t[2 * ix], t[2 * ix + 1]);
+    };
+    float R = 1.f;
+#pragma unroll
+    for (int l = P::LV; l > P::LI; --l) {
+      const int ix = P::B2 > 0 ? get(P::pos(l, lane >> (l - P::LI)), P::B2) : 0;
+      const float2 c = cs(l, ix);
+      R *= ((lane >> (l - P::LI - 1)) & 1) ? c.y : c.x;
+    }
+    float rad[NI / 2];
+    rad[0] = R;
+#pragma unroll
+    for (int l = P::LI; l >= 2; --l) {
+      const int cnt = NI >> l;
+#pragma unroll
+      for (int j = cnt - 1; j >= 0; --j) {
+        const int ix = P::B2 > 0 ? get(P::pos(l, cnt * lane + j), P::B2) : 0;
+        const float2 c = cs(l, ix);
+        const float pr = rad[j];
+        rad[2 * j] = pr * c.x;
+        rad[2 * j + 1] = pr * c.y;
+      }
+    }
+    float g2 = 0.f;
+#pragma unroll
+    for (int j = 0; j < NI / 2; ++j) {
+      const int ix = get(P::pos(1, (NI / 2) * lane + j), P::B1);
+      const float r0 = y[2 * j] * sc - rad[j] * tab[P::L1 + 2 * ix];
+      const float r1 = y[2 * j + 1] * sc - rad[j] * tab[P::L1 + 2 * ix + 1];
+      rv[NI * lane + 2 * j] = r0;
+      rv[NI * lane + 2 * j + 1] = r1;
+      g2 = fmaf(r0, r0, fmaf(r1, r1, g2));
+    }
+    g2 = warp_sum(g2);
+    __syncwarp();
+    // ---- z = S r in fp64, a ballot per 32 projections
+    for (int jw = 0; jw < m / 32; ++jw) {
+      const int i = 32 * jw + lane;
+      double acc = 0.0;
+#pragma unroll 8
+      for (int k = 0; k < DP; ++k) acc = fma((double)__half2float(St[k * m + i]), (double)rv[k], acc);
+      const uint32_t word = __ballot_sync(FULL, acc >= 0.0);
+      if (lane == 0) signs[v * (m / 32) + jw] = word;
+    }
+    if (lane == 0) rnorms[v] = __half_as_ushort(__float2half_rn(sqrtf(g2)));
+    __syncwarp();
+  }
+}
+
+// QJL term of the polar product-code logits, added to the stage-1 logits:
+// l += n gamma sqrt(pi/2)/m <S q~, 2 s - 1>.  A CTA of 128 threads takes 128
+// keys of one KV head: it rotates the group's queries and projects them
+// (u = S q~) into shared memory, then each thread walks its key's sign bits.
+template <int DP>
+__global__ void __launch_bounds__(128) polar_qjl_logits_kernel(const PArgs a, const uint16_t* S, int m,
+                                                               const uint32_t* signs, const uint16_t* rnorms,
+                                                               float kappa) {
+  __shared__ float qt[8][DP];
+  __shared__ float u[8][DP];
+  const int kv = blockIdx.y;
+  const int tid = threadIdx.x;
+  // q~ = H D q / sqrt(DP): butterflies in shared memory
+  for (int e = tid; e < a.group * DP; e += blockDim.x) {
+    const int g = e / DP, c = e % DP;
+    qt[g][c] = c < a.d ? a.q[((int64_t)kv * a.group + g) * a.d + c] * (float)a.D[c] : 0.f;
+  }
+  __syncthreads();
+  for (int hs = 1; hs < DP; hs <<= 1) {
+    for (int e = tid; e < a.group * DP / 2; e += blockDim.x) {
+      const int g = e / (DP / 2), p = e % (DP / 2);
+      const int lo = (p / hs) * 2 * hs + (p % hs), hi = lo + hs;
+      const float x0 = qt[g][lo], x1 = qt[g][hi];
+      qt[g][lo] = x0 + x1;
+      qt[g][hi] = x0 - x1;
+    }
+    __syncthreads();
+  }
+  const float rs = rsqrtf((float)DP);
+  for (int e = tid; e < a.group * m; e += blockDim.x) {
+    const int g = e / m, i = e % m;
+    float acc = 0.f;
+    const uint16_t* srow = S + (size_t)i * DP;
+    for (int k = 0; k < DP; ++k) acc = fmaf(__half2float(__ushort_as_half(__ldg(srow + k))), qt[g][k], acc);
+    u[g][i] = acc * rs;
+  }
+  __syncthreads();
+  const int64_t key = (int64_t)blockIdx.x * blockDim.x + tid;
+  if (key >= a.n_keys) return;
+  const int64_t vi = (int64_t)kv * a.n_keys + key;
+  const float n = __half2float(__ushort_as_half(__ldg(a.cnorms + vi)));
+  const float gm = __half2float(__ushort_as_half(__ldg(rnorms + vi)));
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int w = 0; w < m / 32; ++w) {
+    const uint32_t word = __ldg(signs + vi * (m / 32) + w);
+    for (int b = 0; b < 32; ++b) {
+      const bool pos = (word >> b) & 1u;
+      for (int g = 0; g < a.group; ++g) acc[g] += pos ? u[g][32 * w + b] : -u[g][32 * w + b];
+    }
+  }
+  for (int g = 0; g < a.group; ++g) a.logits[((int64_t)kv * a.group + g) * a.n_keys + key] += n * gm * kappa * acc[g];
+}
+
 int launch_err(const char* who) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "%s: launch failed: %s", who, cudaGetErrorString(e));
@@ -432,6 +629,19 @@ int logits_dw(const PArgs& a, int n_kv, cudaStream_t st) {
   else
     polar_logits_kernel<DP, W, 8><<<grid, 128, 0, st>>>(a);
   return launch_err("tq_polar_logits");
+}
+
+template <int DP, int W>
+int qjl_dw(int dtype, const PArgs& a, const uint16_t* S, int m, uint32_t* signs, uint16_t* rnorms, cudaStream_t st) {
+  using P = PL<DP, W>;
+  const size_t smem = (size_t)DP * m * 2 + 8 * DP * 4 + (P::T1 + (P::LV - 1) * P::TL) * 4 + 8 * (P::NW + 1) * 4;
+  void (*kern)(const PArgs, const uint16_t*, int, uint32_t*, uint16_t*) =
+      dtype == TQ_F32 ? polar_qjl_kernel<DP, W, TQ_F32>
+                      : (dtype == TQ_F16 ? polar_qjl_kernel<DP, W, TQ_F16> : polar_qjl_kernel<DP, W, TQ_BF16>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_polar_qjl: %s", cudaGetErrorString(e));
+  kern<<<grid_for(a.n_vec), 256, smem, st>>>(a, S, m, signs, rnorms);
+  return launch_err("tq_polar_qjl");
 }
 
 #define TQ_POLAR_DISPATCH(dp, w, CALL) \
@@ -534,6 +744,76 @@ extern "C" int tq_polar_logits(const tq_polar_params* p, const float* q, int gro
 #define L_CALL(DP, W) logits_dw<DP, W>(a, n_kv_heads, st)
   rc = TQ_POLAR_DISPATCH(p->d_pad, p->w, L_CALL);
 #undef L_CALL
+  if (rc == TQ_OK) clear_error();
+  return rc;
+}
+
+extern "C" int tq_polar_qjl(const tq_polar_params* p, const uint16_t* S, int m, const void* x, int dtype,
+                            int64_t n_vec, int64_t ld, const void* codes, void* signs, uint16_t* rnorms,
+                            tq_stream_t stream) {
+  using namespace tq;
+  int rc = check_polar(p, "tq_polar_qjl");
+  if (rc) return rc;
+  if (m < 32 || m > p->d_pad || m % 32 != 0)
+    return set_error(TQ_EINVAL, "tq_polar_qjl: m must be a multiple of 32 in [32, d_pad]");
+  if (n_vec < 0) return set_error(TQ_EINVAL, "tq_polar_qjl: n_vec < 0");
+  if (n_vec == 0) {
+    clear_error();
+    return TQ_OK;
+  }
+  if (dtype != TQ_F32 && dtype != TQ_F16 && dtype != TQ_BF16) return set_error(TQ_EINVAL, "tq_polar_qjl: dtype");
+  if (!S || !x || !codes || !signs || !rnorms) return set_error(TQ_EINVAL, "tq_polar_qjl: NULL pointer argument");
+  if (ld < p->d) return set_error(TQ_EINVAL, "tq_polar_qjl: ld < d");
+  const int es = dtype == TQ_F32 ? 4 : 2;
+  if (!aligned(x, 16) || ((ld * es) % 16) != 0 || ((int64_t)p->d * es) % 16 != 0 || !aligned(codes, 16) ||
+      !aligned(signs, 4) || !aligned(rnorms, 2))
+    return set_error(TQ_EINVAL, "tq_polar_qjl: x, ld*elem, d*elem and codes must be 16-byte aligned, signs 4-byte");
+  PArgs a{};
+  a.x = static_cast<const uint8_t*>(x);
+  a.n_vec = n_vec;
+  a.ld = ld;
+  a.d = p->d;
+  a.tables = p->tables;
+  a.D = p->signs_D;
+  a.ccodes = static_cast<const uint8_t*>(codes);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* sg = static_cast<uint32_t*>(signs);
+#define J_CALL(DP, W) qjl_dw<DP, W>(dtype, a, S, m, sg, rnorms, st)
+  rc = TQ_POLAR_DISPATCH(p->d_pad, p->w, J_CALL);
+#undef J_CALL
+  if (rc == TQ_OK) clear_error();
+  return rc;
+}
+
+extern "C" int tq_polar_logits_prod(const tq_polar_params* p, const uint16_t* S, int m, const float* q, int group,
+                                    const void* codes, const uint16_t* norms, const void* signs,
+                                    const uint16_t* rnorms, int64_t n_keys, int n_kv_heads, float* logits,
+                                    tq_stream_t stream) {
+  using namespace tq;
+  if (!p) return set_error(TQ_EINVAL, "tq_polar_logits_prod: NULL params");
+  if (m < 32 || m > p->d_pad || m % 32 != 0)
+    return set_error(TQ_EINVAL, "tq_polar_logits_prod: m must be a multiple of 32 in [32, d_pad]");
+  if (!S || !signs || !rnorms) return set_error(TQ_EINVAL, "tq_polar_logits_prod: NULL pointer argument");
+  if (!aligned(signs, 4)) return set_error(TQ_EINVAL, "tq_polar_logits_prod: signs must be 4-byte aligned");
+  int rc = tq_polar_logits(p, q, group, codes, norms, n_keys, n_kv_heads, logits, stream);
+  if (rc) return rc;
+  if (n_keys == 0 || n_kv_heads == 0) return TQ_OK;
+  PArgs a{};
+  a.d = p->d;
+  a.D = p->signs_D;
+  a.cnorms = norms;
+  a.q = q;
+  a.logits = logits;
+  a.n_keys = n_keys;
+  a.group = group;
+  const float kappa = (float)(std::sqrt(M_PI / 2.0) / m);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid((unsigned)((n_keys + 127) / 128), (unsigned)n_kv_heads);
+  if (p->d_pad == 128)
+    polar_qjl_logits_kernel<128><<<grid, 128, 0, st>>>(a, S, m, static_cast<const uint32_t*>(signs), rnorms, kappa);
+  else
+    polar_qjl_logits_kernel<256><<<grid, 128, 0, st>>>(a, S, m, static_cast<const uint32_t*>(signs), rnorms, kappa);
+  rc = launch_err("tq_polar_logits_prod");
   if (rc == TQ_OK) clear_error();
   return rc;
 }
