@@ -98,8 +98,8 @@ struct TL {
   static constexpr int W_EXP0 = 5, W_EPI0 = 13;
   static constexpr int NTHREADS = 21 * 32;
   static constexpr int OFF_IMG = 1024;
-  static constexpr int OFF_PREP = OFF_IMG + 2 * IMG;      // q_rot float4[128], u float4[128], partial u [2][128]
-  static constexpr int OFF_RING = OFF_PREP + 4 * 128 * 16;
+  static constexpr int OFF_PREP = OFF_IMG + 2 * IMG;  // q_rot [2][128], u [2][128], partial u [2][2][128] (float4)
+  static constexpr int OFF_RING = OFF_PREP + 8 * 128 * 16;
   static constexpr int smem(int stages) { return OFF_RING + stages * STAGE; }
 };
 
@@ -116,26 +116,49 @@ __device__ __forceinline__ float pow2(int k) {
   return (k >= -126 && k <= 127) ? __uint_as_float((uint32_t)(127 + k) << 23) : ldexpf(1.f, k);
 }
 
-// B image of KV head `head` into `img`, by the 256 threads of warps 13-20
-// (et = 0..255).  Steps: q_rot = H D q / sqrt(128) (warp per query);
-// u = S q_rot (thread = row of S x half of the coordinates); per-query scales
-// 2^F, 2^G putting the largest weight just below 2^23; digits into the image.
+// Global loads of the query preparation, issued early so their latency overlaps
+// other work: warp ew's query (image ew / 4, query ew % 4), times the sign flips,
+// and thread et's half row of S (row et % 128, coordinates 64 (et / 128) ..).
+struct PrepRegs {
+  float y[4];
+  uint4 sv[8];
+};
+
+template <int SI>
+__device__ __forceinline__ void prep_load(const TArgs& a, int64_t head0, int n_img, int et, PrepRegs& pr) {
+  const int ew = et >> 5, lane = et & 31;
+  const int k = ew >> 2, j = ew & 3;
+  const bool valid = k < n_img && j < a.group;
+  const int64_t row = (head0 + k) * a.group + j;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = 32 * i + lane;
+    pr.y[i] = (valid && c < a.d) ? __ldg(a.q + row * a.d + c) * (float)__ldg(a.D + c) : 0.f;
+  }
+  if constexpr (SI) {
+    const int r = et & 127, h = et >> 7;
+    const uint4* srow = reinterpret_cast<const uint4*>(a.S + (size_t)r * DP) + 8 * h;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) pr.sv[kk] = r < a.m ? __ldg(srow + kk) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// B images of n_img (1 or 2) consecutive KV heads into img0 / img1, by the 256
+// threads of warps 13-20 (et = 0..255) from the loads in pr.  Steps:
+// q_rot = H D q / sqrt(128) (warp per query: image ew / 4, query ew % 4);
+// u = S q_rot (thread = row of S x half of the coordinates, both images);
+// per-query scales 2^F, 2^G putting the largest weight just below 2^23; digits.
 template <int KB, int SI>
-__device__ void make_image(const TArgs& a, int64_t head, uint8_t* img, float4* qT, float4* uT, float4* up,
-                           const float* alpha, float* red, int et, GroupSync& gs) {
+__device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* img0, uint8_t* img1, float4* qT,
+                            float4* uT, float4* up, const float* alpha, float* red, int et, GroupSync& gs) {
   using L = TL<KB, SI>;
   const int ew = et >> 5, lane = et & 31;
-  float* qTf = reinterpret_cast<float*>(qT);
-  float* uTf = reinterpret_cast<float*>(uT);
-  if (ew < 4) {  // warp = query ew; lane holds coordinates lane + 32 i
-    const bool valid = ew < a.group;
-    const int64_t row = head * a.group + ew;
-    float y[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j = 32 * i + lane;
-      y[i] = (valid && j < a.d) ? __ldg(a.q + row * a.d + j) * (float)__ldg(a.D + j) : 0.f;
-    }
+  const int kq = ew >> 2, jq = ew & 3;  // this warp's image and query
+  float* qTf = reinterpret_cast<float*>(qT);  // [2][128][4]
+  float* uTf = reinterpret_cast<float*>(uT);  // [2][128][4]
+  float* rd = red + 16 * kq;                  // per query of image kq: sum, max, 2^F, 2^G
+  {
+    float* y = pr.y;
 #pragma unroll
     for (int h = 1; h < 4; h <<= 1)
 #pragma unroll
@@ -156,58 +179,55 @@ __device__ void make_image(const TArgs& a, int64_t head, uint8_t* img, float4* q
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float v = y[i] * 0.08838834764831845f;  // 1/sqrt(128)
-      qTf[4 * (32 * i + lane) + ew] = v;
+      qTf[512 * kq + 4 * (32 * i + lane) + jq] = v;
       sum += v;
       mx = fmaxf(mx, fabsf(v));
     }
     sum = warp_sum(sum);
     mx = warp_max(mx);
     if (lane == 0) {
-      red[4 * ew] = sum;
-      red[4 * ew + 1] = mx;
+      rd[4 * jq] = sum;
+      rd[4 * jq + 1] = mx;
     }
   }
   gs.sync(lane);
   if constexpr (SI) {  // u = S q_rot: row i = et % 128, coordinates 64h .. 64h + 63 (h = et / 128)
     const int i = et & 127, h = et >> 7;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), acc2 = acc;
-    if (i < a.m) {
-      const uint4* srow = reinterpret_cast<const uint4*>(a.S + (size_t)i * DP) + 8 * h;
-      uint4 sv[8];
+    float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
 #pragma unroll
-      for (int k = 0; k < 8; ++k) sv[k] = __ldg(srow + k);
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t wv[4] = {pr.sv[k].x, pr.sv[k].y, pr.sv[k].z, pr.sv[k].w};
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t wv[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w};
+      for (int h2 = 0; h2 < 4; ++h2) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[h2]));
+        const int j = 64 * h + 8 * k + 2 * h2;
 #pragma unroll
-        for (int h2 = 0; h2 < 4; ++h2) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[h2]));
-          const int j = 64 * h + 8 * k + 2 * h2;
-          const float4 q0 = qT[j], q1 = qT[j + 1];
-          acc.x = fmaf(f.x, q0.x, acc.x);
-          acc.y = fmaf(f.x, q0.y, acc.y);
-          acc.z = fmaf(f.x, q0.z, acc.z);
-          acc.w = fmaf(f.x, q0.w, acc.w);
-          acc2.x = fmaf(f.y, q1.x, acc2.x);
-          acc2.y = fmaf(f.y, q1.y, acc2.y);
-          acc2.z = fmaf(f.y, q1.z, acc2.z);
-          acc2.w = fmaf(f.y, q1.w, acc2.w);
+        for (int im = 0; im < 2; ++im) {
+          if (im < n_img) {
+            const float4 q0 = qT[128 * im + j], q1 = qT[128 * im + j + 1];
+            acc[im].x = fmaf(f.y, q1.x, fmaf(f.x, q0.x, acc[im].x));
+            acc[im].y = fmaf(f.y, q1.y, fmaf(f.x, q0.y, acc[im].y));
+            acc[im].z = fmaf(f.y, q1.z, fmaf(f.x, q0.z, acc[im].z));
+            acc[im].w = fmaf(f.y, q1.w, fmaf(f.x, q0.w, acc[im].w));
+          }
         }
       }
     }
-    up[128 * h + i] = make_float4(acc.x + acc2.x, acc.y + acc2.y, acc.z + acc2.z, acc.w + acc2.w);
+#pragma unroll
+    for (int im = 0; im < 2; ++im) up[256 * im + 128 * h + i] = acc[im];
     gs.sync(lane);
-    if (et < 128) {
-      const float4 p0 = up[et], p1 = up[128 + et];
-      uT[et] = make_float4(p0.x + p1.x, p0.y + p1.y, p0.z + p1.z, p0.w + p1.w);
+    {
+      const int im = et >> 7, r = et & 127;  // thread = (image, row)
+      const float4 p0 = up[256 * im + r], p1 = up[256 * im + 128 + r];
+      uT[128 * im + r] = make_float4(p0.x + p1.x, p0.y + p1.y, p0.z + p1.z, p0.w + p1.w);
     }
     gs.sync(lane);
   }
-  if (ew < 4) {  // scales and per-query scalars: warp = query ew
+  if (kq < n_img) {  // scales and per-query scalars: warp = (image kq, query jq)
     float su = 0.f, mu = 0.f;
     if constexpr (SI) {
       for (int i = lane; i < a.m; i += 32) {
-        const float v = uTf[4 * i + ew];
+        const float v = uTf[512 * kq + 4 * i + jq];
         su += v;
         mu = fmaxf(mu, fabsf(v));
       }
@@ -217,27 +237,30 @@ __device__ void make_image(const TArgs& a, int64_t head, uint8_t* img, float4* q
     float amax = 0.f;
 #pragma unroll
     for (int T = 0; T < L::NT; ++T) amax = fmaxf(amax, fabsf(alpha[T]));
-    const float mc = 2.f * amax * red[4 * ew + 1], ms = 2.f * mu;
+    const float mc = 2.f * amax * rd[4 * jq + 1], ms = 2.f * mu;
     const int F = mc > 0.f ? 23 - exponent_of(mc) : 0;
     const int G = ms > 0.f ? 23 - exponent_of(ms) : 0;
     if (lane == 0) {
-      red[4 * ew + 2] = pow2(F);
-      red[4 * ew + 3] = pow2(G);
+      rd[4 * jq + 2] = pow2(F);
+      rd[4 * jq + 3] = pow2(G);
       // sum_T alpha_T = c[L-1] (all index bits set)
-      reinterpret_cast<float4*>(img)[ew] =
-          make_float4(pow2(-(F + 7)), alpha[4] * red[4 * ew], pow2(-(G + 7)), su);
+      reinterpret_cast<float4*>(kq ? img1 : img0)[jq] =
+          make_float4(pow2(-(F + 7)), alpha[4] * rd[4 * jq], pow2(-(G + 7)), su);
     }
   }
   gs.sync(lane);
-  // Digit words, one thread per (query q, plane P, bit class c, word w): the weights of
-  // coordinates 32w + 8b + c (b = 0..3) give word w of K chunk c of plane P in the 4
-  // digit rows 4q + d.  Scaling by 2^F (2^G) is exact.
-  for (int e = et; e < 4 * L::NP * 32; e += 256) {
-    const int w = e & 3, c = (e >> 2) & 7, pq = e >> 5;
+  // Digit words, one thread per (image, query q, plane P, bit class c, word w): the
+  // weights of coordinates 32w + 8b + c (b = 0..3) give word w of K chunk c of plane P
+  // in the 4 digit rows 4q + d.  Scaling by 2^F (2^G) is exact.
+  constexpr int PER = 4 * L::NP * 32;
+  for (int e = et; e < n_img * PER; e += 256) {
+    const int im = e / PER, e2 = e - im * PER;
+    const int w = e2 & 3, c = (e2 >> 2) & 7, pq = e2 >> 5;
     const int q = pq / L::NP, P = pq - q * L::NP;
     const bool cen = P < L::NT;
-    const float scale = cen ? 2.f * alpha[P] * red[4 * q + 2] : 2.f * red[4 * q + 3];
-    const float* src = cen ? qTf : uTf;
+    const float* r2 = red + 16 * im;
+    const float scale = cen ? 2.f * alpha[P] * r2[4 * q + 2] : 2.f * r2[4 * q + 3];
+    const float* src = (cen ? qTf : uTf) + 512 * im;
     uint32_t W[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
@@ -252,11 +275,11 @@ __device__ void make_image(const TArgs& a, int64_t head, uint8_t* img, float4* q
       W[3] |= (uint32_t)(uint8_t)X << (8 * b);
     }
     const int kc = cen ? 8 * P + c : c;
-    uint8_t* base = img + (cen ? L::IMG_C : L::IMG_S) + kc * 256 + (q >> 1) * 128 + 4 * w;
+    uint8_t* base = (im ? img1 : img0) + (cen ? L::IMG_C : L::IMG_S) + kc * 256 + (q >> 1) * 128 + 4 * w;
 #pragma unroll
     for (int dd = 0; dd < 4; ++dd) *reinterpret_cast<uint32_t*>(base + (4 * (q & 1) + dd) * 16) = W[dd];
   }
-  fence_async_smem();  // the image is read by the tensor core (async proxy)
+  fence_async_smem();  // the images are read by the tensor core (async proxy)
   gs.sync(lane);
 }
 
@@ -276,11 +299,11 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
   uint64_t* gbar = imgfree + 2;                        // barrier of the 8 prep / epilogue warps (8)
   uint32_t* tbase = reinterpret_cast<uint32_t*>(gbar + 1);
   float* alpha = reinterpret_cast<float*>(tbase + 4);  // [5] Walsh coefficients, then c[L-1]
-  float* red = alpha + 8;                              // [16] per query: sum, max, 2^F, 2^G
+  float* red = alpha + 8;                              // [2][16] per image and query: sum, max, 2^F, 2^G
   uint8_t* imgs = smem + L::OFF_IMG;
   float4* qT = reinterpret_cast<float4*>(smem + L::OFF_PREP);
-  float4* uT = qT + 128;
-  float4* up = uT + 128;
+  float4* uT = qT + 256;
+  float4* up = uT + 256;
   uint8_t* ring = smem + L::OFF_RING;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -294,21 +317,26 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
   if (threadIdx.x == 0) {
     for (int s = 0; s < MAX_STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 16);
+      mbar_init(&empty[s], 8);  // the 4 expansion and 4 epilogue warps of the item's parity
     }
     for (int b = 0; b < 3; ++b) {
-      mbar_init(&afull[b], 8);
+      mbar_init(&afull[b], 4);
       mbar_init(&mdone[b], 2);
     }
     for (int c = 0; c < 4; ++c) {
       mbar_init(&cfull[c], 2);
-      mbar_init(&accfree[c], 8);
+      mbar_init(&accfree[c], 4);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&imgfull[k], 1);
       mbar_init(&imgfree[k], 4);
     }
     mbar_init(gbar, 8);
+  }
+  PrepRegs pr;
+  if (warp >= W_EPI0) {  // the first one or two heads' query loads overlap the set-up
+    grid_dependency_wait();  // queries may come from the preceding kernel in the stream
+    prep_load<SI>(a, h_first, n_img < 2 ? n_img : 2, threadIdx.x - 32 * W_EPI0, pr);
   }
   if (warp == 0) tmem_alloc(tbase, 512);
   tc_fence_before();
@@ -386,10 +414,12 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
     __syncwarp();
   } else if (warp < W_EPI0) {
     // ---------------- expansion: code bits -> A in tensor memory ----------------
+    // warps 5-8 take the even items, 9-12 the odd ones; each covers one lane quadrant
+    // (a 32-key tile of the item) and all 8 bit classes of every plane
     const int ew = warp - W_EXP0;
-    const int qd = warp & 3;  // tensor-memory lane quadrant = 32-key code tile within the item
-    const int cg = ew >> 2;   // bit classes 4cg .. 4cg+3
-    for (int i = 0, s = 0, use = 0; i < n; ++i, (++s == S ? (s = 0, ++use) : 0)) {
+    const int qd = warp & 3, par = ew >> 2;
+    for (int i = par; i < n; i += 2) {
+      const int s = i % S, use = i / S;
       const int b = i % L::NA, ua = i / L::NA;
       if (!mbar_wait(&full[s], use & 1)) break;
       if (ua >= 1 && !mbar_wait(&mdone[b], (ua - 1) & 1)) break;  // MMAs of item i - NA have read A[b]
@@ -406,19 +436,22 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
         it[3] = make_uint4(pw[0].x ^ pw[1].x ^ pw[2].x, pw[0].y ^ pw[1].y ^ pw[2].y, pw[0].z ^ pw[1].z ^ pw[2].z,
                            pw[0].w ^ pw[1].w ^ pw[2].w);
       if constexpr (SI) it[L::NT] = pw[KB];
-      const uint32_t lanebase = a_col(b) + ((uint32_t)(32 * qd) << 16) + 16 * cg;
+      const uint32_t lanebase = a_col(b) + ((uint32_t)(32 * qd) << 16);
 #pragma unroll
       for (int P = 0; P < L::NP; ++P) {
-        uint32_t r[16];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const uint32_t mk = 0x01010101u << (4 * cg + cc);
-          r[4 * cc + 0] = it[P].x & mk;
-          r[4 * cc + 1] = it[P].y & mk;
-          r[4 * cc + 2] = it[P].z & mk;
-          r[4 * cc + 3] = it[P].w & mk;
+        for (int cg = 0; cg < 2; ++cg) {
+          uint32_t r[16];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const uint32_t mk = 0x01010101u << (4 * cg + cc);
+            r[4 * cc + 0] = it[P].x & mk;
+            r[4 * cc + 1] = it[P].y & mk;
+            r[4 * cc + 2] = it[P].z & mk;
+            r[4 * cc + 3] = it[P].w & mk;
+          }
+          tmem_st16(lanebase + 32 * P + 16 * cg, r);
         }
-        tmem_st16(lanebase + 32 * P, r);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -427,47 +460,49 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
     }
   } else {
     // ---------------- query preparation, then the epilogue ----------------
+    // warps 13-16 take the even items, 17-20 the odd ones; each covers one lane quadrant
+    // (32 keys) and all the query heads of the KV head
     const int et = threadIdx.x - 32 * W_EPI0;
     const int ew = warp - W_EPI0;
-    const int qd = warp & 3, qp = ew >> 2;  // keys 32qd + lane; queries 2qp, 2qp+1
-    grid_dependency_wait();                // queries may come from the preceding kernel in the stream
-    if (et < L::NT + 1) {                  // Walsh coefficients of the odd-symmetric codebook (fp64), c[L-1]
+    const int qd = warp & 3, par = ew >> 2;
+    if (et < L::NT + 1) {  // Walsh coefficients of the odd-symmetric codebook (fp64), c[L-1]
       const int Lv = 1 << KB;
-      double s = 0.0;
+      double sacc = 0.0;
       if (et < L::NT) {
         const int mask = walsh_mask(KB, et);
-        for (int l = 0; l < Lv; ++l) s += (double)__ldg(a.cent + l) * ((__popc(l & mask) & 1) ? 1.0 : -1.0);
-        alpha[et] = (float)(s / Lv);
+        for (int l = 0; l < Lv; ++l) sacc += (double)__ldg(a.cent + l) * ((__popc(l & mask) & 1) ? 1.0 : -1.0);
+        alpha[et] = (float)(sacc / Lv);
       } else {
         alpha[4] = __ldg(a.cent + Lv - 1);
       }
     }
     GroupSync gs{gbar, 0u};
     gs.sync(lane);
-    for (int k = 0; k < n_img && k < 2; ++k) {
-      make_image<KB, SI>(a, h_first + k, imgs + k * L::IMG, qT, uT, up, alpha, red, et, gs);
-      if (et == 0) mbar_arrive(&imgfull[k]);
+    if (n_img > 0) {
+      make_images<KB, SI>(a, pr, n_img < 2 ? n_img : 2, imgs, imgs + L::IMG, qT, uT, up, alpha, red, et, gs);
+      if (et == 0) {
+        mbar_arrive(&imgfull[0]);
+        if (n_img > 1) mbar_arrive(&imgfull[1]);
+      }
     }
     int64_t head = h_first;
     int t = (int)(i0 % a.tiles_per_head);
     int kimg = 0;
-    float4 sc[2] = {};
-    bool fresh = true;
-    for (int i = 0, s = 0, use = 0, c = 0, cu = 0; i < n;
-         ++i, ++t, (++s == S ? (s = 0, ++use) : 0), (++c == L::NB ? (c = 0, ++cu) : 0)) {
-      if (t == a.tiles_per_head) t = 0, ++head, ++kimg, fresh = true;
-      if (fresh) {
-        fresh = false;
-        const float4* qs = reinterpret_cast<const float4*>(imgs + (kimg & 1) * L::IMG);
-        sc[0] = qs[2 * qp];
-        sc[1] = qs[2 * qp + 1];
+    for (int i = 0; i < n; ++i, ++t) {
+      if (t == a.tiles_per_head) {
+        t = 0, ++head, ++kimg;
         const int kn = kimg + 1;  // the next head's image, into the slot image kimg - 1 used
         if (kn >= 2 && kn < n_img) {
           mbar_wait(&imgfree[kn & 1], ((kn - 2) >> 1) & 1);  // on a time-out the fault word is set; go on
-          make_image<KB, SI>(a, head + 1, imgs + (kn & 1) * L::IMG, qT, uT, up, alpha, red, et, gs);
+          PrepRegs pr2;
+          prep_load<SI>(a, head + 1, 1, et, pr2);
+          uint8_t* slot = imgs + (kn & 1) * L::IMG;
+          make_images<KB, SI>(a, pr2, 1, slot, slot, qT, uT, up, alpha, red, et, gs);
           if (et == 0) mbar_arrive(&imgfull[kn & 1]);
         }
       }
+      if ((i & 1) != par) continue;
+      const int s = i % S, use = i / S, c = i % L::NB, cu = i / L::NB;
       const int64_t key = (int64_t)t * TK + 32 * qd + lane;
       const bool kvalid = key < a.n_keys;
       if (!mbar_wait(&full[s], use & 1)) break;  // long complete: makes the stage's norms visible here
@@ -478,39 +513,42 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       if (lane == 0) mbar_arrive(&empty[s]);
       if (!mbar_wait(&cfull[c], cu & 1)) break;
       tc_fence_after();
-      uint32_t c0[8], c1[8], s0[8], s1[8];
-      const uint32_t lrow = acc_col(c) + ((uint32_t)(32 * qd) << 16) + 8 * qp;
-      tmem_ld8_issue(lrow, c0);
-      tmem_ld8_issue(lrow + 32, c1);
-      if constexpr (SI) {
-        tmem_ld8_issue(lrow + 16, s0);
-        tmem_ld8_issue(lrow + 48, s1);
-      } else {
+      const uint32_t lrow = acc_col(c) + ((uint32_t)(32 * qd) << 16);
+      uint32_t C[16], Z[16];  // 4 queries x 4 digits, centroid and sign sums
+      {
+        uint32_t c1[16];
+        tmem_ld16_issue(lrow, C);
+        tmem_ld16_issue(lrow + 32, c1);
+        tmem_ld_wait16x2(C, c1);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s0[e] = s1[e] = 0u;
+        for (int e = 0; e < 16; ++e) C[e] += c1[e];  // exact: the full sums stay below 2^24
       }
-      tmem_ld_wait8x4(c0, c1, s0, s1);
+      if constexpr (SI) {
+        uint32_t s1[16];
+        tmem_ld16_issue(lrow + 16, Z);
+        tmem_ld16_issue(lrow + 48, s1);
+        tmem_ld_wait16x2(Z, s1);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) Z[e] += s1[e];
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&accfree[c]);
+      const float4* qs = reinterpret_cast<const float4*>(imgs + (kimg & 1) * L::IMG);
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        const int qi = 2 * qp + jj;
+      for (int qi = 0; qi < 4; ++qi) {
         if (qi < a.group && kvalid) {
+          const float4 sc = qs[qi];
           // sum_d 256^d C[d]: each C[d] an exact int32 below 2^24; one fp32 rounding per step
-          int C[4], Z[4];
-#pragma unroll
-          for (int dd = 0; dd < 4; ++dd) {
-            C[dd] = (int)(c0[4 * jj + dd] + c1[4 * jj + dd]);
-            Z[dd] = (int)(s0[4 * jj + dd] + s1[4 * jj + dd]);
-          }
-          const float cen =
-              fmaf((float)C[3], 16777216.f, fmaf((float)C[2], 65536.f, fmaf((float)C[1], 256.f, (float)C[0])));
-          float l = fmaf(cen, sc[jj].x, -sc[jj].y);
+          const float cen = fmaf((float)(int)C[4 * qi + 3], 16777216.f,
+                                 fmaf((float)(int)C[4 * qi + 2], 65536.f,
+                                      fmaf((float)(int)C[4 * qi + 1], 256.f, (float)(int)C[4 * qi])));
+          float l = fmaf(cen, sc.x, -sc.y);
           if constexpr (SI) {
-            const float sg =
-                fmaf((float)Z[3], 16777216.f, fmaf((float)Z[2], 65536.f, fmaf((float)Z[1], 256.f, (float)Z[0])));
-            l = fmaf(gam * a.kappa, fmaf(sg, sc[jj].z, -sc[jj].w), l);
+            const float sg = fmaf((float)(int)Z[4 * qi + 3], 16777216.f,
+                                  fmaf((float)(int)Z[4 * qi + 2], 65536.f,
+                                       fmaf((float)(int)Z[4 * qi + 1], 256.f, (float)(int)Z[4 * qi])));
+            l = fmaf(gam * a.kappa, fmaf(sg, sc.z, -sc.w), l);
           }
           a.logits[(head * a.group + qi) * a.ld + key] = nrm * l;
         }
