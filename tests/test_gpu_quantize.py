@@ -67,3 +67,18 @@ def test_edge_sizes_and_zero_vectors(n):
 def test_short_dim_zero_padding():
     x = wl.to_bf16(wl.head_vectors(300, 64, seed=8))
     _run(64, 3, tq.TQ_MODE_PROD, x, torch.bfloat16)
+
+
+def test_fp16_prod_full_m_and_stride():
+    # fp16 input with a row stride of 136 elements (272 bytes) at m = 128
+    x = wl.head_vectors(500, 128, seed=9).astype(np.float16).astype(np.float32)
+    _run(128, 4, tq.TQ_MODE_PROD, x, torch.float16, ld=136)
+
+
+@pytest.mark.parametrize("bits,mode", [(3, tq.TQ_MODE_PROD), (4, tq.TQ_MODE_MSE), (2, tq.TQ_MODE_PROD)])
+def test_many_tiles_per_cta(bits, mode):
+    # 148 * 128 * 5 + 77 vectors: every CTA of a one-per-SM grid takes five or six
+    # tiles of 128, so the input ring and both accumulator buffers wrap several times
+    n = 148 * 128 * 5 + 77
+    x = wl.to_bf16(wl.head_vectors(n, 128, seed=10))
+    _run(128, bits, mode, x, torch.bfloat16)

@@ -21,7 +21,9 @@ __global__ void bounded_wait_probe_kernel(uint32_t polls) {
 
 namespace tq {
 int fault_word_quantize(int clear, int* value);
+int fault_word_quantize_rt(int clear, int* value);
 int fault_word_logits(int clear, int* value);
+int fault_word_search(int clear, int* value);
 
 int fault_word_diag(int clear, int* value) {
   cudaError_t e = cudaMemcpyFromSymbol(value, tqd::g_fault, sizeof(int));
@@ -39,7 +41,11 @@ extern "C" int tq_device_status(int clear) {
   struct {
     const char* name;
     int (*read)(int, int*);
-  } fam[] = {{"quantize", tq::fault_word_quantize}, {"logits", tq::fault_word_logits}, {"diagnostic", tq::fault_word_diag}};
+  } fam[] = {{"quantize", tq::fault_word_quantize},
+             {"quantize (tensor-core rotation)", tq::fault_word_quantize_rt},
+             {"logits", tq::fault_word_logits},
+             {"search", tq::fault_word_search},
+             {"diagnostic", tq::fault_word_diag}};
   std::string which;
   for (auto& f : fam) {
     int v = 0;

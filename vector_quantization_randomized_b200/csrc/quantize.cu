@@ -406,6 +406,9 @@ int dispatch_kb(int kb, bool prod, int dt, const QArgs& a, int smc, cudaStream_t
 
 namespace tq {
 bool quantize128_supported(const tq_params* p, int dtype);
+bool quantize_rt_supported(const tq_params* p, int dtype);
+int launch_quantize_rt(const tq_params* p, const void* x, int dtype, int64_t n_vec, int64_t ld_bytes, void* codes,
+                       uint16_t* norms, uint16_t* rnorms, int smc, cudaStream_t st);
 int launch_quantize128(const tq_params* p, const void* x, int dtype, int64_t n_vec, int64_t ld_bytes, void* codes,
                        uint16_t* norms, uint16_t* rnorms, int smc, cudaStream_t st);
 int sm_count() {
@@ -453,6 +456,11 @@ extern "C" int tq_quantize(const tq_params* p, const void* x, int dtype, int64_t
   a.S = p->S;
   const bool prod = p->mode == TQ_MODE_PROD;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (quantize_rt_supported(p, dtype)) {
+    rc = launch_quantize_rt(p, x, dtype, n_vec, ld * es, codes, norms, rnorms, sm_count(), st);
+    if (rc == TQ_OK) clear_error();
+    return rc;
+  }
   if (quantize128_supported(p, dtype)) {
     rc = launch_quantize128(p, x, dtype, n_vec, ld * es, codes, norms, rnorms, sm_count(), st);
     if (rc == TQ_OK) clear_error();
