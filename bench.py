@@ -11,7 +11,7 @@ Metric: compressed-key logits, keys/s (keys scored per second over the whole
 step, both bit widths), with per-kernel HBM GB/s and fractions of 8 TB/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload layer|decode|quantize|search]
+                    [--workload layer|decode|quantize|search|polar|project]
 
 N > 1 runs under torchrun, one rank per GPU, each rank a full independent
 layer (weak scaling, no collective on the data path).  Rank 0 prints one JSON
@@ -46,7 +46,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="layer", choices=["layer", "decode", "quantize", "search", "polar"])
+    ap.add_argument("--workload", default="layer",
+                    choices=["layer", "decode", "quantize", "search", "polar", "project"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-kernels", action="store_true")
@@ -60,6 +61,17 @@ def measured_peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def measured_bf16_peak():
+    """Dense bf16 FLOP/s of this machine's B200s (sustained, for a kernel timed in a loop)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        for k in ("bf16_tflops_sustained", "bf16_tflops"):
+            if k in d:
+                return float(d[k]) * 1e12
+    return 1.4e15
 
 
 # --------------------------------------------------------------------------- clocks
@@ -665,6 +677,54 @@ def run_secondary(args, world, rank, local, torch, tq, wl):
                 "config": {"workload": "polar-kv8x32768-gqa4-d128-bf16", "w": [2, 3],
                            "l2": "flushed between steps (256 MB write)"},
                 "kernels": kern}
+    elif args.workload == "project":
+        # quantize-on-write: the K projection of one Llama-3.1-8B-shaped layer over a 32768-token
+        # prefill (x [32768, 4096] bf16, W_k [8 * 128, 4096] bf16) coded in the same kernel, against
+        # the unfused path (cuBLAS bf16 GEMM writing K, then tq_quantize per head)
+        T, hid, H, d = 32768, 4096, 8, 128
+        xnp, wnp = wl.projection_inputs(T, hid, H, wl.SEED_KEYS)
+        x = torch.from_numpy(xnp).to(torch.bfloat16).cuda()
+        w = torch.from_numpy(wnp).to(torch.bfloat16).cuda()
+        del xnp, wnp
+        n = H * T
+        flops = 2.0 * T * hid * H * d
+        bf16_peak = measured_bf16_peak()
+        res = {}
+        for b, mode in ((3, tq.TQ_MODE_PROD), (4, tq.TQ_MODE_PROD), (3, tq.TQ_MODE_MSE)):
+            p = tq.Params(d, b, mode, 128 if mode == tq.TQ_MODE_PROD else 0, wl.SEED_PARAMS)
+            c = torch.empty(p.code_bytes(n), dtype=torch.uint8, device="cuda")
+            nn = torch.empty(n, dtype=torch.int16, device="cuda")
+            rn = torch.empty(n, dtype=torch.int16, device="cuda") if mode == tq.TQ_MODE_PROD else None
+            kbuf = torch.empty((T, H * d), dtype=torch.bfloat16, device="cuda")
+            fused = lambda: tq.tq_project_quantize(p, x, w, H, c, nn, rn)
+
+            def unfused():
+                torch.matmul(x, w.T, out=kbuf)
+                for h in range(H):
+                    tq.tq_quantize(p, kbuf[:, h * d:(h + 1) * d], c[h * (p.code_bytes(T)):], nn[h * T:],
+                                   rn[h * T:] if rn is not None else None, n_vec=T, ld=H * d)
+            out = {}
+            for lab, f in (("fused", fused), ("unfused", unfused)):
+                for _ in range(max(3, args.warmup)):
+                    f()
+                torch.cuda.synchronize()
+                e0, e1 = ev(), ev()
+                e0.record()
+                for _ in range(args.steps):
+                    f()
+                e1.record()
+                torch.cuda.synchronize()
+                ms = e0.elapsed_time(e1) / args.steps
+                out[lab + "_us"] = round(ms * 1000, 1)
+                out[lab + "_tflops"] = round(flops / (ms / 1e3) / 1e12, 1)
+            out["frac_bf16_measured"] = round(out["fused_tflops"] * 1e12 / bf16_peak, 4)
+            out["speedup_vs_unfused"] = round(out["unfused_us"] / out["fused_us"], 3)
+            res[f"b{b}_{'prod' if mode == tq.TQ_MODE_PROD else 'mse'}"] = out
+        line = {"metric": "quantize-on-write tokens/s (K projection + code, one layer)",
+                "value": T / (res["b3_prod"]["fused_us"] / 1e6), "unit": "tokens/s",
+                "config": {"workload": "llama3.1-8b-kproj-prefill-32768x4096-kv8", "bits": [3, 4],
+                           "unfused": "torch.matmul (cuBLAS) writing K, then tq_quantize per head"},
+                "per_bits": res}
     elif args.workload == "search":
         n_db, n_q, d, k = 1000000, 10000, 200, 10
         db = torch.from_numpy(wl.search_set(n_db, d, seed=wl.SEED_KEYS)).to(torch.bfloat16).cuda()

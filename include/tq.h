@@ -65,6 +65,15 @@ typedef struct CUstream_st* tq_stream_t; /* same type as cudaStream_t */
 #define TQ_MODE_PROD 0 /* (bits-1)-bit Lloyd-Max code + m QJL sign bits [E1][E2][E3] */
 #define TQ_MODE_MSE 1  /* bits-bit Lloyd-Max code only (values; 2/pi-biased inner products) */
 
+/* code layouts (tq_params.layout) */
+#define TQ_LAYOUT_PLANES 0 /* canonical: per tile, plane p = 32 vectors x d_pad/8 bytes (above) */
+#define TQ_LAYOUT_SLICED 1 /* token-sliced, MSE codes only: per tile, plane p = d_pad little-endian
+                              32-bit words, word j's bit t = bit p of vector t's index at coordinate j
+                              (same bytes per tile; the value cache tq_decode_attn scans on the tensor
+                              cores).  Written by tq_quantize (d_pad 128, 16-bit input), read by
+                              tq_decode_attn (values) and tq_dequantize; other calls return
+                              TQ_EUNSUPPORTED. */
+
 /* input element types */
 #define TQ_F32 0
 #define TQ_F16 1
@@ -87,7 +96,7 @@ typedef struct tq_params {
   int32_t bits;
   int32_t mode;
   int32_t m;
-  int32_t reserved;
+  int32_t layout; /* TQ_LAYOUT_PLANES (0) or TQ_LAYOUT_SLICED (MSE codes only) */
   const float* centroids;
   const float* thresholds;
   const int8_t* signs_D;
@@ -136,6 +145,32 @@ int tq_quantize(const tq_params* p, const void* x, int dtype, int64_t n_vec, int
                 void* codes, uint16_t* norms, uint16_t* rnorms, tq_stream_t stream);
 
 /*
+ * tq_project_quantize - quantize-on-write: the K (or V) projection of an
+ *   attention layer and tq_quantize of its output in one kernel, so the
+ *   projected vectors never go to memory [Z1: the prefill path of the runtime
+ *   port; E1][E2] for the code.
+ *   Per head h and token t the vector is k = bf16(x_t . W_h^T), the 128
+ *   projection outputs of head h rounded to bf16 as a bf16 cache write would
+ *   round them (fp32 accumulation over `hidden`), then coded exactly as
+ *   tq_quantize codes a bf16 row.
+ *   p: d = d_pad = 128; product mode needs m = 128.
+ *   x: device bf16 [n_tok][hidden], row stride ld_x elements; w: device bf16
+ *      [n_heads*128][hidden] (the layer's weight in [out][in] order, head h =
+ *      rows 128h .. 128h + 127), row stride ld_w.  hidden a positive multiple
+ *      of 32; x, w 16-byte aligned; ld_x, ld_w >= hidden, multiples of 8.
+ *   codes/norms/rnorms: as tq_quantize for n_heads*n_tok vectors, vector
+ *      h*n_tok + t = token t of head h (the per-head key order tq_logits
+ *      reads); code buffer tail zeroed.
+ *   k_out: optional (NULL: not written) device bf16 [n_tok][ld_k], head h in
+ *      columns 128h .. 128h + 127: the vectors that were coded.  ld_k >=
+ *      128*n_heads, a multiple of 8; k_out 16-byte aligned.
+ *   Returns TQ_EUNSUPPORTED for other shapes.
+ */
+int tq_project_quantize(const tq_params* p, const void* x, int64_t n_tok, int64_t ld_x, int hidden,
+                        const void* w, int n_heads, int64_t ld_w, void* codes, uint16_t* norms,
+                        uint16_t* rnorms, void* k_out, int64_t ld_k, tq_stream_t stream);
+
+/*
  * tq_dequantize - the reconstruction x_hat = Q^-1(codes) [E2: the QJL part is
  *   sqrt(pi/2)/m * gamma * S^T sigma, sigma = 2s - 1, which makes
  *   E[<y, Q^-1(Q(x))>] = <y, x>]:
@@ -167,7 +202,9 @@ int tq_dequantize(const tq_params* p, const void* codes, const uint16_t* norms,
  *      16-byte aligned norms) prepares the queries inside its kernel and does
  *      not touch the workspace; the other shapes keep their query
  *      preparation there.
- * Supported: d_pad 128 with kb <= 3, d_pad 256 with kb <= 2.
+ * Supported: d_pad 128 with kb <= 3; d_pad 256 with kb <= 2; d_pad 256 with
+ *   kb = 3 in MSE mode or with m = 256 (the tensor-memory scan of
+ *   tq_search_topk writing every score; n_keys % 32 == 0 when n_kv_heads > 1).
  */
 int64_t tq_logits_workspace(const tq_params* p, int n_q);
 int tq_logits(const tq_params* p, const float* q, int n_q, int group, const void* codes,

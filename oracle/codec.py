@@ -28,6 +28,12 @@ vector t at byte offset t*d_pad/8, coordinate j at bit j%32 of little-endian
 32-bit word j//32; then the sign words, 32 x m/8 bytes, sign i at bit i%32 of
 word i//32.  The last tile is zero-filled.  Norms and residual norms are
 separate fp16 arrays indexed by vector.
+
+Token-sliced layout (MSE codes only; the value cache read by the decode scan):
+the same tiles of 32 vectors and the same k_b planes, but plane p of a tile
+is d_pad little-endian 32-bit words, one per coordinate j in order, whose bit
+t is bit p of the index of vector t of the tile at coordinate j.  Same bytes
+per tile as the canonical layout; the last tile is zero-filled.
 """
 import functools
 
@@ -184,3 +190,29 @@ def unpack(buf, n, d_pad, kb, m):
         base = tile * tile_bytes + kb * TILE * pb + slot * sb
         signs = _bytes_to_bits(buf[base[:, None] + np.arange(sb)[None, :]], m)
     return idx, signs
+
+
+def pack_sliced(idx, kb):
+    """Token-sliced code buffer (uint8) from MSE indices [n, d_pad]."""
+    idx = np.asarray(idx, dtype=np.uint8)
+    n, d_pad = idx.shape
+    n_tiles = (n + TILE - 1) // TILE
+    words = np.zeros((n_tiles, kb, d_pad), dtype=np.uint32)
+    for v in range(n):
+        tile, t = divmod(v, TILE)
+        for p in range(kb):
+            bits = ((idx[v] >> p) & 1).astype(np.uint32)
+            words[tile, p] |= bits << np.uint32(t)
+    return words.reshape(-1).astype("<u4").view(np.uint8).copy()
+
+
+def unpack_sliced(buf, n, d_pad, kb):
+    """Inverse of `pack_sliced`: indices uint8 [n, d_pad]."""
+    n_tiles = (n + TILE - 1) // TILE
+    words = np.asarray(buf, dtype=np.uint8)[:n_tiles * kb * d_pad * 4].view("<u4").reshape(n_tiles, kb, d_pad)
+    idx = np.zeros((n, d_pad), dtype=np.uint8)
+    for v in range(n):
+        tile, t = divmod(v, TILE)
+        for p in range(kb):
+            idx[v] |= (((words[tile, p] >> np.uint32(t)) & 1) << p).astype(np.uint8)
+    return idx

@@ -23,12 +23,12 @@ class OracleParams:
         self.S = qjl_matrix(seed, m, d_pad) if m else None
 
 
-def make_pair(d, bits, mode=tq.TQ_MODE_PROD, m=None, seed=42):
+def make_pair(d, bits, mode=tq.TQ_MODE_PROD, m=None, seed=42, layout=tq.TQ_LAYOUT_PLANES):
     d_pad = 128 if d <= 128 else 256
     if mode == tq.TQ_MODE_PROD and m is None:
         m = d_pad
     m = m if mode == tq.TQ_MODE_PROD else 0
-    return tq.Params(d, bits, mode, m, seed, d_pad), OracleParams(d, bits, mode, m, seed, d_pad)
+    return tq.Params(d, bits, mode, m, seed, d_pad, layout=layout), OracleParams(d, bits, mode, m, seed, d_pad)
 
 
 def gpu_quantize(p, x_t):
@@ -83,6 +83,22 @@ def compare_codes(op, x, codes, norms, rnorms):
         assert np.all(ok_r), f"residual norm mismatches at {np.argwhere(~ok_r)[:10].ravel()}"
         out.update(sign_flagged=int(fl["signs"].sum()), sign_mismatch=int(sd.sum()))
     return out
+
+
+def compare_codes_sliced(op, x, codes, norms):
+    """compare_codes for MSE codes in the token-sliced layout (unpacked by the oracle)."""
+    n = x.shape[0]
+    enc = codec.encode(x, op.D, op.c, op.t, None)
+    fl = codec.boundary_flags(enc, op.t, None)
+    n_tail = (-n) % 32
+    idx_all = codec.unpack_sliced(codes, n + n_tail, op.d_pad, op.kb)
+    assert not np.any(idx_all[n:]), "tail indices not zeroed"
+    idx = idx_all[:n]
+    dif = idx != enc["idx"]
+    assert not np.any(dif & ~fl["idx"]), f"unflagged index mismatches: {np.argwhere(dif & ~fl['idx'])[:10]}"
+    ok_n = (norms == enc["norm_f16"]) | (fl["norm"] & f16_neighbours(norms, enc["norm_f16"]))
+    assert np.all(ok_n), f"norm mismatches at {np.argwhere(~ok_n)[:10].ravel()}"
+    return dict(n=n, idx_flagged=int(fl["idx"].sum()), idx_mismatch=int(dif.sum()))
 
 
 def oracle_codes(op, x):

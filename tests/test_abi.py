@@ -63,11 +63,11 @@ def test_code_bytes():
 
 
 def _fake_params(**kw):
-    p = dict(d=128, d_pad=128, bits=4, mode=tq.TQ_MODE_PROD, m=128)
+    p = dict(d=128, d_pad=128, bits=4, mode=tq.TQ_MODE_PROD, m=128, layout=tq.TQ_LAYOUT_PLANES)
     p.update(kw)
     buf = np.zeros(64, np.float32)
     ptr = buf.ctypes.data
-    st = tq.tq_params(p["d"], p["d_pad"], p["bits"], p["mode"], p["m"], 0, ptr, ptr, ptr, ptr)
+    st = tq.tq_params(p["d"], p["d_pad"], p["bits"], p["mode"], p["m"], p["layout"], ptr, ptr, ptr, ptr)
     return st, buf
 
 
@@ -80,6 +80,8 @@ def _fake_params(**kw):
     (dict(m=48), tq.TQ_EINVAL),
     (dict(mode=7), tq.TQ_EINVAL),
     (dict(mode=tq.TQ_MODE_MSE, m=128), tq.TQ_EINVAL),
+    (dict(layout=7), tq.TQ_EINVAL),                                     # unknown layout
+    (dict(layout=tq.TQ_LAYOUT_SLICED), tq.TQ_EINVAL),                   # sliced holds MSE codes only
 ])
 def test_validation_rejects_bad_params(kw, code):
     st, keep = _fake_params(**kw)
@@ -112,8 +114,8 @@ def test_validation_rejects_null_and_misaligned():
     # logits: workspace too small
     assert lib.tq_logits(ctypes.byref(st), base16, 4, 4, base16, base16, base16, 100, 1, base16, base16, 16,
                          None) == tq.TQ_EINVAL
-    # logits: unsupported shape (d_pad 256 with 3 index bits)
-    st2, keep2 = _fake_params(d=200, d_pad=256, m=256)
+    # logits: unsupported shape (d_pad 256 with 3 index bits takes MSE codes or m = 256)
+    st2, keep2 = _fake_params(d=200, d_pad=256, m=128)
     assert lib.tq_logits(ctypes.byref(st2), base16, 4, 4, base16, base16, base16, 100, 1, base16, base16,
                          1 << 20, None) == tq.TQ_EUNSUPPORTED
     # decode: value params must be MSE mode

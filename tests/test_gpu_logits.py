@@ -69,3 +69,31 @@ def test_small_m():
 def test_tiny():
     _check(128, 4, tq.TQ_MODE_PROD, n_heads=1, group=1, n_keys=1)
     _check(128, 4, tq.TQ_MODE_PROD, n_heads=1, group=4, n_keys=9)
+
+
+# d_pad 256 with 3 index bits (b = 4 product codes at d = 200, config 4's codes; b = 3 MSE codes):
+# the tensor-memory search scan writing every score
+@pytest.mark.parametrize("bits,mode,n_heads,group,n_keys", [
+    (4, tq.TQ_MODE_PROD, 1, 4, 700),      # one head, ragged key count
+    (4, tq.TQ_MODE_PROD, 2, 5, 640),      # a 16-query chunk with 5 queries per head
+    (4, tq.TQ_MODE_PROD, 2, 20, 320),     # two chunks per head
+    (3, tq.TQ_MODE_MSE, 2, 4, 8992),      # three key splits per head
+])
+def test_padded_dim_256_three_index_bits(bits, mode, n_heads, group, n_keys):
+    _check(200, bits, mode, n_heads=n_heads, group=group, n_keys=n_keys)
+
+
+def test_padded_dim_256_three_index_bits_unsupported_shapes():
+    p, _ = make_pair(200, 4, tq.TQ_MODE_PROD, m=128)   # the scan needs m = 256 (or MSE)
+    q = torch.zeros((4, 200), device="cuda")
+    c = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+    nn = torch.zeros(64, dtype=torch.int16, device="cuda")
+    out = torch.zeros((4, 64), device="cuda")
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tq.TQError):
+        tq.tq_logits(p, q, 4, c, nn, nn, 64, 1, out, ws)
+    p2, _ = make_pair(200, 4, tq.TQ_MODE_PROD)         # several heads need n_keys % 32 == 0
+    out2 = torch.zeros((8, 50), device="cuda")
+    q2 = torch.zeros((8, 200), device="cuda")
+    with pytest.raises(tq.TQError):
+        tq.tq_logits(p2, q2, 4, c, nn, nn, 50, 2, out2, ws)

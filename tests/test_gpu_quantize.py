@@ -82,3 +82,39 @@ def test_many_tiles_per_cta(bits, mode):
     n = 148 * 128 * 5 + 77
     x = wl.to_bf16(wl.head_vectors(n, 128, seed=10))
     _run(128, bits, mode, x, torch.bfloat16)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_bf16_mse_token_sliced(bits):
+    # value-cache layout: per tile and plane, one 32-bit word per coordinate over the tile's vectors
+    from gpu_util import compare_codes_sliced
+    x = wl.to_bf16(wl.head_vectors(1001, 128, seed=11))
+    p, op = make_pair(128, bits, tq.TQ_MODE_MSE, layout=tq.TQ_LAYOUT_SLICED)
+    xt = torch.from_numpy(x).to(torch.bfloat16).cuda()
+    codes, norms, _ = gpu_quantize(p, xt)
+    compare_codes_sliced(op, x.astype(np.float64), codes, norms)
+    # the same indices as the canonical layout, and the same reconstruction
+    p2, _ = make_pair(128, bits, tq.TQ_MODE_MSE)
+    codes2, norms2, _ = gpu_quantize(p2, xt)
+    from oracle import codec
+    assert np.array_equal(codec.unpack_sliced(codes, 1001, 128, p.kb), codec.unpack(codes2, 1001, 128, p.kb, 0)[0])
+    outs = []
+    for pp, cc, nn in ((p, codes, norms), (p2, codes2, norms2)):
+        out = torch.zeros((1001, 128), device="cuda")
+        tq.tq_dequantize(pp, torch.from_numpy(cc).cuda(), torch.from_numpy(nn.view(np.int16)).cuda(), None, 1001, out)
+        outs.append(out.cpu().numpy())
+    assert np.array_equal(outs[0], outs[1])
+
+
+def test_token_sliced_unsupported_shapes():
+    p, _ = make_pair(128, 3, tq.TQ_MODE_MSE, layout=tq.TQ_LAYOUT_SLICED)
+    x = torch.zeros((64, 128), dtype=torch.float32, device="cuda")     # fp32 input: not on the sliced path
+    c = torch.zeros(p.code_bytes(64), dtype=torch.uint8, device="cuda")
+    nn = torch.zeros(64, dtype=torch.int16, device="cuda")
+    with pytest.raises(tq.TQError):
+        tq.tq_quantize(p, x, c, nn)
+    q = torch.zeros((4, 128), device="cuda")
+    out = torch.zeros((4, 64), device="cuda")
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tq.TQError):                                     # logits read canonical planes only
+        tq.tq_logits(p, q, 4, c, nn, None, 64, 1, out, ws)

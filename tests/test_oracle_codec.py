@@ -181,3 +181,39 @@ def test_signs_follow_projection():
     np.testing.assert_array_equal(enc["signs"], (z >= 0).astype(np.uint8))
     # the estimator's QJL term needs E[sign] structure: about half the bits set
     assert 0.4 < enc["signs"].mean() < 0.6
+
+
+def test_sliced_layout_hand_example():
+    # 33 vectors of d_pad 8 at kb = 2: vector 1 has index 3 at coordinate 5 (both planes), vector 32
+    # (tile 1, t = 0) has index 2 at coordinate 0 (plane 1 only); everything else 0
+    idx = np.zeros((33, 8), dtype=np.uint8)
+    idx[1, 5] = 3
+    idx[32, 0] = 2
+    buf = codec.pack_sliced(idx, 2)
+    w = buf.view("<u4").reshape(2, 2, 8)          # [tile][plane][coordinate]
+    want = np.zeros((2, 2, 8), dtype=np.uint32)
+    want[0, 0, 5] = 1 << 1
+    want[0, 1, 5] = 1 << 1
+    want[1, 1, 0] = 1
+    assert np.array_equal(w, want)
+    assert buf.size == codec.code_bytes(8, 2, 0, 33)
+    assert np.array_equal(codec.unpack_sliced(buf, 33, 8, 2), idx)
+
+
+def test_sliced_layout_is_the_transposed_tile():
+    # each tile's plane in the sliced layout is the 32 x d_pad bit matrix of the canonical plane, transposed
+    r = np.random.default_rng(3)
+    n, d_pad, kb = 77, 128, 3
+    idx = r.integers(0, 1 << kb, size=(n, d_pad)).astype(np.uint8)
+    s = codec.pack_sliced(idx, kb)
+    assert np.array_equal(codec.unpack_sliced(s, n, d_pad, kb), idx)
+    c = codec.pack(idx, None, kb, 0)
+    assert s.size == c.size
+    tb = 32 * kb * d_pad // 8
+    for tile in range((n + 31) // 32):
+        for p in range(kb):
+            cp = np.unpackbits(c[tile * tb + p * 32 * d_pad // 8: tile * tb + (p + 1) * 32 * d_pad // 8]
+                               .reshape(32, d_pad // 8), axis=1, bitorder="little")          # [t][j]
+            sp = np.unpackbits(s[tile * tb + p * d_pad * 4: tile * tb + (p + 1) * d_pad * 4]
+                               .reshape(d_pad, 4), axis=1, bitorder="little")                # [j][t]
+            assert np.array_equal(cp.T, sp)

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libtq.so")
 TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECUDA, TQ_ETIMEOUT = 0, -1, -2, -3, -4
 TQ_MODE_PROD, TQ_MODE_MSE = 0, 1
 TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
+TQ_LAYOUT_PLANES, TQ_LAYOUT_SLICED = 0, 1
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} not found: build it with `python vector_quantization_randomized_b200/build.py`")
@@ -26,7 +27,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 class tq_params(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("d_pad", ctypes.c_int32), ("bits", ctypes.c_int32),
-                ("mode", ctypes.c_int32), ("m", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("mode", ctypes.c_int32), ("m", ctypes.c_int32), ("layout", ctypes.c_int32),
                 ("centroids", ctypes.c_void_p), ("thresholds", ctypes.c_void_p),
                 ("signs_D", ctypes.c_void_p), ("S", ctypes.c_void_p)]
 
@@ -44,6 +45,7 @@ _SIGS = {
     "tq_make_params": (_i32, [_i32, _i32, _u64, _vp, _vp]),
     "tq_code_bytes": (_i64, [_i32, _i32, _i32, _i64]),
     "tq_quantize": (_i32, [_P, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "tq_project_quantize": (_i32, [_P, _vp, _i64, _i64, _i32, _vp, _i32, _i64, _vp, _vp, _vp, _vp, _i64, _vp]),
     "tq_dequantize": (_i32, [_P, _vp, _vp, _vp, _i64, _vp, _i64, _vp]),
     "tq_logits_workspace": (_i64, [_P, _i32]),
     "tq_logits": (_i32, [_P, _vp, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _i64, _vp]),
@@ -149,7 +151,7 @@ def tq_code_bytes(d_pad, kb, m, n_vec):
 class Params:
     """A quantizer: host-made codebook/D/S copied to the device, plus the C struct."""
 
-    def __init__(self, d, bits, mode=TQ_MODE_PROD, m=None, seed=42, d_pad=None, device="cuda"):
+    def __init__(self, d, bits, mode=TQ_MODE_PROD, m=None, seed=42, d_pad=None, device="cuda", layout=0):
         import torch
         d_pad = d_pad or (128 if d <= 128 else 256)
         if mode == TQ_MODE_PROD and m is None:
@@ -164,7 +166,8 @@ class Params:
         self.thresholds = torch.from_numpy(t).to(device)
         self.D = torch.from_numpy(D).to(device)
         self.S = torch.from_numpy(S.view(np.int16)).to(device) if m else None
-        self.struct = tq_params(d, d_pad, bits, mode, m, 0, _ptr(self.centroids), _ptr(self.thresholds),
+        self.layout = layout
+        self.struct = tq_params(d, d_pad, bits, mode, m, layout, _ptr(self.centroids), _ptr(self.thresholds),
                                 _ptr(self.D), _ptr(self.S))
 
     @property
@@ -186,6 +189,15 @@ def tq_quantize(p, x, codes, norms, rnorms=None, n_vec=None, ld=None, stream=Non
     ld = x.stride(0) if ld is None else ld
     return _check(_lib.tq_quantize(p.ref, _ptr(x), _dtype_code(x), n_vec, ld, _ptr(codes), _ptr(norms),
                                    _ptr(rnorms), _stream(stream)))
+
+
+def tq_project_quantize(p, x, w, n_heads, codes, norms, rnorms=None, k_out=None, stream=None):
+    """Fused K/V projection + encode: vectors bf16(x W_h^T) of every head h (x: device bf16
+    [n_tok, hidden]; w: device bf16 [n_heads * 128, hidden]); vector h * n_tok + t is token t of
+    head h.  k_out (optional, device bf16 [n_tok, >= n_heads * 128]) receives the projected rows."""
+    return _check(_lib.tq_project_quantize(p.ref, _ptr(x), x.shape[0], x.stride(0), x.shape[1], _ptr(w), n_heads,
+                                           w.stride(0), _ptr(codes), _ptr(norms), _ptr(rnorms), _ptr(k_out),
+                                           k_out.stride(0) if k_out is not None else 0, _stream(stream)))
 
 
 def tq_dequantize(p, codes, norms, rnorms, n_vec, out, ld=None, stream=None):

@@ -24,5 +24,7 @@ inline int index_bits(const tq_params* p) { return p->mode == TQ_MODE_PROD ? p->
 
 // Validate a tq_params struct; returns TQ_OK or a TQ_E* (message set).
 int check_params(const tq_params* p, const char* who);
+// TQ_EUNSUPPORTED unless the codes are in the canonical bit-plane layout.
+int check_planes(const tq_params* p, const char* who);
 
 }  // namespace tq

@@ -542,7 +542,10 @@ extern "C" int64_t tq_decode_attn_workspace(const tq_params* kp, int batch, int 
   const int nqc = (group + tqd::QCHUNK - 1) / tqd::QCHUNK;
   int64_t prep = (int64_t)batch * n_kv_heads * nqc * tqd::prep_chunk_bytes(sh.fr);
   prep = (prep + 255) & ~(int64_t)255;
-  return prep + decode_ws_parts(batch, n_q_heads, max_tokens);
+  // the values' layout is not known here: enough for either decode
+  const int64_t sliced = tq::decode_sliced_workspace(kb, kp->mode == TQ_MODE_PROD ? kp->m : 0, batch, n_q_heads,
+                                                     n_kv_heads, max_tokens);
+  return std::max<int64_t>(prep + decode_ws_parts(batch, n_q_heads, max_tokens), sliced);
 }
 
 namespace {
@@ -552,9 +555,17 @@ int decode_attn(const tq_params* kp, const tq_params* vp, const float* q, int ba
                 float* out, float* partial_out, void* workspace, int64_t workspace_bytes, tq_stream_t stream) {
   using namespace tq;
   int rc = check_params(kp, "tq_decode_attn(kp)");
+  if (!rc) rc = check_planes(kp, "tq_decode_attn(kp)");
   if (rc) return rc;
   rc = check_params(vp, "tq_decode_attn(vp)");
   if (rc) return rc;
+  if (vp->layout != TQ_LAYOUT_PLANES) {  // token-sliced values: the tensor-memory decode
+    if (partial_out || v_eps != 0.f)
+      return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: token-sliced values take the full decode only");
+    return decode_attn_sliced(kp, vp, q, batch, n_q_heads, n_kv_heads, kcodes, knorms, krnorms, vcodes, vnorms,
+                              seq_lens, max_tokens, scale, out, workspace, workspace_bytes,
+                              reinterpret_cast<cudaStream_t>(stream));
+  }
   if (kp->mode != TQ_MODE_PROD || vp->mode != TQ_MODE_MSE)
     return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: needs product-code keys and MSE-code values");
   if (kp->d_pad != 128 || vp->d_pad != 128 || kp->d != vp->d)

@@ -34,6 +34,7 @@ struct QArgs {
   const uint16_t* S;
   int64_t n_vec, ld;
   int d, m, tb;
+  int sliced;   // token-sliced layout (MSE codes): plane p of a tile = DP words, word j bit t
   float kappa;  // sqrt(pi/2) / m
   float* out;
 };
@@ -61,11 +62,20 @@ __global__ void __launch_bounds__(256) dequant_kernel(const QArgs a) {
     // index bits of this lane's coordinates: word NI*lane/32, bits (NI*lane) % 32 ..
     const int wsel = (NI * lane) >> 5, sh = (NI * lane) & 31;
     int idx[NI] = {};
+    if (!PROD && a.sliced) {  // words NI*lane .. of each plane, bit `slot`
 #pragma unroll
-    for (int p = 0; p < KB; ++p) {
-      const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(tile + p * TILE * (DP / 8) + slot * (DP / 8)) + wsel);
+      for (int p = 0; p < KB; ++p) {
+        const uint32_t* wp = reinterpret_cast<const uint32_t*>(tile + p * (DP * 4)) + NI * lane;
 #pragma unroll
-      for (int k = 0; k < NI; ++k) idx[k] |= (int)((w >> (sh + k)) & 1u) << p;
+        for (int k = 0; k < NI; ++k) idx[k] |= (int)((__ldg(wp + k) >> slot) & 1u) << p;
+      }
+    } else {
+#pragma unroll
+      for (int p = 0; p < KB; ++p) {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(tile + p * TILE * (DP / 8) + slot * (DP / 8)) + wsel);
+#pragma unroll
+        for (int k = 0; k < NI; ++k) idx[k] |= (int)((w >> (sh + k)) & 1u) << p;
+      }
     }
     float y[NI];
 #pragma unroll
@@ -179,6 +189,7 @@ extern "C" int tq_dequantize(const tq_params* p, const void* codes, const uint16
   a.d = p->d;
   a.m = prod ? p->m : 0;
   a.tb = tqd::tile_bytes(p->d_pad, kb, a.m);
+  a.sliced = p->layout == TQ_LAYOUT_SLICED;
   a.kappa = prod ? (float)(std::sqrt(M_PI / 2.0) / p->m) : 0.f;
   a.out = out;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -41,10 +41,20 @@ int check_params(const tq_params* p, const char* who) {
   } else {
     return set_error(TQ_EINVAL, "%s: unknown mode %d", who, p->mode);
   }
+  if (p->layout != TQ_LAYOUT_PLANES && p->layout != TQ_LAYOUT_SLICED)
+    return set_error(TQ_EINVAL, "%s: unknown code layout %d", who, p->layout);
+  if (p->layout == TQ_LAYOUT_SLICED && p->mode != TQ_MODE_MSE)
+    return set_error(TQ_EINVAL, "%s: the token-sliced layout holds MSE codes only", who);
   if (!p->centroids || !p->thresholds || !p->signs_D)
     return set_error(TQ_EINVAL, "%s: centroids/thresholds/signs_D must be non-NULL", who);
   if (!aligned(p->centroids, 4) || !aligned(p->thresholds, 4))
     return set_error(TQ_EINVAL, "%s: codebook arrays must be 4-byte aligned", who);
+  return TQ_OK;
+}
+
+int check_planes(const tq_params* p, const char* who) {
+  if (p->layout != TQ_LAYOUT_PLANES)
+    return set_error(TQ_EUNSUPPORTED, "%s: needs codes in the canonical bit-plane layout", who);
   return TQ_OK;
 }
 

@@ -280,11 +280,18 @@ int64_t prep_chunk_bytes_max(int dp, int kb, int m) {
 }
 }  // namespace tq
 
+// d_pad 256 with 3 index bits runs on the tensor-memory search scan in all-scores mode.
+static bool logits_on_stc(const tq_params* p, int kb) {
+  return p->d_pad == 256 && kb == 3 && tq::search_tc_supported(256, kb, p->mode == TQ_MODE_PROD ? p->m : 0);
+}
+
 extern "C" int64_t tq_logits_workspace(const tq_params* p, int n_q) {
   if (!p || n_q < 0) return -1;
   const int kb = p->mode == TQ_MODE_PROD ? p->bits - 1 : p->bits;
   if (kb < 1 || kb > 4 || (p->d_pad != 128 && p->d_pad != 256)) return -1;
-  return (int64_t)n_q * tq::prep_chunk_bytes_max(p->d_pad, kb, p->mode == TQ_MODE_PROD ? p->m : 0);
+  const int m = p->mode == TQ_MODE_PROD ? p->m : 0;
+  if (logits_on_stc(p, kb)) return tq::logits_stc_workspace(kb, m, n_q);
+  return (int64_t)n_q * tq::prep_chunk_bytes_max(p->d_pad, kb, m);
 }
 
 extern "C" int tq_logits_ld(const tq_params* p, const float* q, int n_q, int group, const void* codes,
@@ -293,12 +300,15 @@ extern "C" int tq_logits_ld(const tq_params* p, const float* q, int n_q, int gro
                             tq_stream_t stream) {
   using namespace tq;
   int rc = check_params(p, "tq_logits");
+  if (!rc) rc = check_planes(p, "tq_logits");
   if (rc) return rc;
   if (ld_logits < n_keys) return set_error(TQ_EINVAL, "tq_logits: ld_logits < n_keys");
   const int kb = index_bits(p);
   const bool prod = p->mode == TQ_MODE_PROD;
-  if (!scan_supported(p->d_pad, kb))
-    return set_error(TQ_EUNSUPPORTED, "tq_logits: d_pad=%d with %d index bits is not supported", p->d_pad, kb);
+  const bool stc = logits_on_stc(p, kb);
+  if (!scan_supported(p->d_pad, kb) && !stc)
+    return set_error(TQ_EUNSUPPORTED, "tq_logits: d_pad=%d with %d index bits (m=%d) is not supported", p->d_pad,
+                     kb, p->m);
   if (group < 1 || n_kv_heads < 1 || (int64_t)n_kv_heads * group != n_q)
     return set_error(TQ_EINVAL, "tq_logits: need n_q == n_kv_heads * group (n_q=%d, heads=%d, group=%d)", n_q,
                      n_kv_heads, group);
@@ -312,13 +322,24 @@ extern "C" int tq_logits_ld(const tq_params* p, const float* q, int n_q, int gro
   if (!aligned(codes, 16) || !aligned(workspace, 16) || !aligned(q, 4) || !aligned(logits, 4))
     return set_error(TQ_EINVAL, "tq_logits: misaligned pointer (codes/workspace need 16 bytes)");
   const int m = prod ? p->m : 0;
+  cudaStream_t st0 = reinterpret_cast<cudaStream_t>(stream);
+  if (stc) {  // tensor-memory scan of the search kernel, every score written
+    if (n_kv_heads > 1 && n_keys % 32 != 0)
+      return set_error(TQ_EUNSUPPORTED, "tq_logits: d_pad 256 with 3 index bits needs n_keys %% 32 == 0 for "
+                                        "more than one KV head");
+    const int64_t need = logits_stc_workspace(kb, m, n_q);
+    if (workspace_bytes < need)
+      return set_error(TQ_EINVAL, "tq_logits: workspace too small (%lld < %lld bytes)", (long long)workspace_bytes,
+                       (long long)need);
+    rc = launch_logits_stc(p, kb, q, n_kv_heads, group, codes, norms, rnorms, n_keys, logits, ld_logits, workspace,
+                           st0);
+    if (rc == TQ_OK) clear_error();
+    return rc;
+  }
   const tqd::ScanShape sh(p->d_pad, kb, m);
   const int nqc = (group + tqd::QCHUNK - 1) / tqd::QCHUNK;
   const int chunks = n_kv_heads * nqc;
   const int64_t need = (int64_t)chunks * tqd::prep_chunk_bytes(sh.fr);
-  if (workspace_bytes < need)
-    return set_error(TQ_EINVAL, "tq_logits: workspace too small (%lld < %lld bytes)", (long long)workspace_bytes,
-                     (long long)need);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (logits_tc_supported(p->d_pad, kb, m, group, n_keys, norms, rnorms)) {
     // tensor-memory scan with the query preparation inside the kernel: the workspace is not used
@@ -327,6 +348,9 @@ extern "C" int tq_logits_ld(const tq_params* p, const float* q, int n_q, int gro
     if (rc == TQ_OK) clear_error();
     return rc;
   }
+  if (workspace_bytes < need)  // the other scans keep their query preparation in the workspace
+    return set_error(TQ_EINVAL, "tq_logits: workspace too small (%lld < %lld bytes)", (long long)workspace_bytes,
+                     (long long)need);
   tqd::PrepArgs pa;
   pa.q = q;
   pa.d = p->d;
@@ -454,6 +478,7 @@ extern "C" int tq_logits_noalloc(const tq_params* p, const float* q, int n_q, in
                                  float* logits, tq_stream_t stream) {
   using namespace tq;
   int rc = check_params(p, "tq_logits_noalloc");
+  if (!rc) rc = check_planes(p, "tq_logits_noalloc");
   if (rc) return rc;
   if (group < 1 || n_kv_heads < 1 || (int64_t)n_kv_heads * group != n_q)
     return set_error(TQ_EINVAL, "tq_logits_noalloc: need n_q == n_kv_heads * group");

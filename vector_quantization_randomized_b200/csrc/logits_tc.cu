@@ -122,6 +122,7 @@ __device__ __forceinline__ float pow2(int k) {
 struct PrepRegs {
   float y[4];
   uint4 sv[8];
+  float cv;  // centroid et (et < 2^kb)
 };
 
 template <int SI>
@@ -129,6 +130,7 @@ __device__ __forceinline__ void prep_load(const TArgs& a, int64_t head0, int n_i
   const int ew = et >> 5, lane = et & 31;
   const int k = ew >> 2, j = ew & 3;
   const bool valid = k < n_img && j < a.group;
+  pr.cv = et < (1 << a.kb) ? __ldg(a.cent + et) : 0.f;
   const int64_t row = (head0 + k) * a.group + j;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -148,9 +150,9 @@ __device__ __forceinline__ void prep_load(const TArgs& a, int64_t head0, int n_i
 // q_rot = H D q / sqrt(128) (warp per query: image ew / 4, query ew % 4);
 // u = S q_rot (thread = row of S x half of the coordinates, both images);
 // per-query scales 2^F, 2^G putting the largest weight just below 2^23; digits.
-template <int KB, int SI>
+template <int KB, int SI, class Sync>
 __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* img0, uint8_t* img1, float4* qT,
-                            float4* uT, float4* up, const float* alpha, float* red, int et, GroupSync& gs) {
+                            float4* uT, float4* up, const float* alpha, float* red, int et, Sync&& sync) {
   using L = TL<KB, SI>;
   const int ew = et >> 5, lane = et & 31;
   const int kq = ew >> 2, jq = ew & 3;  // this warp's image and query
@@ -190,38 +192,40 @@ __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* im
       rd[4 * jq + 1] = mx;
     }
   }
-  gs.sync(lane);
+  sync();
   if constexpr (SI) {  // u = S q_rot: row i = et % 128, coordinates 64h .. 64h + 63 (h = et / 128)
     const int i = et & 127, h = et >> 7;
-    float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+    float2 acc[2][2];  // [image][queries 0-1, 2-3], packed fp32x2
+#pragma unroll
+    for (int im = 0; im < 2; ++im) acc[im][0] = acc[im][1] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const uint32_t wv[4] = {pr.sv[k].x, pr.sv[k].y, pr.sv[k].z, pr.sv[k].w};
 #pragma unroll
       for (int h2 = 0; h2 < 4; ++h2) {
         const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[h2]));
+        const float2 fx = make_float2(f.x, f.x), fy = make_float2(f.y, f.y);
         const int j = 64 * h + 8 * k + 2 * h2;
 #pragma unroll
         for (int im = 0; im < 2; ++im) {
           if (im < n_img) {
             const float4 q0 = qT[128 * im + j], q1 = qT[128 * im + j + 1];
-            acc[im].x = fmaf(f.y, q1.x, fmaf(f.x, q0.x, acc[im].x));
-            acc[im].y = fmaf(f.y, q1.y, fmaf(f.x, q0.y, acc[im].y));
-            acc[im].z = fmaf(f.y, q1.z, fmaf(f.x, q0.z, acc[im].z));
-            acc[im].w = fmaf(f.y, q1.w, fmaf(f.x, q0.w, acc[im].w));
+            acc[im][0] = __ffma2_rn(fy, make_float2(q1.x, q1.y), __ffma2_rn(fx, make_float2(q0.x, q0.y), acc[im][0]));
+            acc[im][1] = __ffma2_rn(fy, make_float2(q1.z, q1.w), __ffma2_rn(fx, make_float2(q0.z, q0.w), acc[im][1]));
           }
         }
       }
     }
 #pragma unroll
-    for (int im = 0; im < 2; ++im) up[256 * im + 128 * h + i] = acc[im];
-    gs.sync(lane);
+    for (int im = 0; im < 2; ++im)
+      up[256 * im + 128 * h + i] = make_float4(acc[im][0].x, acc[im][0].y, acc[im][1].x, acc[im][1].y);
+    sync();
     {
       const int im = et >> 7, r = et & 127;  // thread = (image, row)
       const float4 p0 = up[256 * im + r], p1 = up[256 * im + 128 + r];
       uT[128 * im + r] = make_float4(p0.x + p1.x, p0.y + p1.y, p0.z + p1.z, p0.w + p1.w);
     }
-    gs.sync(lane);
+    sync();
   }
   if (kq < n_img) {  // scales and per-query scalars: warp = (image kq, query jq)
     float su = 0.f, mu = 0.f;
@@ -248,7 +252,7 @@ __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* im
           make_float4(pow2(-(F + 7)), alpha[4] * rd[4 * jq], pow2(-(G + 7)), su);
     }
   }
-  gs.sync(lane);
+  sync();
   // Digit words, one thread per (image, query q, plane P, bit class c, word w): the
   // weights of coordinates 32w + 8b + c (b = 0..3) give word w of K chunk c of plane P
   // in the 4 digit rows 4q + d.  Scaling by 2^F (2^G) is exact.
@@ -280,7 +284,7 @@ __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* im
     for (int dd = 0; dd < 4; ++dd) *reinterpret_cast<uint32_t*>(base + (4 * (q & 1) + dd) * 16) = W[dd];
   }
   fence_async_smem();  // the images are read by the tensor core (async proxy)
-  gs.sync(lane);
+  sync();
 }
 
 template <int KB, int SI>
@@ -427,8 +431,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       uint4 pw[KB + SI];
 #pragma unroll
       for (int p = 0; p < KB + SI; ++p) pw[p] = *reinterpret_cast<const uint4*>(st + p * 512);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      release_to_copy(&empty[s], lane);  // the stage is refilled once its 8 readers release it
       uint4 it[L::NP];
 #pragma unroll
       for (int T = 0; T < L::NT; ++T) it[T] = pw[T < KB ? T : 0];
@@ -465,21 +468,25 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
     const int et = threadIdx.x - 32 * W_EPI0;
     const int ew = warp - W_EPI0;
     const int qd = warp & 3, par = ew >> 2;
-    if (et < L::NT + 1) {  // Walsh coefficients of the odd-symmetric codebook (fp64), c[L-1]
-      const int Lv = 1 << KB;
+    if (et < 32) {  // Walsh coefficients of the odd-symmetric codebook (fp64), c[L-1]; lane l holds c[l]
+      constexpr int Lv = 1 << KB;
+      const int mask = et < L::NT ? walsh_mask(KB, et) : 0;
       double sacc = 0.0;
-      if (et < L::NT) {
-        const int mask = walsh_mask(KB, et);
-        for (int l = 0; l < Lv; ++l) sacc += (double)__ldg(a.cent + l) * ((__popc(l & mask) & 1) ? 1.0 : -1.0);
-        alpha[et] = (float)(sacc / Lv);
-      } else {
-        alpha[4] = __ldg(a.cent + Lv - 1);
+#pragma unroll
+      for (int l = 0; l < Lv; ++l) {
+        const float cl = __shfl_sync(FULL, pr.cv, l);
+        sacc += (double)cl * ((__popc(l & mask) & 1) ? 1.0 : -1.0);
       }
+      const float ctop = __shfl_sync(FULL, pr.cv, Lv - 1);
+      if (et < L::NT) alpha[et] = (float)(sacc / Lv);
+      if (et == 0) alpha[4] = ctop;
     }
     GroupSync gs{gbar, 0u};
-    gs.sync(lane);
     if (n_img > 0) {
-      make_images<KB, SI>(a, pr, n_img < 2 ? n_img : 2, imgs, imgs + L::IMG, qT, uT, up, alpha, red, et, gs);
+      // every prep / epilogue warp gets here once, before any wait that can give up: a
+      // named barrier (its first sync also publishes alpha)
+      make_images<KB, SI>(a, pr, n_img < 2 ? n_img : 2, imgs, imgs + L::IMG, qT, uT, up, alpha, red, et,
+                          [] { named_sync(1, 256); });
       if (et == 0) {
         mbar_arrive(&imgfull[0]);
         if (n_img > 1) mbar_arrive(&imgfull[1]);
@@ -497,7 +504,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
           PrepRegs pr2;
           prep_load<SI>(a, head + 1, 1, et, pr2);
           uint8_t* slot = imgs + (kn & 1) * L::IMG;
-          make_images<KB, SI>(a, pr2, 1, slot, slot, qT, uT, up, alpha, red, et, gs);
+          make_images<KB, SI>(a, pr2, 1, slot, slot, qT, uT, up, alpha, red, et, [&] { gs.sync(lane); });
           if (et == 0) mbar_arrive(&imgfull[kn & 1]);
         }
       }
@@ -509,8 +516,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       const __half* nst = reinterpret_cast<const __half*>(ring + s * L::STAGE + 4 * L::TILEB);
       const float nrm = __half2float(nst[32 * qd + lane]);
       const float gam = SI ? __half2float(nst[128 + 32 * qd + lane]) : 0.f;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      release_to_copy(&empty[s], lane);
       if (!mbar_wait(&cfull[c], cu & 1)) break;
       tc_fence_after();
       const uint32_t lrow = acc_col(c) + ((uint32_t)(32 * qd) << 16);

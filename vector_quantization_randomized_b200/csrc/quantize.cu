@@ -456,6 +456,8 @@ extern "C" int tq_quantize(const tq_params* p, const void* x, int dtype, int64_t
   a.S = p->S;
   const bool prod = p->mode == TQ_MODE_PROD;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (p->layout == TQ_LAYOUT_SLICED && !quantize_rt_supported(p, dtype))
+    return set_error(TQ_EUNSUPPORTED, "tq_quantize: the token-sliced layout needs d_pad 128 and 16-bit input");
   if (quantize_rt_supported(p, dtype)) {
     rc = launch_quantize_rt(p, x, dtype, n_vec, ld * es, codes, norms, rnorms, sm_count(), st);
     if (rc == TQ_OK) clear_error();

@@ -348,6 +348,7 @@ extern "C" int tq_search_topk(const tq_params* p, const float* q, int n_q, const
                               void* workspace, int64_t workspace_bytes, tq_stream_t stream) {
   using namespace tq;
   int rc = check_params(p, "tq_search_topk");
+  if (!rc) rc = check_planes(p, "tq_search_topk");
   if (rc) return rc;
   const int kb = index_bits(p);
   const bool prod = p->mode == TQ_MODE_PROD;

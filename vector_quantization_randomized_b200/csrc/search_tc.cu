@@ -69,6 +69,7 @@ struct SL {
 struct PrepS {
   const float* q;
   int n_q, d, kb, m;
+  int group, n_chunks;  // queries per head; 16-query chunks per head (image i = head * n_chunks + chunk)
   const float* cent;
   const int8_t* D;
   const uint16_t* S;
@@ -97,9 +98,10 @@ __global__ void __launch_bounds__(256) search_prep_kernel(const PrepS a) {
   __shared__ float alpha[5];
   __shared__ float stat[QC][4];  // sum q_rot, max |q_rot|, sum u, max |u|
   __shared__ float FG[QC][2];
-  const int chunk = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int head = blockIdx.x / a.n_chunks, chunk = blockIdx.x - head * a.n_chunks;
   const int NT = walsh_planes(a.kb), L = 1 << a.kb;
-  uint8_t* img = a.img + (int64_t)chunk * a.img_bytes;
+  uint8_t* img = a.img + (int64_t)blockIdx.x * a.img_bytes;
   if (tid < NT) {
     const int mask = walsh_mask(a.kb, tid);
     double s = 0.0;
@@ -108,8 +110,8 @@ __global__ void __launch_bounds__(256) search_prep_kernel(const PrepS a) {
   }
   if (tid == 32) alpha[4] = __ldg(a.cent + L - 1);
   for (int jq = 0; jq < 2; ++jq) {  // warp = queries 2 warp, 2 warp + 1; lane holds coordinates lane + 32 i
-    const int j = 2 * warp + jq, qi = chunk * QC + j;
-    const bool valid = qi < a.n_q;
+    const int j = 2 * warp + jq, qi = head * a.group + chunk * QC + j;
+    const bool valid = chunk * QC + j < a.group;
     float y[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -235,19 +237,23 @@ struct SArgsTC {
   const uint8_t* codes;
   const uint16_t* norms;
   const uint16_t* rnorms;
-  int64_t n_db;
+  int64_t n_db;         // keys per head (the database in search)
   int n_q, n_chunks, nsplit, tb;
+  int group;            // queries per head (search: n_q, one head)
   int64_t split_keys;   // keys per split (a multiple of 32)
-  int64_t n_units;      // nsplit * n_chunks, split-major
-  const uint8_t* img;   // [n_chunks][img_bytes]
+  int64_t n_units;      // heads * nsplit * n_chunks: head-major, then split-major
+  const uint8_t* img;   // [heads][n_chunks][img_bytes]
   int img_bytes;
-  float2* cand;         // [n_q][nsplit][KEEP] (score, id bits)
+  float2* cand;         // top-k: [n_q][nsplit][KEEP] (score, id bits)
+  float* logits;        // all scores: row head * group + query, stride ld
+  int64_t ld;
   float kappa;
 };
 
 __device__ __forceinline__ bool better(float s, int i, float s2, int i2) { return s > s2 || (s == s2 && i < i2); }
 
-template <int KB, int SI>
+// ALL: write every score to the logits rows instead of keeping a top-16 per query
+template <int KB, int SI, bool ALL>
 __global__ void __launch_bounds__(SL<KB, SI>::NTHREADS, 1) search_tc_kernel(const SArgsTC a) {
   using L = SL<KB, SI>;
   constexpr int NP = L::NP, NT = L::NT;
@@ -293,12 +299,20 @@ __global__ void __launch_bounds__(SL<KB, SI>::NTHREADS, 1) search_tc_kernel(cons
   auto acc_col = [&](int c) { return tmem + (uint32_t)(128 * c); };
   auto slot_col = [&](int s) { return tmem + 256u + (uint32_t)(64 * s); };
 
-  // the units of this CTA: u = blockIdx.x + k * gridDim.x; unit -> (split, chunk), split-major
+  // the units of this CTA: u = blockIdx.x + k * gridDim.x; unit -> (head, split, chunk);
+  // k0 = first key of the unit (global over heads), nk = its key count
+  const int64_t per_head = (int64_t)a.nsplit * a.n_chunks;
   auto unit_keys = [&](int64_t u, int64_t& k0, int64_t& nk) {
-    const int64_t split = u / a.n_chunks;
-    k0 = split * a.split_keys;
-    nk = std::min<int64_t>(a.split_keys, a.n_db - k0);
+    const int64_t head = u / per_head;
+    const int64_t split = (u - head * per_head) / a.n_chunks;
+    const int64_t kl = split * a.split_keys;
+    nk = std::min<int64_t>(a.split_keys, a.n_db - kl);
     if (nk < 0) nk = 0;
+    k0 = head * a.n_db + kl;
+  };
+  auto unit_image = [&](int64_t u) {  // image index head * n_chunks + chunk
+    const int64_t head = u / per_head;
+    return head * a.n_chunks + (u - head * per_head) % a.n_chunks;
   };
 
   if (warp == 0) {
@@ -334,7 +348,7 @@ __global__ void __launch_bounds__(SL<KB, SI>::NTHREADS, 1) search_tc_kernel(cons
     uint32_t bph = 0, dph = 0;
     bool ok = true;
     for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
-      const int64_t chunk = u % a.n_chunks;
+      const int64_t chunk = unit_image(u);
       int64_t k0, nk;
       unit_keys(u, k0, nk);
       if (u != blockIdx.x) {  // every MMA reading the old image has completed
@@ -403,8 +417,7 @@ __global__ void __launch_bounds__(SL<KB, SI>::NTHREADS, 1) search_tc_kernel(cons
           pw[p][0] = *reinterpret_cast<const uint4*>(src + p * 1024);
           pw[p][1] = *reinterpret_cast<const uint4*>(src + p * 1024 + 16);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
+        release_to_copy(&empty[st], lane);  // the stage is refilled once all 8 warps release it
 #pragma unroll
         for (int P = 0; P < NP; ++P, ++gp) {
           uint32_t wv[8];
@@ -465,10 +478,11 @@ __global__ void __launch_bounds__(SL<KB, SI>::NTHREADS, 1) search_tc_kernel(cons
     int64_t gi = 0;
     bool ok = true;
     for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
-      const int64_t chunk = u % a.n_chunks, split = u / a.n_chunks;
+      const int64_t img_i = unit_image(u), head = u / per_head;
+      const int64_t chunk = img_i - head * a.n_chunks, split = (u - head * per_head) / a.n_chunks;
       int64_t k0, nk;
       unit_keys(u, k0, nk);
-      const float4* scal = reinterpret_cast<const float4*>(a.img + chunk * a.img_bytes) + 8 * hq;
+      const float4* scal = reinterpret_cast<const float4*>(a.img + img_i * a.img_bytes) + 8 * hq;
       // per query: entry `lane` (< 16) of the sorted list; the 16th entry is the threshold
       float ls[8];
       int li[8];
@@ -520,6 +534,15 @@ __global__ void __launch_bounds__(SL<KB, SI>::NTHREADS, 1) search_tc_kernel(cons
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&accfree[c]);
+        if constexpr (ALL) {
+          const int64_t kl = key - head * a.n_db;  // key within the head
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int qj = (int)chunk * QC + 8 * hq + j;
+            if (kvalid && qj < a.group) a.logits[(head * a.group + qj) * a.ld + kl] = nrm * lv[j];
+          }
+          continue;
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float l = lv[j];
@@ -553,6 +576,7 @@ __global__ void __launch_bounds__(SL<KB, SI>::NTHREADS, 1) search_tc_kernel(cons
         }
       }
       if (!ok) break;
+      if constexpr (ALL) continue;
       // unit end: the four quadrant lists of each query -> one top-16 per (query, split)
       if (lane < KEEP) {
 #pragma unroll
@@ -616,10 +640,10 @@ __global__ void __launch_bounds__(SL<KB, SI>::NTHREADS, 1) search_tc_kernel(cons
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-template <int KB, int SI>
+template <int KB, int SI, bool ALL>
 int launch_stc(const SArgsTC& a, int sm, cudaStream_t st) {
   using L = SL<KB, SI>;
-  auto kern = search_tc_kernel<KB, SI>;
+  auto kern = search_tc_kernel<KB, SI, ALL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_search_topk: %s", cudaGetErrorString(e));
   cudaLaunchConfig_t cfg = {};
@@ -637,12 +661,78 @@ int launch_stc(const SArgsTC& a, int sm, cudaStream_t st) {
   return TQ_OK;
 }
 
+template <bool ALL>
+int dispatch_stc(int kb, int si, const SArgsTC& a, int sm, cudaStream_t st) {
+  if (si) {
+    switch (kb) {
+      case 1: return launch_stc<1, 1, ALL>(a, sm, st);
+      case 2: return launch_stc<2, 1, ALL>(a, sm, st);
+      default: return launch_stc<3, 1, ALL>(a, sm, st);
+    }
+  }
+  switch (kb) {
+    case 1: return launch_stc<1, 0, ALL>(a, sm, st);
+    case 2: return launch_stc<2, 0, ALL>(a, sm, st);
+    default: return launch_stc<3, 0, ALL>(a, sm, st);
+  }
+}
+
 int image_bytes(int kb, int si) {
   const int nt = walsh_planes(kb);
   return 256 + (nt + si) * 16 * 1024;
 }
 
 int splits_for(int64_t n_db) { return (int)std::max<int64_t>(1, std::min<int64_t>(MAX_SPLITS, (n_db + 16383) / 16384)); }
+
+// The images of every (head, 16-query chunk), then the scan.
+int run_stc(const tq_params* p, int kb, const float* q, int n_heads, int group, const void* codes,
+            const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys, void* workspace, bool all, float* logits,
+            int64_t ld, float2** cand, int* nsplit, cudaStream_t st) {
+  const int m = p->mode == TQ_MODE_PROD ? p->m : 0;
+  const int si = m > 0 ? 1 : 0;
+  const int n_chunks = (group + QC - 1) / QC;
+  const int ib = image_bytes(kb, si);
+  PrepS pa;
+  pa.q = q;
+  pa.n_q = n_heads * group;
+  pa.d = p->d;
+  pa.kb = kb;
+  pa.m = m;
+  pa.group = group;
+  pa.n_chunks = n_chunks;
+  pa.cent = p->centroids;
+  pa.D = p->signs_D;
+  pa.S = p->S;
+  pa.img = static_cast<uint8_t*>(workspace);
+  pa.img_bytes = ib;
+  pa.np = walsh_planes(kb) + si;
+  search_prep_kernel<<<n_heads * n_chunks, 256, 0, st>>>(pa);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tensor-core scan: prep launch failed: %s", cudaGetErrorString(e));
+  SArgsTC a;
+  a.codes = static_cast<const uint8_t*>(codes);
+  a.norms = norms;
+  a.rnorms = rnorms;
+  a.n_db = n_keys;
+  a.n_q = n_heads * group;
+  a.n_chunks = n_chunks;
+  a.group = group;
+  a.nsplit = all ? (int)std::max<int64_t>(1, std::min<int64_t>(MAX_SPLITS, (n_keys + 4095) / 4096)) : splits_for(n_keys);
+  a.tb = tqd::tile_bytes(256, kb, m);
+  a.split_keys = ((n_keys + a.nsplit - 1) / a.nsplit + TK - 1) / TK * TK;
+  a.n_units = (int64_t)n_heads * a.nsplit * n_chunks;
+  a.img = pa.img;
+  a.img_bytes = ib;
+  const int64_t img_total = ((int64_t)n_heads * n_chunks * ib + 255) & ~(int64_t)255;
+  a.cand = all ? nullptr : reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + img_total);
+  a.logits = logits;
+  a.ld = ld;
+  a.kappa = (float)(std::sqrt(M_PI / 2.0) / (m > 0 ? m : 1));
+  if (cand) *cand = a.cand;
+  if (nsplit) *nsplit = a.nsplit;
+  const int sm = tq::sm_count();
+  return all ? dispatch_stc<true>(kb, si, a, sm, st) : dispatch_stc<false>(kb, si, a, sm, st);
+}
 
 }  // namespace
 
@@ -661,56 +751,18 @@ int64_t search_tc_workspace(int kb, int m, int n_q, int64_t n_db) {
 int launch_search_tc(const tq_params* p, int kb, const float* q, int n_q, const void* codes, const uint16_t* norms,
                      const uint16_t* rnorms, int64_t n_db, void* workspace, float2** cand, int* nsplit,
                      cudaStream_t st) {
-  const int m = p->mode == TQ_MODE_PROD ? p->m : 0;
-  const int si = m > 0 ? 1 : 0;
-  const int n_chunks = (n_q + QC - 1) / QC;
-  const int ib = image_bytes(kb, si);
-  PrepS pa;
-  pa.q = q;
-  pa.n_q = n_q;
-  pa.d = p->d;
-  pa.kb = kb;
-  pa.m = m;
-  pa.cent = p->centroids;
-  pa.D = p->signs_D;
-  pa.S = p->S;
-  pa.img = static_cast<uint8_t*>(workspace);
-  pa.img_bytes = ib;
-  pa.np = walsh_planes(kb) + si;
-  search_prep_kernel<<<n_chunks, 256, 0, st>>>(pa);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return set_error(TQ_ECUDA, "tq_search_topk: prep launch failed: %s", cudaGetErrorString(e));
-  SArgsTC a;
-  a.codes = static_cast<const uint8_t*>(codes);
-  a.norms = norms;
-  a.rnorms = rnorms;
-  a.n_db = n_db;
-  a.n_q = n_q;
-  a.n_chunks = n_chunks;
-  a.nsplit = splits_for(n_db);
-  a.tb = tqd::tile_bytes(256, kb, m);
-  a.split_keys = ((n_db + a.nsplit - 1) / a.nsplit + TK - 1) / TK * TK;
-  a.n_units = (int64_t)a.nsplit * n_chunks;
-  a.img = pa.img;
-  a.img_bytes = ib;
-  const int64_t img_total = ((int64_t)n_chunks * ib + 255) & ~(int64_t)255;
-  a.cand = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + img_total);
-  a.kappa = (float)(std::sqrt(M_PI / 2.0) / (m > 0 ? m : 1));
-  *cand = a.cand;
-  *nsplit = a.nsplit;
-  const int sm = sm_count();
-  if (si) {
-    switch (kb) {
-      case 1: return launch_stc<1, 1>(a, sm, st);
-      case 2: return launch_stc<2, 1>(a, sm, st);
-      default: return launch_stc<3, 1>(a, sm, st);
-    }
-  }
-  switch (kb) {
-    case 1: return launch_stc<1, 0>(a, sm, st);
-    case 2: return launch_stc<2, 0>(a, sm, st);
-    default: return launch_stc<3, 0>(a, sm, st);
-  }
+  return run_stc(p, kb, q, 1, n_q, codes, norms, rnorms, n_db, workspace, false, nullptr, 0, cand, nsplit, st);
+}
+
+// Logits on the same scan (d_pad 256): bytes of the query images for n_q = n_heads * group queries
+// (an upper bound over every split of n_q into heads and groups).
+int64_t logits_stc_workspace(int kb, int m, int n_q) { return (int64_t)n_q * image_bytes(kb, m > 0 ? 1 : 0) + 256; }
+
+int launch_logits_stc(const tq_params* p, int kb, const float* q, int n_heads, int group, const void* codes,
+                      const uint16_t* norms, const uint16_t* rnorms, int64_t n_keys, float* logits, int64_t ld,
+                      void* workspace, cudaStream_t st) {
+  return run_stc(p, kb, q, n_heads, group, codes, norms, rnorms, n_keys, workspace, true, logits, ld, nullptr,
+                 nullptr, st);
 }
 
 }  // namespace tq

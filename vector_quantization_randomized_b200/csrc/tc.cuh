@@ -69,6 +69,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
 }
+
+// Release a shared-memory buffer that a bulk copy (async proxy) will refill, after
+// this warp read it with ordinary loads (generic proxy): the proxy fence orders
+// those reads before the copy's writes.  A plain arrive let the next copy land
+// under reads still in flight (seen as corrupted 32-key tiles in the scans).
+__device__ __forceinline__ void release_to_copy(uint64_t* bar, int lane) {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
 // arrive and add `bytes` to the phase's expected transaction count
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)

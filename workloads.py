@@ -12,6 +12,13 @@ Data law for keys/values (the pages give none; this is the stated workload):
 Queries are N(0, 1).  Each (sequence, head) has its own generator stream
 derived from (seed, sequence, head).
 
+Projection inputs (the fused projection + quantize path): a layer input
+x[t, k] = z[t, k] * rho_t (z ~ N(0, 1), rho_t = exp(N(0, 0.3^2))) and a
+weight w[o, k] = z'[o, k] * sigma_o * (20 if o is an outlier row) / sqrt(hidden)
+with 4 outlier output rows per head, both rounded to bf16, so that the
+projected vectors follow the key law above (per-channel lognormal scales,
+4 outlier channels, per-token norm multiplier).
+
 Search set: x ~ N(0, Q diag(i^-0.8) Q^T), i = 1..d, Q a seeded Haar-random
 orthogonal matrix (QR of a Gaussian matrix with the sign of R's diagonal
 folded into Q), rows normalised to unit length.  It stands in for the GloVe
@@ -59,6 +66,19 @@ def kv_block(n_seq, n_heads, n_tokens, d, seed, token_scale=True, bf16=True, seq
             v = head_vectors(n_tokens, d, seed, s, h, token_scale)
             out[i, h] = to_bf16(v) if bf16 else v
     return out
+
+
+def projection_inputs(n_tok, hidden, n_heads, seed, d=128):
+    """(x [n_tok, hidden], w [n_heads * d, hidden]): bf16-valued float32 arrays."""
+    r = _rng(seed, 21, 21)
+    rho = np.exp(r.normal(0.0, 0.3, size=n_tok)).astype(np.float32)
+    x = to_bf16(r.standard_normal(size=(n_tok, hidden), dtype=np.float32) * rho[:, None])
+    sig = np.exp(r.normal(0.0, 0.5, size=n_heads * d))
+    for h in range(n_heads):
+        sig[h * d + r.permutation(d)[:4]] *= 20.0
+    w = r.standard_normal(size=(n_heads * d, hidden), dtype=np.float32)
+    w = to_bf16(w * (sig / np.sqrt(hidden)).astype(np.float32)[:, None])
+    return x, w
 
 
 def queries(n, d, seed=SEED_QUERIES):
