@@ -550,6 +550,21 @@ def measure_decode(torch, tq, wl, steps, warmup, peak, sparse=True):
     res = {"us": round(ms * 1000, 2), "tokens_per_s": n / (ms / 1e3), "metric_bytes": mbytes, "gbs": round(gbs, 1),
            "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4), "frac_measured": round(gbs / peak, 4),
            "workload": "decode-64x8x16384-Kprod3-Vmse3-hq32", "inputs": "> L2 (856 MB of codes)"}
+    # the same values in the token-sliced layout: the tensor-memory decode
+    vps = tq.Params(d, 3, tq.TQ_MODE_MSE, 0, wl.SEED_PARAMS + 1, layout=tq.TQ_LAYOUT_SLICED)
+    x = gpu_kv(torch, B, Hkv, T, d, wl.SEED_VALUES)
+    vcs = torch.empty(vps.code_bytes(n), dtype=torch.uint8, device="cuda")
+    vns = torch.empty(n, dtype=torch.int16, device="cuda")
+    tq.tq_quantize(vps, x, vcs, vns)
+    torch.cuda.synchronize()
+    del x
+    ms_t = timed(lambda: tq.tq_decode_attn(kp, vps, q, Hkv, bufs["k"][0], bufs["k"][1], bufs["k"][2], vcs, vns, sl, T,
+                                           out, ws))
+    gbs_t = mbytes / (ms_t / 1e3) / 1e9
+    res["tensor_memory"] = {"us": round(ms_t * 1000, 2), "tokens_per_s": n / (ms_t / 1e3), "gbs": round(gbs_t, 1),
+                            "frac_measured": round(gbs_t / peak, 4),
+                            "how": "values in the token-sliced layout (tq_params.layout = 1): decode_tc_kernel"}
+    del vcs, vns
     if sparse:
         sp = {}
         for eps in (1e-4, 1e-3):

@@ -7,20 +7,22 @@ import torch
 
 import vector_quantization_randomized_b200 as tq
 import workloads as wl
-from oracle import estimate
+from oracle import codec, estimate
 from gpu_util import make_pair, oracle_codes
 
 pytestmark = pytest.mark.gpu
 
 
-def _check(B, Hkv, Hq, T, seq_lens, kbits=3, vbits=3, d=128, scale=0.0):
+def _check(B, Hkv, Hq, T, seq_lens, kbits=3, vbits=3, d=128, scale=0.0, layout=tq.TQ_LAYOUT_PLANES):
     kp, kop = make_pair(d, kbits, tq.TQ_MODE_PROD, seed=42)
-    vp, vop = make_pair(d, vbits, tq.TQ_MODE_MSE, seed=43)
+    vp, vop = make_pair(d, vbits, tq.TQ_MODE_MSE, seed=43, layout=layout)
     K = wl.kv_block(B, Hkv, T, d, seed=wl.SEED_KEYS).reshape(-1, d)
     V = wl.kv_block(B, Hkv, T, d, seed=wl.SEED_VALUES).reshape(-1, d)
     q = wl.queries(B * Hq, d, seed=wl.SEED_QUERIES).reshape(B, Hq, d)
     kc, kn, krn, ke = oracle_codes(kop, K)
     vc, vn, _, ve = oracle_codes(vop, V)
+    if layout == tq.TQ_LAYOUT_SLICED:
+        vc = codec.pack_sliced(ve["idx"], vop.kb)  # the value cache in the token-sliced layout
     ref = estimate.decode_attention(q, kop.D, kop.S, ke["idx"], ke["signs"], kn, krn, kop.c, kop.m,
                                     vop.D, ve["idx"], vn, vop.c, d, seq_lens, Hq, Hkv, T, scale=scale)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
@@ -60,3 +62,48 @@ def test_decode_bit_widths(kbits, vbits):
 
 def test_decode_explicit_scale():
     _check(B=1, Hkv=1, Hq=4, T=256, seq_lens=[256], scale=0.02)
+
+
+# token-sliced values: the tensor-memory decode (keys with m = 128 and at most 3 index bits,
+# values with at most 3, at most 4 query heads per KV head, max_tokens a multiple of 32)
+SL = tq.TQ_LAYOUT_SLICED
+
+
+def test_sliced_gqa4_segments_and_ragged_lengths():
+    # 1120 tokens: two 1024-token segments, the second ragged; a 517-token and a 1-token sequence
+    _check(B=3, Hkv=2, Hq=8, T=1120, seq_lens=[1120, 517, 1], layout=SL)
+
+
+def test_sliced_empty_sequence_and_single_item():
+    _check(B=2, Hkv=1, Hq=4, T=96, seq_lens=[0, 96], layout=SL)
+
+
+@pytest.mark.parametrize("Hq", [1, 2])
+def test_sliced_group_sizes(Hq):
+    _check(B=2, Hkv=1, Hq=Hq, T=640, seq_lens=[640, 333], layout=SL)
+
+
+@pytest.mark.parametrize("kbits,vbits", [(2, 1), (3, 2), (4, 3)])
+def test_sliced_bit_widths(kbits, vbits):
+    _check(B=1, Hkv=2, Hq=4, T=704, seq_lens=[650], kbits=kbits, vbits=vbits, layout=SL)
+
+
+def test_sliced_many_units_per_cta():
+    # 2 x 8 KV heads x 4096 tokens (64 segments over <= 148 CTAs, several per CTA, heads changing
+    # inside a CTA's range), 32 query heads
+    _check(B=2, Hkv=8, Hq=32, T=4096, seq_lens=[4096, 3000], layout=SL)
+
+
+def test_sliced_explicit_scale_matches_planes():
+    a, _ = _check(B=1, Hkv=1, Hq=4, T=256, seq_lens=[256], scale=0.02, layout=SL)
+    b, _ = _check(B=1, Hkv=1, Hq=4, T=256, seq_lens=[256], scale=0.02)
+    # both are within the oracle's tolerance; they agree row by row to the sum of the two
+    for h in range(4):
+        assert np.linalg.norm(a[0, h] - b[0, h]) <= 4e-3 * np.linalg.norm(b[0, h])
+
+
+def test_sliced_unsupported_shapes():
+    with pytest.raises(tq.TQError):   # five query heads per KV head
+        _check(B=1, Hkv=1, Hq=5, T=128, seq_lens=[128], layout=SL)
+    with pytest.raises(tq.TQError):   # max_tokens not a multiple of 32
+        _check(B=1, Hkv=1, Hq=4, T=100, seq_lens=[100], layout=SL)

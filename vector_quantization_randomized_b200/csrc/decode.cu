@@ -738,3 +738,29 @@ extern "C" int tq_decode_attn_merge(const tq_params* vp, const float* partials, 
   clear_error();
   return TQ_OK;
 }
+
+namespace tq {
+// The log-sum-exp combine (and inverse rotation) over partial rows, for the
+// tensor-memory decode (decode_tc.cu).
+int launch_combine(const float* part, int64_t row_stride, int64_t chunk_stride, const int8_t* vD,
+                   const int32_t* seq_lens, float* out, int nch, int d, int dp, int hq, int64_t rows,
+                   cudaStream_t st) {
+  if (rows > 0x7fffffff || nch > 2048) return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: combine shape too large");
+  CArgs ca;
+  ca.part = part;
+  ca.row_stride = row_stride;
+  ca.chunk_stride = chunk_stride;
+  ca.vD = vD;
+  ca.seq_lens = seq_lens;
+  ca.out = out;
+  ca.part_out = nullptr;
+  ca.nch = nch;
+  ca.d = d;
+  ca.dp = dp;
+  ca.hq = hq;
+  combine_kernel<<<(unsigned)rows, 128, 0, st>>>(ca);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(TQ_ECUDA, "tq_decode_attn: combine launch failed: %s", cudaGetErrorString(e));
+  return TQ_OK;
+}
+}  // namespace tq

@@ -810,12 +810,14 @@ int dispatch_rt(int kb, const CUtensorMap& map, const CUtensorMap& map_w, const 
 
 namespace tq {
 
-// Whether the tensor-core rotation kernel handles this call: d_pad 128, 16-bit input,
-// m 0 or 128, index bits up to 4 (3 in product mode).
+// Whether tq_quantize runs on the tensor-core rotation kernel: d_pad 128, 16-bit input, MSE
+// codes (either layout).  Product codes stay on the register kernel (quantize_tc.cu), which is
+// faster there (72 against 101 us for 2^18 keys at b = 3): with the sign read-back added, this
+// kernel issues about 108 warp-instructions per vector at an IPC near 1.  The product form of
+// this kernel serves the fused projection path.
 bool quantize_rt_supported(const tq_params* p, int dtype) {
   const int kb = index_bits(p);
-  return p->d_pad == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && kb >= 1 && kb <= 4 &&
-         (p->mode == TQ_MODE_MSE || p->m == 128);
+  return p->d_pad == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && kb >= 1 && kb <= 4 && p->mode == TQ_MODE_MSE;
 }
 
 int launch_quantize_rt(const tq_params* p, const void* x, int dtype, int64_t n_vec, int64_t ld_bytes, void* codes,
