@@ -51,6 +51,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-kernels", action="store_true")
+    ap.add_argument("--decode-batch", type=int, default=64, help="sequences of the decode workload (64)")
     ap.add_argument("--no-configs", action="store_true")
     return ap.parse_args()
 
@@ -508,11 +509,11 @@ def gpu_kv(torch, n_seq, n_heads, n_tokens, d, seed):
     return out.reshape(-1, d)
 
 
-def measure_decode(torch, tq, wl, steps, warmup, peak, sparse=True):
-    """Decode attention, 64 sequences x 8 KV heads x 16384 tokens, d 128, 32 query heads:
+def measure_decode(torch, tq, wl, steps, warmup, peak, sparse=True, batch=64):
+    """Decode attention, `batch` (64) sequences x 8 KV heads x 16384 tokens, d 128, 32 query heads:
     K product code b = 3, V MSE code b = 3 (inputs drawn on the GPU, then quantized)."""
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    B, Hkv, T, d, Hq = 64, 8, 16384, 128, 32
+    B, Hkv, T, d, Hq = batch, 8, 16384, 128, 32
     kp = tq.Params(d, 3, tq.TQ_MODE_PROD, 128, wl.SEED_PARAMS)
     vp = tq.Params(d, 3, tq.TQ_MODE_MSE, 0, wl.SEED_PARAMS + 1)
     n = B * Hkv * T
@@ -549,7 +550,7 @@ def measure_decode(torch, tq, wl, steps, warmup, peak, sparse=True):
     gbs = mbytes / (ms / 1e3) / 1e9
     res = {"us": round(ms * 1000, 2), "tokens_per_s": n / (ms / 1e3), "metric_bytes": mbytes, "gbs": round(gbs, 1),
            "frac_8tbs": round(gbs / HBM_NOMINAL_GBS, 4), "frac_measured": round(gbs / peak, 4),
-           "workload": "decode-64x8x16384-Kprod3-Vmse3-hq32", "inputs": "> L2 (856 MB of codes)"}
+           "workload": f"decode-{B}x8x16384-Kprod3-Vmse3-hq32", "inputs": f"> L2 ({mbytes / 1e6:.0f} MB of codes)"}
     # the same values in the token-sliced layout: the tensor-memory decode
     vps = tq.Params(d, 3, tq.TQ_MODE_MSE, 0, wl.SEED_PARAMS + 1, layout=tq.TQ_LAYOUT_SLICED)
     x = gpu_kv(torch, B, Hkv, T, d, wl.SEED_VALUES)
@@ -649,8 +650,8 @@ def run_secondary(args, world, rank, local, torch, tq, wl):
     peak, peak_kind = measured_peaks()
     ev = lambda: torch.cuda.Event(enable_timing=True)
     if args.workload == "decode":
-        r = measure_decode(torch, tq, wl, args.steps, args.warmup, peak)
-        n = 64 * 8 * 16384
+        r = measure_decode(torch, tq, wl, args.steps, args.warmup, peak, batch=args.decode_batch)
+        n = args.decode_batch * 8 * 16384
         line = {"metric": "decode attention tokens/s", "value": r["tokens_per_s"], "unit": "tokens/s",
                 "ms_per_step": r["us"] / 1000, "config": {"workload": r["workload"]}, "decode": r}
     elif args.workload == "quantize":

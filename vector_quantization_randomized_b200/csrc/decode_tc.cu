@@ -17,8 +17,9 @@
 //    in tensor memory with lane = coordinate: the token-sliced layout stores, per
 //    tile of 32 tokens, one 32-bit word per coordinate, and (word & 0x01010101 << c)
 //    is the K-major byte row of 4 tokens; B = 4 base-256 digits of the weights
-//    2 alpha_T w 2^F (23 bits) pre-shifted by 7 - (token class), one digit image
-//    per Walsh plane, all planes accumulated into one 16-column accumulator.
+//    w 2^F (23 bits) pre-shifted by 7 - (token class), one image per item, each
+//    Walsh plane into a 16-column accumulator of its own (combined with 2 alpha_T
+//    in the epilogue).
 // Integer sums stay below 2^22, so their conversion to fp32 is exact.
 //
 // Work: pairs (sequence, KV head) x segments of 8 items of 128 tokens; each
@@ -31,9 +32,11 @@
 //   warp 2       MMA issue for the value sum (per Walsh plane);
 //   warps 3-6    key bits -> tensor-memory plane slots (lane quadrant = 32 tokens);
 //   warps 7-10   value words -> tensor-memory plane slots (lane quadrant = 32 coordinates);
-//   warps 11-14  softmax: logits from the accumulators, the running maximum, the
-//                weights, their digit images for the value MMAs;
-//   warps 15-18  value epilogue: accumulators -> rescaled fp32 sums per coordinate.
+//   warps 11-18  softmax, two groups of 4 taking alternate items, each with a running
+//                maximum, sum and weight sum of its own: logits from the
+//                accumulators, the weights, their digit image for the value MMAs;
+//   warps 19-22  value epilogue: accumulators -> rescaled fp32 sums per coordinate,
+//                one set per softmax group; a unit leaves one partial per group.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -53,9 +56,9 @@ constexpr int TK = 128;       // tokens per item
 constexpr int SEG = 8;        // items per unit (segment of 1024 tokens)
 constexpr int NST = 8;        // code stages
 constexpr int NSK = 4;        // key plane slots (32 columns each)
-constexpr int NSV = 8;        // value plane slots (32 columns each)
+constexpr int NSV = 6;        // value plane slots (32 columns each)
 constexpr int NBK = 2;        // logits accumulator sets (32 columns: 16 centroid + 16 sign)
-constexpr int NBV = 2;        // value accumulator sets (16 columns)
+constexpr int NBV = 2;        // value accumulator sets (per Walsh plane 16 columns)
 
 template <int KB, int VKB>
 struct DL {
@@ -71,16 +74,16 @@ struct DL {
   static constexpr int OFF_KN = 4 * KTILE;            // key norms, residual norms, value norms (256 B each)
   static constexpr int OFF_V = OFF_KN + 768;
   static constexpr int STAGE = OFF_V + 4 * VTILE;
-  static constexpr int BVB = NTV * 2048;              // value digit images of an item (NTV x 16 rows x 128 B)
+  static constexpr int BVB = 2048;                    // value weight digits of an item (16 rows x 128 B)
   static constexpr int OFF_IMG = 1024;
   static constexpr int OFF_BV = OFF_IMG + 2 * IMG;
   static constexpr int OFF_ST = OFF_BV + 2 * BVB;     // stats ring: [2][16 floats]
-  static constexpr int OFF_X = OFF_ST + 2 * 64;       // softmax exchange: 2 x [4 warps][8] item maxima, [4][8] sums
-  static constexpr int OFF_RING = (OFF_X + 384 + 127) / 128 * 128;
+  static constexpr int OFF_X = OFF_ST + 2 * 64;       // per softmax group: 2 x [4 warps][8] item maxima, [4][8] sums
+  static constexpr int OFF_RING = (OFF_X + 2 * 384 + 127) / 128 * 128;
   static constexpr int SMEM = OFF_RING + NST * STAGE;
-  static constexpr int NTHREADS = 19 * 32;
+  static constexpr int NTHREADS = 23 * 32;
   // tensor-memory columns
-  static constexpr int C_KACC = 0, C_VACC = 64, C_KS = 96, C_VS = 224;
+  static constexpr int C_KACC = 0, C_VACC = 64, C_KS = 192, C_VS = 320;
   static_assert(C_VS + NSV * 32 <= 512, "tensor memory");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -118,6 +121,17 @@ struct DPrepArgs {
   uint8_t* img;
   int img_bytes, ntk, img_s;
 };
+
+// warp maximum of a float (redux.sync; -inf and finite values only)
+__device__ __forceinline__ float warp_max_f32(float v) {
+  float r;
+  asm volatile("redux.sync.max.NaN.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+// int32 |x| < 2^22 to fp32, exactly, on the FP pipe (1.5 * 2^23 + x has x in its mantissa)
+__device__ __forceinline__ float i2f_exact(uint32_t x) {
+  return __uint_as_float(x + 0x4B400000u) - 12582912.f;
+}
 
 __device__ __forceinline__ int exponent_of(float x) {
   const uint32_t b = __float_as_uint(x) & 0x7FFFFFFFu;
@@ -312,8 +326,8 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
   uint64_t* imf = str_ + 2;                            // [2] query image loaded (1 + tx)
   uint64_t* imr = imf + 2;                             // [2] query image no longer read by the MMAs (1)
   uint64_t* imq = imr + 2;                             // [2] query image scalars copied by the softmax (4)
-  uint64_t* sbar = imq + 2;                            // softmax warps' barrier (4)
-  uint32_t* tbase = reinterpret_cast<uint32_t*>(sbar + 1);
+  uint64_t* sbar = imq + 2;                            // [2] barrier of each softmax group (4)
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(sbar + 2);
   uint8_t* imgs = smem + L::OFF_IMG;
   uint8_t* bv = smem + L::OFF_BV;
   float* stats = reinterpret_cast<float*>(smem + L::OFF_ST);  // [2][16]: alpha[4], 2^-(F_q+7)[4], sum w[4], last
@@ -353,9 +367,10 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
       mbar_init(&str_[k], 4);
       mbar_init(&imf[k], 1);
       mbar_init(&imr[k], 1);
-      mbar_init(&imq[k], 4);
+      mbar_init(&imq[k], 8);
     }
-    mbar_init(sbar, 4);
+    mbar_init(&sbar[0], 4);
+    mbar_init(&sbar[1], 4);
   }
   fence_async_smem();
   if (warp == 0) tmem_alloc(tbase, 512);
@@ -479,7 +494,7 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
           ok = false;
           break;
         }
-        const uint32_t d = tmem + L::C_VACC + 16u * c;
+        const uint32_t d = tmem + L::C_VACC + 64u * c;
         const uint32_t sbv = smem_u32(bv + sb * L::BVB);
 #pragma unroll 1
         for (int T = 0; T < NTV; ++T, ++gp) {
@@ -490,11 +505,11 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
           }
           __syncwarp();
           tc_fence_after();
-          const uint64_t bd = smem_desc(sbv + 2048 * T, 256, 128);
+          const uint64_t bd = smem_desc(sbv, 256, 128);
           const uint32_t acol = tmem + L::C_VS + 32u * s;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)  // K = 32 tokens: 2 K chunks of the digit image
-            umma_i8_ts_elect(d, acol + 8u * ks, bd + (uint64_t)(32 * ks), idesc, (T == 0 && ks == 0) ? 0u : 1u);
+            umma_i8_ts_elect(d + 16u * T, acol + 8u * ks, bd + (uint64_t)(32 * ks), idesc, ks == 0 ? 0u : 1u);
           umma_commit_elect(&vsr[s]);
         }
         if (!ok) break;
@@ -619,24 +634,25 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
         }
       }
     }
-  } else if (warp < 15) {
-    // ---------------- softmax (lane = token 32 qd + lane) ----------------
-    const int sw = warp - 11;  // 0..3
+  } else if (warp < 19) {
+    // ---------------- softmax (lane = token 32 qd + lane), group sg takes the items of parity sg ----------------
+    const int sg = (warp - 11) >> 2, sw = (warp - 11) & 3;
     const int qd = warp & 3;
     const int tk = 32 * qd + lane;
-    const int cls = lane & 7;  // bit class of the token inside its 32-token tile
+    const int cls = lane & 7;                           // bit class of the token inside its 32-token tile
     const int kpos = 32 * qd + 4 * cls + (lane >> 3);  // its K byte in the value MMAs
-    GroupSync gs{sbar, 0u};
+    const int sh = 7 - cls;
+    GroupSync gs{&sbar[sg], 0u};
+    float* xg = xch + sg * 96;  // this group's exchange: [2][4 warps][8] item maxima, then [4][8] sums
     int64_t gi = 0, kimg = 0, prev_pair = -1;
     float4 qsc[4];
-    const float va[4] = {a.vco[0], a.vco[1], a.vco[2], a.vco[3]};
-    const float vamax = a.vco[5];
     bool ok = true;
     for (int64_t u = u0; u < u1 && ok; ++u) {
       int64_t pair;
       int seg, n_items, len;
       walk.unit(u, pair, seg, n_items, len);
       const int b = (int)(pair / a.hkv), g = (int)(pair - (int64_t)b * a.hkv);
+      const int sub = (int)((sg ^ gi) & 1);  // this group's items in the unit: it = sub, sub + 2, ...
       float mrun[4], lw[4], ww[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -655,6 +671,7 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
         ++kimg;
       }
       for (int it = 0; it < n_items && ok; ++it, ++gi) {
+        if ((gi & 1) != sg) continue;
         const int st = (int)(gi % NST), c = (int)(gi % NBK), sb = (int)(gi & 1);
         const int t0 = (seg * SEG + it) * TK;
         const bool valid = t0 + tk < len;
@@ -690,29 +707,27 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
           const float cen = fmaf((float)(int)C[4 * q + 3], 16777216.f,
                                  fmaf((float)(int)C[4 * q + 2], 65536.f,
                                       fmaf((float)(int)C[4 * q + 1], 256.f, (float)(int)C[4 * q])));
-          const float sg = fmaf((float)(int)Z[4 * q + 3], 16777216.f,
-                                fmaf((float)(int)Z[4 * q + 2], 65536.f,
-                                     fmaf((float)(int)Z[4 * q + 1], 256.f, (float)(int)Z[4 * q])));
-          const float l = fmaf(gam * a.kappa, fmaf(sg, sc.z, -sc.w), fmaf(cen, sc.x, -sc.y));
+          const float sg2 = fmaf((float)(int)Z[4 * q + 3], 16777216.f,
+                                 fmaf((float)(int)Z[4 * q + 2], 65536.f,
+                                      fmaf((float)(int)Z[4 * q + 1], 256.f, (float)(int)Z[4 * q])));
+          const float l = fmaf(gam * a.kappa, fmaf(sg2, sc.z, -sc.w), fmaf(cen, sc.x, -sc.y));
           s[q] = (valid && q < a.group) ? kn * l * a.sl2 : -INFINITY;
-          xm[q] = warp_max(s[q]);
+          xm[q] = warp_max_f32(s[q]);
         }
-        xm[4] = warp_max(valid ? vn : 0.f);
-        // item maxima over the 4 softmax warps
-        float* xb = xch + (gi & 1) * 32;  // two buffers: a fast warp may reach the next item
+        xm[4] = warp_max_f32(valid ? vn : 0.f);
+        // item maxima over the group's 4 warps
+        float* xb = xg + ((gi >> 1) & 1) * 32;  // two buffers: a fast warp may reach the group's next item
         if (lane == 0) {
 #pragma unroll
           for (int q = 0; q < 5; ++q) xb[8 * sw + q] = xm[q];
         }
         gs.sync(lane);
-        float mnew[4], alf[4];
         float vmax = 0.f;
 #pragma unroll
         for (int k = 0; k < 4; ++k) vmax = fmaxf(vmax, xb[8 * k + 4]);
-        // per query: weights 2 alpha_T w 2^F_q below 2^23, F_q from the bound
-        // w <= 2^(item max - running max) * (item's largest value norm)
+        // per query: weights w 2^F_q below 2^23, F_q from the bound w <= 2^(item max - running max) * max n_v
+        float mnew[4], alf[4], fq[4];
         int Fq[4];
-        float fq[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float mi = -INFINITY;
@@ -720,9 +735,9 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
           for (int k = 0; k < 4; ++k) mi = fmaxf(mi, xb[8 * k + q]);
           mnew[q] = fmaxf(mrun[q], mi);
           alf[q] = mrun[q] == -INFINITY ? 0.f : exp2f(mrun[q] - mnew[q]);
-          const float mc = mi == -INFINITY ? 0.f : 2.f * vamax * vmax * exp2f(mi - mnew[q]);
+          const float mc = mi == -INFINITY ? 0.f : vmax * exp2f(mi - mnew[q]);
           Fq[q] = mc > 0.f ? 23 - exponent_of(mc) : 0;
-          fq[q] = 2.f * pow2(Fq[q]);
+          fq[q] = pow2(Fq[q]);
         }
         float wq[4];
 #pragma unroll
@@ -733,32 +748,29 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
           ww[q] = fmaf(ww[q], alf[q], wq[q]);
           mrun[q] = mnew[q];
         }
-        // value digit images: plane T, row 4q + d, K byte kpos
+        // the value MMAs' weight image: row 4q + d, K byte kpos; 4 base-256 digits of w 2^F_q << (7 - class)
         if (gi >= 2 && !mbar_wait(&bvr[sb], (uint32_t)(((gi - 2) >> 1) & 1))) {
           ok = false;
           break;
         }
         uint8_t* img = bv + sb * L::BVB + (kpos >> 4) * 256 + (kpos & 15);
 #pragma unroll
-        for (int T = 0; T < NTV; ++T) {
+        for (int q = 0; q < 4; ++q) {
+          int X = __float2int_rn(wq[q] * fq[q]) << sh;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            int X = __float2int_rn(va[T] * wq[q] * fq[q]) * (1 << (7 - cls));
-#pragma unroll
-            for (int dd = 0; dd < 4; ++dd) {
-              const int r = 4 * q + dd;
-              const int lowb = dd < 3 ? (int)(int8_t)(X & 0xFF) : X;
-              img[T * 2048 + (r >> 3) * 128 + (r & 7) * 16] = (uint8_t)lowb;
-              X = (X - lowb) >> 8;
-            }
+          for (int dd = 0; dd < 4; ++dd) {
+            const int r = 4 * q + dd;
+            const int lowb = dd < 3 ? (int)(int8_t)(X & 0xFF) : X;
+            img[(r >> 3) * 128 + (r & 7) * 16] = (uint8_t)lowb;
+            X = (X - lowb) >> 8;
           }
         }
-        fence_async_smem();  // the images are read by the tensor core
+        fence_async_smem();  // the image is read by the tensor core
         __syncwarp();
         if (lane == 0) mbar_arrive(&bvf[sb]);
-        const bool last = it == n_items - 1;
-        if (last) {  // the unit's sums over the 4 warps
-          float* xs = xch + 64;  // [4][8]
+        const bool last = it + 2 >= n_items;  // the group's last item of the unit
+        if (last) {  // the group's sums over its 4 warps
+          float* xs = xg + 64;  // [4][8]
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float l1 = warp_sum(lw[q]), w1 = warp_sum(ww[q]);
@@ -773,9 +785,9 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
             lw[q] = xs[q] + xs[8 + q] + xs[16 + q] + xs[24 + q];
             ww[q] = xs[4 + q] + xs[12 + q] + xs[20 + q] + xs[28 + q];
           }
-          gs.sync(lane);  // xs is reused by the next unit
+          gs.sync(lane);  // xs is reused by the group's next unit
         }
-        // item stats for the value epilogue (one writer)
+        // item stats for the value epilogue (one writer per group)
         if (sw == 0) {
           if (gi >= 2 && !mbar_wait(&str_[sb], (uint32_t)(((gi - 2) >> 1) & 1))) {
             ok = false;
@@ -796,26 +808,28 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
         }
       }
       if (!ok) break;
-      // the unit's m and l (log2 units), one writer per query
+      // the group's partial of the unit (m, l in log2 units): chunk 2 seg + sub, one writer per query
       if (sw == 0 && lane < a.group) {
+        const bool has = n_items > sub;
         const int q = lane;
         float mq = -INFINITY, lq = 0.f;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           if (k == q) {
-            mq = n_items > 0 ? mrun[k] : -INFINITY;
-            lq = n_items > 0 ? lw[k] : 0.f;
+            mq = has ? mrun[k] : -INFINITY;
+            lq = has ? lw[k] : 0.f;
           }
         const int64_t row = (int64_t)b * a.hq + (int64_t)g * a.group + q;
-        float* dst = a.part + (row * a.nseg + seg) * (DP + 2);
+        float* dst = a.part + (row * (2 * a.nseg) + 2 * seg + sub) * (DP + 2);
         dst[DP] = mq;
         dst[DP + 1] = lq;
       }
     }
   } else {
-    // ---------------- value epilogue (lane = coordinate 32 qd + lane) ----------------
+    // ---------------- value epilogue (lane = coordinate 32 qd + lane), one sum set per item parity ----------------
     const int qd = warp & 3;
     const int j = 32 * qd + lane;
+    const float va2[4] = {2.f * a.vco[0], 2.f * a.vco[1], 2.f * a.vco[2], 2.f * a.vco[3]};
     const float vctop = a.vco[4];
     int64_t gi = 0;
     bool ok = true;
@@ -824,18 +838,46 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
       int seg, n_items, len;
       walk.unit(u, pair, seg, n_items, len);
       const int b = (int)(pair / a.hkv), g = (int)(pair - (int64_t)b * a.hkv);
-      float o[4] = {0.f, 0.f, 0.f, 0.f};
-      float wsum[4] = {0.f, 0.f, 0.f, 0.f};
+      float o[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float wsum[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       for (int it = 0; it < n_items && ok; ++it, ++gi) {
-        const int c = (int)(gi % NBV), sb = (int)(gi & 1);
+        const int c = (int)(gi % NBV), sb = (int)(gi & 1), sub = it & 1;
         if (!mbar_wait(&vaf[c], (uint32_t)((gi / NBV) & 1))) {
           ok = false;
           break;
         }
         __syncwarp();
         tc_fence_after();
-        uint32_t D[16];
-        tmem_ld16(tmem + L::C_VACC + 16u * c + ((uint32_t)(32 * qd) << 16), D);
+        // sum_T 2 alpha_T sum_d 256^d D_T[4q + d] = 2^(7+F_q) sum_T 2 alpha_T sum_t w b_T (each D exact,
+        // below 2^22), two planes (32 columns) at a time
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+          const uint32_t lrow = tmem + L::C_VACC + 64u * c + ((uint32_t)(32 * qd) << 16);
+#pragma unroll
+          for (int T0 = 0; T0 < NTV; T0 += 2) {
+            uint32_t d0[16], d1[16];
+            tmem_ld16_issue(lrow + 16 * T0, d0);
+            if (T0 + 1 < NTV) {
+              tmem_ld16_issue(lrow + 16 * T0 + 16, d1);
+              tmem_ld_wait16x2(d0, d1);
+            } else {
+              tmem_ld_wait16(d0);
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (T0 + h < NTV) {
+                const uint32_t* dt = h ? d1 : d0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const float cT = fmaf(i2f_exact(dt[4 * q + 3]), 16777216.f,
+                                        fmaf(i2f_exact(dt[4 * q + 2]), 65536.f,
+                                             fmaf(i2f_exact(dt[4 * q + 1]), 256.f, i2f_exact(dt[4 * q]))));
+                  v[q] = fmaf(va2[T0 + h], cT, v[q]);
+                }
+              }
+            }
+          }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&var_[c]);
@@ -850,29 +892,26 @@ __global__ void __launch_bounds__(DL<KB, VKB>::NTHREADS, 1) decode_tc_kernel(con
           alf[q] = sp[q];
           inv[q] = sp[4 + q];
         }
-        const bool last = sp[12] != 0.f;
-        if (last) {
+        if (sp[12] != 0.f) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) wsum[q] = sp[8 + q];
+          for (int q = 0; q < 4; ++q) wsum[sub][q] = sp[8 + q];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&str_[sb]);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          // sum_d 256^d D[4q + d] = 2^(7+F) sum_T 2 alpha_T sum_t w b_T (each D an exact integer below 2^22)
-          const float v = fmaf((float)(int)D[4 * q + 3], 16777216.f,
-                               fmaf((float)(int)D[4 * q + 2], 65536.f,
-                                    fmaf((float)(int)D[4 * q + 1], 256.f, (float)(int)D[4 * q])));
-          o[q] = fmaf(o[q], alf[q], v * inv[q]);
-        }
+        for (int q = 0; q < 4; ++q) o[sub][q] = fmaf(o[sub][q], alf[q], v[q] * inv[q]);
       }
       if (!ok) break;
-      // o_rot = sum_T 2 alpha_T sum_t w b_T - c[L-1] sum_t w
+      // o_rot = sum_T 2 alpha_T sum_t w b_T - c[L-1] sum_t w, one partial per item parity
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (q < a.group) {
-          const int64_t row = (int64_t)b * a.hq + (int64_t)g * a.group + q;
-          a.part[(row * a.nseg + seg) * (DP + 2) + j] = n_items > 0 ? fmaf(-vctop, wsum[q], o[q]) : 0.f;
+      for (int sbb = 0; sbb < 2; ++sbb) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (q < a.group) {
+            const int64_t row = (int64_t)b * a.hq + (int64_t)g * a.group + q;
+            a.part[(row * (2 * a.nseg) + 2 * seg + sbb) * (DP + 2) + j] =
+                n_items > sbb ? fmaf(-vctop, wsum[sbb][q], o[sbb][q]) : 0.f;
+          }
         }
       }
     }
@@ -928,7 +967,7 @@ int64_t decode_sliced_workspace(int kb, int m, int batch, int n_q_heads, int n_k
   const int64_t nseg = std::max<int64_t>(1, (max_tokens + SEG * TK - 1) / (SEG * TK));
   int64_t img = pairs * image_bytes(kb);
   img = (img + 255) & ~(int64_t)255;
-  return img + 256 + (int64_t)batch * n_q_heads * nseg * (DP + 2) * 4;
+  return img + 256 + (int64_t)batch * n_q_heads * 2 * nseg * (DP + 2) * 4;
 }
 
 int launch_combine(const float* part, int64_t row_stride, int64_t chunk_stride, const int8_t* vD,
@@ -963,7 +1002,7 @@ int decode_attn_sliced(const tq_params* kp, const tq_params* vp, const float* q,
   const int group = n_q_heads / n_kv_heads;
   const int64_t pairs = (int64_t)batch * n_kv_heads;
   const int nseg = (int)std::max<int64_t>(1, (max_tokens + SEG * TK - 1) / (SEG * TK));
-  if (nseg > 2048) return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: max_tokens too large for the combine");
+  if (2 * nseg > 2048) return set_error(TQ_EUNSUPPORTED, "tq_decode_attn: max_tokens too large for the combine");
   const int ib = image_bytes(kb);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int64_t img_total = (pairs * ib + 255) & ~(int64_t)255;
@@ -1018,7 +1057,7 @@ int decode_attn_sliced(const tq_params* kp, const tq_params* vp, const float* q,
     default: rc = dispatch_vkb<3>(vkb, a, sm, st); break;
   }
   if (rc) return rc;
-  rc = launch_combine(part, (int64_t)nseg * (DP + 2), DP + 2, vp->signs_D, seq_lens, out, nseg, vp->d, DP,
+  rc = launch_combine(part, (int64_t)2 * nseg * (DP + 2), DP + 2, vp->signs_D, seq_lens, out, 2 * nseg, vp->d, DP,
                       n_q_heads, (int64_t)batch * n_q_heads, st);
   if (rc == TQ_OK) clear_error();
   return rc;
