@@ -24,17 +24,18 @@
 //
 // Warp roles, one persistent CTA per SM over a contiguous range of
 // (KV head, 128-key tile) items, all hand-offs on mbarriers with bounded waits:
-//   warp 0      bulk copies of code tiles and norms into a ring of stages;
-//   warps 1-4   MMA issue: two pairs take alternate items; each warp of a pair
-//               issues every other K step of the item into its own partial
-//               accumulator.  The loops are warp-uniform and one lane, chosen
-//               by elect.sync, issues, with the descriptors of a whole item
-//               unrolled from two base values;
-//   warps 5-12  expansion: stage -> masked words -> tcgen05.st into one of two
-//               or three A buffers (warp = lane quadrant x 4 bit classes);
-//   warps 13-20 query preparation into a ring of two B images, then the
+//   warp 0      bulk copies of the code tiles into a ring of stages, two items
+//               per copy;
+//   warps 1-2   MMA issue: warp 1 + p takes the items of parity p, all K steps
+//               of an item into one accumulator set.  The loops are warp-uniform
+//               and one lane, chosen by elect.sync, issues, with the
+//               descriptors of a whole item unrolled from two base values;
+//   warps 3-10  expansion: stage -> masked words -> tcgen05.st into one of two
+//               or four A buffers (warp = lane quadrant; 3-6 even items, 7-10 odd);
+//   warps 11-18 query preparation into a ring of two B images, then the
 //               epilogue: tcgen05.ld of the partial accumulators, digit
-//               combination, norms, logits (warp = lane quadrant x 2 queries).
+//               combination, norms (plain loads issued two items ahead), logits
+//               (warp = lane quadrant).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -51,6 +52,7 @@ using namespace tqd;
 constexpr int TK = 128;  // keys per item (MMA M)
 constexpr int DP = 128;
 constexpr int MAX_STAGES = 12;
+constexpr int GI = 2;  // items per code copy (a bulk copy costs a few hundred cycles of the copy engine)
 
 struct TArgs {
   const uint8_t* codes;
@@ -60,7 +62,8 @@ struct TArgs {
   int group;           // query heads per KV head, 1..4
   int tb;              // bytes of one 32-key code tile
   int tiles_per_head;  // ceil(n_keys / 128)
-  int64_t n_items;     // n_kv_heads * tiles_per_head
+  int64_t n_items;     // n_kv_heads * tiles_per_head (below 2^31)
+  uint32_t per_cta, rem_cta;  // n_items = per_cta * gridDim.x + rem_cta
   const float* q;      // [n_kv_heads * group][d] fp32
   int d;
   int kb;
@@ -71,7 +74,7 @@ struct TArgs {
   float* logits;
   int64_t ld;          // logits row stride
   float kappa;         // sqrt(pi/2) / m
-  int stages;          // ring stages (<= MAX_STAGES)
+  int stages;          // ring stages of GI items (<= MAX_STAGES)
 };
 
 template <int KB, int SI>
@@ -88,15 +91,17 @@ struct TL {
   static constexpr int IMG_S = 64 + NT * 2048;
   static constexpr int IMG = (64 + NP * 2048 + 127) / 128 * 128;
   static constexpr int TILEB = 32 * 16 * (KB + SI);  // one 32-key code tile
-  static constexpr int NORMB = 256 * (1 + SI);       // fp16 norms (+ residual norms) of 128 keys
-  static constexpr int STAGE = 4 * TILEB + NORMB;    // one item: code tiles, then norms
-  static constexpr int ACC = 64;                     // accumulator set: 2 partials x (16 centroid + 16 sign)
-  static constexpr int NA = (3 * ACOLS + 3 * ACC <= 512) ? 3 : 2;
-  static constexpr int NB0 = (512 - NA * ACOLS) / ACC;
-  static constexpr int NB = NB0 < 4 ? NB0 : 4;
-  static_assert(NB >= 2 && NA * ACOLS + NB * ACC <= 512, "tensor-memory budget");
-  static constexpr int W_EXP0 = 5, W_EPI0 = 13;
-  static constexpr int NTHREADS = 21 * 32;
+  static constexpr int STAGE = GI * 4 * TILEB;       // the code tiles of GI items
+  static constexpr int ACC = 32;                     // accumulator set: 16 centroid + 16 sign columns
+  // Even buffer counts: item i and item i - NA (i - NB) have the same parity, so one MMA pair,
+  // one expansion group and one epilogue group meet every phase of a buffer's barriers in turn.
+  // (With an odd count a waiter could arrive two phases ahead, see the parity of the phase
+  // before and pass without waiting.)
+  static constexpr int NA = (4 * ACOLS + 2 * ACC <= 512) ? 4 : 2;
+  static constexpr int NB = (NA * ACOLS + 4 * ACC <= 512) ? 4 : 2;
+  static_assert(NA * ACOLS + NB * ACC <= 512, "tensor-memory budget");
+  static constexpr int W_EXP0 = 3, W_EPI0 = 11;
+  static constexpr int NTHREADS = 19 * 32;
   static constexpr int OFF_IMG = 1024;
   static constexpr int OFF_PREP = OFF_IMG + 2 * IMG;  // q_rot [2][128], u [2][128], partial u [2][2][128] (float4)
   static constexpr int OFF_RING = OFF_PREP + 8 * 128 * 16;
@@ -117,12 +122,17 @@ __device__ __forceinline__ float pow2(int k) {
 }
 
 // Global loads of the query preparation, issued early so their latency overlaps
-// other work: warp ew's query (image ew / 4, query ew % 4), times the sign flips,
-// and thread et's half row of S (row et % 128, coordinates 64 (et / 128) ..).
+// other work: warp ew's query (image ew / 4, query ew % 4), the sign flips, and
+// thread et's half row of S (row et % 128, coordinates 64 (et / 128) ..).  The
+// loaded values are only stored here (no arithmetic or select on them), so the
+// loads do not hold the warp before their first use; out-of-range elements load
+// from a valid address and are zeroed by `ymask` in make_images.
 struct PrepRegs {
   float y[4];
+  int ds[4];
+  uint32_t ymask;  // bit i: coordinate 32 i + lane of a real query
   uint4 sv[8];
-  float cv;  // centroid et (et < 2^kb)
+  float cv;  // centroid et (et < 2^kb; other lanes hold centroid 0)
 };
 
 template <int SI>
@@ -130,18 +140,22 @@ __device__ __forceinline__ void prep_load(const TArgs& a, int64_t head0, int n_i
   const int ew = et >> 5, lane = et & 31;
   const int k = ew >> 2, j = ew & 3;
   const bool valid = k < n_img && j < a.group;
-  pr.cv = et < (1 << a.kb) ? __ldg(a.cent + et) : 0.f;
-  const int64_t row = (head0 + k) * a.group + j;
+  pr.cv = __ldg(a.cent + (et < (1 << a.kb) ? et : 0));
+  const int64_t row = valid ? (head0 + k) * a.group + j : 0;
+  pr.ymask = 0u;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int c = 32 * i + lane;
-    pr.y[i] = (valid && c < a.d) ? __ldg(a.q + row * a.d + c) * (float)__ldg(a.D + c) : 0.f;
+    const bool ok = valid && c < a.d;
+    pr.ymask |= ok ? (1u << i) : 0u;
+    pr.y[i] = __ldg(a.q + (ok ? row * a.d + c : 0));
+    pr.ds[i] = __ldg(a.D + c);
   }
-  if constexpr (SI) {
+  if constexpr (SI) {  // m = 128: every row of S exists
     const int r = et & 127, h = et >> 7;
     const uint4* srow = reinterpret_cast<const uint4*>(a.S + (size_t)r * DP) + 8 * h;
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) pr.sv[kk] = r < a.m ? __ldg(srow + kk) : make_uint4(0, 0, 0, 0);
+    for (int kk = 0; kk < 8; ++kk) pr.sv[kk] = __ldg(srow + kk);
   }
 }
 
@@ -161,6 +175,8 @@ __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* im
   float* rd = red + 16 * kq;                  // per query of image kq: sum, max, 2^F, 2^G
   {
     float* y = pr.y;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) y[i] = ((pr.ymask >> i) & 1u) ? y[i] * (float)pr.ds[i] : 0.f;
 #pragma unroll
     for (int h = 1; h < 4; h <<= 1)
 #pragma unroll
@@ -287,19 +303,55 @@ __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* im
   sync();
 }
 
+// The code tiles of the next GI items (or fewer, at the end of the CTA's range of nleft items)
+// into one stage: one bulk copy when the tiles are contiguous in global memory (every item but
+// the last of the group holds 128 keys), else one per item.  (head, t) is the next item's KV
+// head and 128-key tile, advanced here (no integer division on the producer's path).
+template <int KB, int SI>
+__device__ __forceinline__ void copy_group(const TArgs& a, int nleft, int64_t& head, int& t, uint8_t* dst,
+                                           uint64_t* bar) {
+  using L = TL<KB, SI>;
+  int64_t tile[GI];
+  int nt[GI];
+  uint32_t total = 0;
+  bool whole = true;
+#pragma unroll
+  for (int j = 0; j < GI; ++j) {
+    nt[j] = 0;
+    tile[j] = 0;
+    if (j < nleft) {
+      const int64_t k0 = (int64_t)t * TK;
+      const int64_t nk = a.n_keys - k0 < TK ? a.n_keys - k0 : TK;
+      tile[j] = (head * a.n_keys + k0) >> 5;
+      nt[j] = (int)(nk >> 5);
+      total += (uint32_t)(nt[j] * L::TILEB);
+      if (j + 1 < nleft && j + 1 < GI && nt[j] != 4) whole = false;
+      if (++t == a.tiles_per_head) t = 0, ++head;
+    }
+  }
+  mbar_expect_tx(bar, total);
+  if (whole) {
+    bulk_g2s(dst, a.codes + tile[0] * L::TILEB, total, bar);
+  } else {
+#pragma unroll
+    for (int j = 0; j < GI; ++j)
+      if (nt[j] > 0) bulk_g2s(dst + j * 4 * L::TILEB, a.codes + tile[j] * L::TILEB, nt[j] * L::TILEB, bar);
+  }
+}
+
 template <int KB, int SI>
 __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(const TArgs a) {
   using L = TL<KB, SI>;
   constexpr int W_EXP0 = L::W_EXP0, W_EPI0 = L::W_EPI0;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // [MAX_STAGES] stage loaded
-  uint64_t* empty = full + MAX_STAGES;                 // [MAX_STAGES] stage read by expansion and epilogue
-  uint64_t* afull = empty + MAX_STAGES;                // [3] A buffer written (8 arrivals)
-  uint64_t* mdone = afull + 3;                         // [3] MMAs of the item done: its A buffer is free (2)
-  uint64_t* cfull = mdone + 3;                         // [4] accumulator set full (2)
-  uint64_t* accfree = cfull + 4;                       // [4] accumulator set read (8)
+  uint64_t* empty = full + MAX_STAGES;                 // [MAX_STAGES] stage read by the 8 expansion warps
+  uint64_t* afull = empty + MAX_STAGES;                // [4] A buffer written (4 arrivals)
+  uint64_t* mdone = afull + 4;                         // [4] MMAs of the item done: its A buffer is free (1)
+  uint64_t* cfull = mdone + 4;                         // [4] accumulator set full (1)
+  uint64_t* accfree = cfull + 4;                       // [4] accumulator set read (4)
   uint64_t* imgfull = accfree + 4;                     // [2] B image ready (1)
-  uint64_t* imgfree = imgfull + 2;                     // [2] no MMA reads the B image any more (4)
+  uint64_t* imgfree = imgfull + 2;                     // [2] no MMA reads the B image any more (2)
   uint64_t* gbar = imgfree + 2;                        // barrier of the 8 prep / epilogue warps (8)
   uint32_t* tbase = reinterpret_cast<uint32_t*>(gbar + 1);
   float* alpha = reinterpret_cast<float*>(tbase + 4);  // [5] Walsh coefficients, then c[L-1]
@@ -312,35 +364,65 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.stages;
-  const int64_t i0 = (int64_t)blockIdx.x * a.n_items / gridDim.x;
-  const int64_t i1 = (int64_t)(blockIdx.x + 1) * a.n_items / gridDim.x;
-  const int n = (int)(i1 - i0);
-  const int64_t h_first = i0 / a.tiles_per_head;
-  const int n_img = n > 0 ? (int)((i1 - 1) / a.tiles_per_head - h_first) + 1 : 0;
+  // this CTA's items [i0, i1) = [b n_items / G, (b + 1) n_items / G), in 32-bit arithmetic
+  // (a 64-bit division costs hundreds of cycles on the start-up path)
+  const uint32_t bx = blockIdx.x;
+  const uint32_t u0 = bx * a.per_cta + bx * a.rem_cta / gridDim.x;
+  const uint32_t u1 = (bx + 1) * a.per_cta + (bx + 1) * a.rem_cta / gridDim.x;
+  const int64_t i0 = u0;
+  const int n = (int)(u1 - u0);
+  const uint32_t tph = (uint32_t)a.tiles_per_head;
+  const int64_t h_first = u0 / tph;
+  const int t_first = (int)(u0 - (uint32_t)h_first * tph);
+  const int n_img = n > 0 ? (int)((u1 - 1) / tph - (uint32_t)h_first) + 1 : 0;
+  const int n_groups = (n + GI - 1) / GI;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < MAX_STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 8);  // the 4 expansion and 4 epilogue warps of the item's parity
+      mbar_init(&empty[s], 8);  // the 4 expansion warps of each of the GI = 2 items
     }
-    for (int b = 0; b < 3; ++b) {
+    for (int b = 0; b < 4; ++b) {
       mbar_init(&afull[b], 4);
-      mbar_init(&mdone[b], 2);
+      mbar_init(&mdone[b], 1);
     }
     for (int c = 0; c < 4; ++c) {
-      mbar_init(&cfull[c], 2);
+      mbar_init(&cfull[c], 1);
       mbar_init(&accfree[c], 4);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&imgfull[k], 1);
-      mbar_init(&imgfree[k], 4);
+      mbar_init(&imgfree[k], 2);
     }
     mbar_init(gbar, 8);
   }
+
   PrepRegs pr;
+  // epilogue warps: the norms of key 32 qd + lane of an item, plain loads issued two of the warp's
+  // items (four items) ahead; (nh, ntl) walks the items being loaded, nidx is the next one's index
+  const int epar = ((warp - W_EPI0) >> 2) & 1;
+  int64_t nh = h_first;
+  int ntl = t_first, nidx = 0;
+  // (raw fp16 bits, converted where used; keys past the range load key 0 and are never used)
+  auto norms_next = [&](uint16_t& nr, uint16_t& ga) {  // item nidx, then advance the walk by 2
+    const int64_t key = (int64_t)ntl * TK + 32 * (warp & 3) + lane;
+    const int64_t at = (nidx < n && key < a.n_keys) ? nh * a.n_keys + key : 0;
+    nr = __ldg(a.norms + at);
+    if constexpr (SI) ga = __ldg(a.rnorms + at);
+    nidx += 2;
+    ntl += 2;
+    while (ntl >= a.tiles_per_head) ntl -= a.tiles_per_head, ++nh;
+  };
+  uint16_t nrm0 = 0, gam0 = 0, nrm1 = 0, gam1 = 0;
   if (warp >= W_EPI0) {  // the first one or two heads' query loads overlap the set-up
-    grid_dependency_wait();  // queries may come from the preceding kernel in the stream
+    grid_dependency_wait();  // queries and norms may come from the preceding kernel in the stream
     prep_load<SI>(a, h_first, n_img < 2 ? n_img : 2, threadIdx.x - 32 * W_EPI0, pr);
+    if (epar) {  // this group's first item is item 1
+      nidx = 1;
+      if (++ntl == a.tiles_per_head) ntl = 0, ++nh;
+    }
+    norms_next(nrm0, gam0);
+    norms_next(nrm1, gam1);
   }
   if (warp == 0) tmem_alloc(tbase, 512);
   tc_fence_before();
@@ -352,35 +434,26 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
   auto a_col = [&](int b) { return tmem + (uint32_t)(L::ACC * L::NB + b * L::ACOLS); };
 
   if (warp == 0) {
-    // ---------------- producer: code tiles and norms into the ring ----------------
+    // ---------------- producer: code tiles into the ring, GI items per stage ----------------
     grid_dependency_wait();  // codes may come from the preceding kernel in the stream
     if (lane == 0) {
+      int64_t ph = h_first;  // the next item's KV head and tile
+      int pt = t_first;
       int issued = 0;
-      int64_t head = h_first;
-      int t = (int)(i0 % a.tiles_per_head);
-      for (int i = 0, s = 0, use = 0; i < n; ++i) {
-        if (i >= S && !mbar_wait(&empty[s], (use - 1) & 1)) break;
-        const int64_t k0 = (int64_t)t * TK;
-        const int nk = (int)((a.n_keys - k0) < TK ? (a.n_keys - k0) : TK);
-        const int64_t tile0 = (head * a.n_keys + k0) >> 5;
-        const uint32_t bytes = (uint32_t)((nk >> 5) * a.tb);
-        uint8_t* dst = ring + s * L::STAGE;
-        mbar_expect_tx(&full[s], bytes + (uint32_t)(2 * nk * (1 + SI)));
-        bulk_g2s(dst, a.codes + tile0 * a.tb, bytes, &full[s]);
-        bulk_g2s(dst + 4 * L::TILEB, a.norms + head * a.n_keys + k0, 2 * nk, &full[s]);
-        if constexpr (SI) bulk_g2s(dst + 4 * L::TILEB + 256, a.rnorms + head * a.n_keys + k0, 2 * nk, &full[s]);
-        issued = i + 1;
-        if (++t == a.tiles_per_head) t = 0, ++head;
+      for (int g = 0, s = 0, use = 0; g < n_groups; ++g) {
+        if (use >= 1 && !mbar_wait(&empty[s], (use - 1) & 1)) break;
+        copy_group<KB, SI>(a, n - GI * g, ph, pt, ring + s * L::STAGE, &full[s]);
+        issued = g + 1;
         if (++s == S) s = 0, ++use;
       }
       // nothing may still be in flight into shared memory when the CTA ends
-      for (int i = (issued > S ? issued - S : 0); i < issued; ++i) mbar_wait(&full[i % S], (i / S) & 1);
+      for (int g = (issued > S ? issued - S : 0); g < issued; ++g) mbar_wait(&full[g % S], (g / S) & 1);
     }
   } else if (warp < W_EXP0) {
     // ---------------- MMA issue (warp-uniform, elected lane) ----------------
-    const int j = warp - 1, par = j >> 1, k = j & 1;
+    const int par = warp - 1;
     constexpr uint32_t idesc = idesc_u8s8_s32(TK, 16);
-    int t = (int)(i0 % a.tiles_per_head);
+    int t = t_first;
     int kimg = 0;
     bool ok = n > 0 && mbar_wait(&imgfull[0], 0);
     uint32_t simg = smem_u32(imgs);
@@ -399,18 +472,17 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       if (cu >= 1 && !mbar_wait(&accfree[c], (cu - 1) & 1)) break;
       __syncwarp();  // elect.sync needs the whole warp converged
       tc_fence_after();
-      const uint32_t dacc = acc_col(c) + 32u * (uint32_t)k;
-      const uint32_t abuf = a_col(b) + 8u * (uint32_t)k;
-      const uint64_t dc = smem_desc(simg + L::IMG_C + 512 * k, 256, 128);
+      const uint32_t dacc = acc_col(c);
+      const uint32_t abuf = a_col(b);
+      const uint64_t dc = smem_desc(simg + L::IMG_C, 256, 128);
 #pragma unroll
-      for (int u = 0; u < L::CSTEPS / 2; ++u)  // K steps k, k+2, ...: 1024 bytes of image apart
-        umma_i8_ts_elect(dacc, abuf + 16u * u, dc + (uint64_t)(64 * u), idesc, u > 0 ? 1u : 0u);
+      for (int u = 0; u < L::CSTEPS; ++u)  // K step u: 8 A columns (32 bytes), 512 bytes of image
+        umma_i8_ts_elect(dacc, abuf + 8u * u, dc + (uint64_t)(32 * u), idesc, u > 0 ? 1u : 0u);
       if constexpr (SI) {
-        const uint64_t ds = smem_desc(simg + L::IMG_S + 512 * k, 256, 128);
+        const uint64_t ds = smem_desc(simg + L::IMG_S, 256, 128);
 #pragma unroll
-        for (int u = 0; u < L::SSTEPS / 2; ++u)
-          umma_i8_ts_elect(dacc + 16u, abuf + 32u * L::NT + 16u * u, ds + (uint64_t)(64 * u), idesc,
-                           u > 0 ? 1u : 0u);
+        for (int u = 0; u < L::SSTEPS; ++u)
+          umma_i8_ts_elect(dacc + 16u, abuf + 32u * L::NT + 8u * u, ds + (uint64_t)(32 * u), idesc, u > 0 ? 1u : 0u);
       }
       umma_commit_elect(&mdone[b]);
       umma_commit_elect(&cfull[c]);
@@ -418,20 +490,22 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
     __syncwarp();
   } else if (warp < W_EPI0) {
     // ---------------- expansion: code bits -> A in tensor memory ----------------
-    // warps 5-8 take the even items, 9-12 the odd ones; each covers one lane quadrant
-    // (a 32-key tile of the item) and all 8 bit classes of every plane
+    // warps 3-6 take the even items, 7-10 the odd ones; each covers one lane quadrant
+    // (a 32-key tile of the item) and all 8 bit classes of every plane.  They start once
+    // the first query image is built, leaving the SM's issue slots to its preparation.
     const int ew = warp - W_EXP0;
     const int qd = warp & 3, par = ew >> 2;
-    for (int i = par; i < n; i += 2) {
-      const int s = i % S, use = i / S;
+    const bool go = n > 0 && mbar_wait(&imgfull[0], 0);
+    for (int i = par, s = 0, use = 0; go && i < n; i += 2) {  // item i sits in group i / 2: stage s, pass use
       const int b = i % L::NA, ua = i / L::NA;
       if (!mbar_wait(&full[s], use & 1)) break;
       if (ua >= 1 && !mbar_wait(&mdone[b], (ua - 1) & 1)) break;  // MMAs of item i - NA have read A[b]
-      const uint8_t* st = ring + s * L::STAGE + qd * L::TILEB + lane * 16;
+      const uint8_t* st = ring + s * L::STAGE + (i % GI) * 4 * L::TILEB + qd * L::TILEB + lane * 16;
       uint4 pw[KB + SI];
 #pragma unroll
       for (int p = 0; p < KB + SI; ++p) pw[p] = *reinterpret_cast<const uint4*>(st + p * 512);
       release_to_copy(&empty[s], lane);  // the stage is refilled once its 8 readers release it
+      if (++s == S) s = 0, ++use;
       uint4 it[L::NP];
 #pragma unroll
       for (int T = 0; T < L::NT; ++T) it[T] = pw[T < KB ? T : 0];
@@ -493,7 +567,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       }
     }
     int64_t head = h_first;
-    int t = (int)(i0 % a.tiles_per_head);
+    int t = t_first;
     int kimg = 0;
     for (int i = 0; i < n; ++i, ++t) {
       if (t == a.tiles_per_head) {
@@ -509,33 +583,24 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
         }
       }
       if ((i & 1) != par) continue;
-      const int s = i % S, use = i / S, c = i % L::NB, cu = i / L::NB;
+      const int c = i % L::NB, cu = i / L::NB;
       const int64_t key = (int64_t)t * TK + 32 * qd + lane;
       const bool kvalid = key < a.n_keys;
-      if (!mbar_wait(&full[s], use & 1)) break;  // long complete: makes the stage's norms visible here
-      const __half* nst = reinterpret_cast<const __half*>(ring + s * L::STAGE + 4 * L::TILEB);
-      const float nrm = __half2float(nst[32 * qd + lane]);
-      const float gam = SI ? __half2float(nst[128 + 32 * qd + lane]) : 0.f;
-      release_to_copy(&empty[s], lane);
+      const float nrm = __half2float(__ushort_as_half(nrm0)), gam = SI ? __half2float(__ushort_as_half(gam0)) : 0.f;
+      nrm0 = nrm1;
+      gam0 = gam1;
+      norms_next(nrm1, gam1);  // item i + 4
       if (!mbar_wait(&cfull[c], cu & 1)) break;
       tc_fence_after();
       const uint32_t lrow = acc_col(c) + ((uint32_t)(32 * qd) << 16);
-      uint32_t C[16], Z[16];  // 4 queries x 4 digits, centroid and sign sums
-      {
-        uint32_t c1[16];
-        tmem_ld16_issue(lrow, C);
-        tmem_ld16_issue(lrow + 32, c1);
-        tmem_ld_wait16x2(C, c1);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) C[e] += c1[e];  // exact: the full sums stay below 2^24
-      }
+      uint32_t C[16], Z[16];  // 4 queries x 4 digits, centroid and sign sums (exact int32, below 2^24)
       if constexpr (SI) {
-        uint32_t s1[16];
+        tmem_ld16_issue(lrow, C);
         tmem_ld16_issue(lrow + 16, Z);
-        tmem_ld16_issue(lrow + 48, s1);
-        tmem_ld_wait16x2(Z, s1);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) Z[e] += s1[e];
+        tmem_ld_wait16x2(C, Z);
+      } else {
+        tmem_ld16_issue(lrow, C);
+        tmem_ld_wait16(C);
       }
       tc_fence_before();
       __syncwarp();
@@ -579,7 +644,10 @@ int launch_tc(const TArgs& a0, int sm, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return tq::set_error(TQ_ECUDA, "tq_logits: %s", cudaGetErrorString(e));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(sm, a.n_items)));
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(sm, a.n_items));
+  a.per_cta = (uint32_t)(a.n_items / grid);
+  a.rem_cta = (uint32_t)(a.n_items % grid);
+  cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(L::NTHREADS);
   cfg.dynamicSmemBytes = bytes;
   cfg.stream = st;
@@ -626,6 +694,7 @@ int launch_logits_tc(int kb, int m, const float* q, int d, const float* cent, co
   a.ld = ld;
   a.kappa = (float)(std::sqrt(M_PI / 2.0) / (m > 0 ? m : 1));
   a.stages = MAX_STAGES;
+  if (a.n_items >= (int64_t(1) << 31)) return set_error(TQ_EINVAL, "tq_logits: more than 2^31 tiles of 128 keys");
   const int sm = sm_count();
   if (m > 0) {
     switch (kb) {
