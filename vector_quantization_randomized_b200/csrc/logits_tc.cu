@@ -103,8 +103,9 @@ struct TL {
   static constexpr int W_EXP0 = 3, W_EPI0 = 11;
   static constexpr int NTHREADS = 19 * 32;
   static constexpr int OFF_IMG = 1024;
-  static constexpr int OFF_PREP = OFF_IMG + 2 * IMG;  // q_rot [2][128], u [2][128], partial u [2][2][128] (float4)
-  static constexpr int OFF_RING = OFF_PREP + 8 * 128 * 16;
+  static constexpr int OFF_PREP = OFF_IMG + 2 * IMG;  // q_rot [2][128], u [2][128], partial u [2][4][128] (float4)
+  static constexpr int OFF_S = OFF_PREP + 12 * 128 * 16;     // S, fp16 [128][128], chunks swizzled (SI)
+  static constexpr int OFF_RING = OFF_S + (SI ? 128 * 256 : 0);
   static constexpr int smem(int stages) { return OFF_RING + stages * STAGE; }
 };
 
@@ -122,21 +123,22 @@ __device__ __forceinline__ float pow2(int k) {
 }
 
 // Global loads of the query preparation, issued early so their latency overlaps
-// other work: warp ew's query (image ew / 4, query ew % 4), the sign flips, and
-// thread et's half row of S (row et % 128, coordinates 64 (et / 128) ..).  The
-// loaded values are only stored here (no arithmetic or select on them), so the
-// loads do not hold the warp before their first use; out-of-range elements load
-// from a valid address and are zeroed by `ymask` in make_images.
+// other work: warp ew's query (image ew / 4, query ew % 4), the sign flips and
+// 16-byte chunks et + 256 k of S (coalesced; make_images stores them to shared
+// memory).  The loaded values are only stored here (no arithmetic or select on
+// them), so the loads do not hold the warp before their first use; out-of-range
+// elements load from a valid address and are zeroed by `ymask` in make_images.
 struct PrepRegs {
   float y[4];
   int ds[4];
   uint32_t ymask;  // bit i: coordinate 32 i + lane of a real query
-  uint4 sv[8];
-  float cv;  // centroid et (et < 2^kb; other lanes hold centroid 0)
+  uint4 sv[8];     // S chunks (SI; the first preparation of the CTA only)
+  float cv;        // centroid et (et < 2^kb; other lanes hold centroid 0)
 };
 
 template <int SI>
-__device__ __forceinline__ void prep_load(const TArgs& a, int64_t head0, int n_img, int et, PrepRegs& pr) {
+__device__ __forceinline__ void prep_load(const TArgs& a, int64_t head0, int n_img, int et, PrepRegs& pr,
+                                          bool with_s) {
   const int ew = et >> 5, lane = et & 31;
   const int k = ew >> 2, j = ew & 3;
   const bool valid = k < n_img && j < a.group;
@@ -151,12 +153,48 @@ __device__ __forceinline__ void prep_load(const TArgs& a, int64_t head0, int n_i
     pr.y[i] = __ldg(a.q + (ok ? row * a.d + c : 0));
     pr.ds[i] = __ldg(a.D + c);
   }
-  if constexpr (SI) {  // m = 128: every row of S exists
-    const int r = et & 127, h = et >> 7;
-    const uint4* srow = reinterpret_cast<const uint4*>(a.S + (size_t)r * DP) + 8 * h;
+  if constexpr (SI) {  // m = 128: S is 32 KB
+    if (with_s) {
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) pr.sv[kk] = __ldg(srow + kk);
+      for (int k = 0; k < 8; ++k) pr.sv[k] = __ldg(reinterpret_cast<const uint4*>(a.S) + et + 256 * k);
+    }
   }
+}
+
+// Partial sums of u = S q_rot for up to two query images: thread x of NQ * 128 takes row
+// i = x % 128 and the 128 / NQ coordinates of part x / 128; up[(NQ im + part) 128 + i]
+// receives its sums for the 4 queries of image im.  S sits in shared memory with 16-byte
+// chunk c of row r at r * 16 + (c ^ (r & 15)) (8 consecutive rows read 8 banks apart).
+template <int NQ>
+__device__ __forceinline__ void sq_part(const float4* qT, const uint8_t* sS, float4* up, int n_img, int x) {
+  constexpr int NC = 16 / NQ;  // 16-byte chunks (8 coordinates) per part
+  const int i = x & 127, part = x >> 7;
+  float2 acc[2][2];  // [image][queries 0-1, 2-3], packed fp32x2
+#pragma unroll
+  for (int im = 0; im < 2; ++im) acc[im][0] = acc[im][1] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    const int c = NC * part + k;
+    const uint4 sv = reinterpret_cast<const uint4*>(sS)[i * 16 + (c ^ (i & 15))];
+    const uint32_t wv[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+    for (int h2 = 0; h2 < 4; ++h2) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[h2]));
+      const float2 fx = make_float2(f.x, f.x), fy = make_float2(f.y, f.y);
+      const int j = 8 * c + 2 * h2;
+#pragma unroll
+      for (int im = 0; im < 2; ++im) {
+        if (im < n_img) {
+          const float4 q0 = qT[128 * im + j], q1 = qT[128 * im + j + 1];
+          acc[im][0] = __ffma2_rn(fy, make_float2(q1.x, q1.y), __ffma2_rn(fx, make_float2(q0.x, q0.y), acc[im][0]));
+          acc[im][1] = __ffma2_rn(fy, make_float2(q1.z, q1.w), __ffma2_rn(fx, make_float2(q0.z, q0.w), acc[im][1]));
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int im = 0; im < 2; ++im)
+    if (im < n_img) up[(NQ * im + part) * 128 + i] = make_float4(acc[im][0].x, acc[im][0].y, acc[im][1].x, acc[im][1].y);
 }
 
 // B images of n_img (1 or 2) consecutive KV heads into img0 / img1, by the 256
@@ -164,9 +202,10 @@ __device__ __forceinline__ void prep_load(const TArgs& a, int64_t head0, int n_i
 // q_rot = H D q / sqrt(128) (warp per query: image ew / 4, query ew % 4);
 // u = S q_rot (thread = row of S x half of the coordinates, both images);
 // per-query scales 2^F, 2^G putting the largest weight just below 2^23; digits.
-template <int KB, int SI, class Sync>
+template <int KB, int SI, bool WIDE, class Sync>
 __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* img0, uint8_t* img1, float4* qT,
-                            float4* uT, float4* up, const float* alpha, float* red, int et, Sync&& sync) {
+                            float4* uT, float4* up, const float* alpha, float* red, uint8_t* sS, bool with_s,
+                            int et, Sync&& sync) {
   using L = TL<KB, SI>;
   const int ew = et >> 5, lane = et & 31;
   const int kq = ew >> 2, jq = ew & 3;  // this warp's image and query
@@ -208,38 +247,41 @@ __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* im
       rd[4 * jq + 1] = mx;
     }
   }
-  sync();
-  if constexpr (SI) {  // u = S q_rot: row i = et % 128, coordinates 64h .. 64h + 63 (h = et / 128)
-    const int i = et & 127, h = et >> 7;
-    float2 acc[2][2];  // [image][queries 0-1, 2-3], packed fp32x2
+  if constexpr (SI) {  // S into shared memory (kept for the CTA's later preparations): 16-byte chunk c of
+    // row r at r * 16 + (c ^ (r & 15)), so both a row's 16 chunks (stored here) and one chunk of 8
+    // consecutive rows (read below) fall in distinct banks
+    if (with_s) {
 #pragma unroll
-    for (int im = 0; im < 2; ++im) acc[im][0] = acc[im][1] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t wv[4] = {pr.sv[k].x, pr.sv[k].y, pr.sv[k].z, pr.sv[k].w};
-#pragma unroll
-      for (int h2 = 0; h2 < 4; ++h2) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[h2]));
-        const float2 fx = make_float2(f.x, f.x), fy = make_float2(f.y, f.y);
-        const int j = 64 * h + 8 * k + 2 * h2;
-#pragma unroll
-        for (int im = 0; im < 2; ++im) {
-          if (im < n_img) {
-            const float4 q0 = qT[128 * im + j], q1 = qT[128 * im + j + 1];
-            acc[im][0] = __ffma2_rn(fy, make_float2(q1.x, q1.y), __ffma2_rn(fx, make_float2(q0.x, q0.y), acc[im][0]));
-            acc[im][1] = __ffma2_rn(fy, make_float2(q1.z, q1.w), __ffma2_rn(fx, make_float2(q0.z, q0.w), acc[im][1]));
-          }
-        }
+      for (int k = 0; k < 8; ++k) {
+        const int g = et + 256 * k, r = g >> 4, c = g & 15;
+        reinterpret_cast<uint4*>(sS)[r * 16 + (c ^ (r & 15))] = pr.sv[k];
       }
     }
-#pragma unroll
-    for (int im = 0; im < 2; ++im)
-      up[256 * im + 128 * h + i] = make_float4(acc[im][0].x, acc[im][0].y, acc[im][1].x, acc[im][1].y);
+  }
+  if constexpr (SI && WIDE) {
+    // u = S q_rot by the 8 expansion warps as well (threads 256 .. 511 of named barrier 2): a
+    // quarter row each
+    named_sync(2, 512);
+    sq_part<4>(qT, sS, up, n_img, et);
+    named_sync(2, 512);
+  } else {
     sync();
-    {
-      const int im = et >> 7, r = et & 127;  // thread = (image, row)
-      const float4 p0 = up[256 * im + r], p1 = up[256 * im + 128 + r];
-      uT[128 * im + r] = make_float4(p0.x + p1.x, p0.y + p1.y, p0.z + p1.z, p0.w + p1.w);
+    if constexpr (SI) {  // a half row per thread
+      sq_part<2>(qT, sS, up, n_img, et);
+      sync();
+    }
+  }
+  if constexpr (SI) {
+    constexpr int NQ = WIDE ? 4 : 2;
+    const int im = et >> 7, r = et & 127;  // thread = (image, row)
+    if (im < n_img) {
+      float4 t = up[(NQ * im) * 128 + r];
+#pragma unroll
+      for (int pp = 1; pp < NQ; ++pp) {
+        const float4 v = up[(NQ * im + pp) * 128 + r];
+        t = make_float4(t.x + v.x, t.y + v.y, t.z + v.z, t.w + v.w);
+      }
+      uT[128 * im + r] = t;
     }
     sync();
   }
@@ -416,7 +458,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
   uint16_t nrm0 = 0, gam0 = 0, nrm1 = 0, gam1 = 0;
   if (warp >= W_EPI0) {  // the first one or two heads' query loads overlap the set-up
     grid_dependency_wait();  // queries and norms may come from the preceding kernel in the stream
-    prep_load<SI>(a, h_first, n_img < 2 ? n_img : 2, threadIdx.x - 32 * W_EPI0, pr);
+    prep_load<SI>(a, h_first, n_img < 2 ? n_img : 2, threadIdx.x - 32 * W_EPI0, pr, true);
     if (epar) {  // this group's first item is item 1
       nidx = 1;
       if (++ntl == a.tiles_per_head) ntl = 0, ++nh;
@@ -491,12 +533,19 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
   } else if (warp < W_EPI0) {
     // ---------------- expansion: code bits -> A in tensor memory ----------------
     // warps 3-6 take the even items, 7-10 the odd ones; each covers one lane quadrant
-    // (a 32-key tile of the item) and all 8 bit classes of every plane.  They start once
-    // the first query image is built, leaving the SM's issue slots to its preparation.
+    // (a 32-key tile of the item) and all 8 bit classes of every plane.  First they take a
+    // share of the CTA's first query preparation (u = S q_rot, between two named barriers
+    // with the 8 preparation warps).
     const int ew = warp - W_EXP0;
     const int qd = warp & 3, par = ew >> 2;
-    const bool go = n > 0 && mbar_wait(&imgfull[0], 0);
-    for (int i = par, s = 0, use = 0; go && i < n; i += 2) {  // item i sits in group i / 2: stage s, pass use
+    if constexpr (SI) {
+      if (n_img > 0) {
+        named_sync(2, 512);
+        sq_part<4>(qT, smem + L::OFF_S, up, n_img < 2 ? n_img : 2, 256 + 32 * ew + lane);
+        named_sync(2, 512);
+      }
+    }
+    for (int i = par, s = 0, use = 0; i < n; i += 2) {  // item i sits in group i / 2: stage s, pass use
       const int b = i % L::NA, ua = i / L::NA;
       if (!mbar_wait(&full[s], use & 1)) break;
       if (ua >= 1 && !mbar_wait(&mdone[b], (ua - 1) & 1)) break;  // MMAs of item i - NA have read A[b]
@@ -559,7 +608,8 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
     if (n_img > 0) {
       // every prep / epilogue warp gets here once, before any wait that can give up: a
       // named barrier (its first sync also publishes alpha)
-      make_images<KB, SI>(a, pr, n_img < 2 ? n_img : 2, imgs, imgs + L::IMG, qT, uT, up, alpha, red, et,
+      make_images<KB, SI, true>(a, pr, n_img < 2 ? n_img : 2, imgs, imgs + L::IMG, qT, uT, up, alpha, red,
+                                smem + L::OFF_S, true, et,
                           [] { named_sync(1, 256); });
       if (et == 0) {
         mbar_arrive(&imgfull[0]);
@@ -576,9 +626,10 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
         if (kn >= 2 && kn < n_img) {
           mbar_wait(&imgfree[kn & 1], ((kn - 2) >> 1) & 1);  // on a time-out the fault word is set; go on
           PrepRegs pr2;
-          prep_load<SI>(a, head + 1, 1, et, pr2);
+          prep_load<SI>(a, head + 1, 1, et, pr2, false);
           uint8_t* slot = imgs + (kn & 1) * L::IMG;
-          make_images<KB, SI>(a, pr2, 1, slot, slot, qT, uT, up, alpha, red, et, [&] { gs.sync(lane); });
+          make_images<KB, SI, false>(a, pr2, 1, slot, slot, qT, uT, up, alpha, red, smem + L::OFF_S, false, et,
+                                     [&] { gs.sync(lane); });
           if (et == 0) mbar_arrive(&imgfull[kn & 1]);
         }
       }
