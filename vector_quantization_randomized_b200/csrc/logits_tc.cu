@@ -100,6 +100,11 @@ struct TL {
   static constexpr int NA = (4 * ACOLS + 2 * ACC <= 512) ? 4 : 2;
   static constexpr int NB = (NA * ACOLS + 4 * ACC <= 512) ? 4 : 2;
   static_assert(NA * ACOLS + NB * ACC <= 512, "tensor-memory budget");
+  // With one A buffer per parity (NA = 2) a buffer is filled and consumed in two halves
+  // (planes [0, NL) and [NL, NP)), each with its own barriers, so the expansion of an item's
+  // first half can start once the MMAs of the previous item of its parity have read that half.
+  static constexpr bool SPLIT = NA == 2;
+  static constexpr int NL = SPLIT ? 3 : NP;
   static constexpr int W_EXP0 = 3, W_EPI0 = 11;
   static constexpr int NTHREADS = 19 * 32;
   static constexpr int OFF_IMG = 1024;
@@ -388,8 +393,8 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // [MAX_STAGES] stage loaded
   uint64_t* empty = full + MAX_STAGES;                 // [MAX_STAGES] stage read by the 8 expansion warps
-  uint64_t* afull = empty + MAX_STAGES;                // [4] A buffer written (4 arrivals)
-  uint64_t* mdone = afull + 4;                         // [4] MMAs of the item done: its A buffer is free (1)
+  uint64_t* afull = empty + MAX_STAGES;                // [4] A buffer (SPLIT: half 2b + h) written (4 arrivals)
+  uint64_t* mdone = afull + 4;                         // [4] its MMAs done: the buffer (half) is free (1)
   uint64_t* cfull = mdone + 4;                         // [4] accumulator set full (1)
   uint64_t* accfree = cfull + 4;                       // [4] accumulator set read (4)
   uint64_t* imgfull = accfree + 4;                     // [2] B image ready (1)
@@ -510,23 +515,41 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
       }
       if ((i & 1) != par) continue;
       const int b = i % L::NA, ua = i / L::NA, c = i % L::NB, cu = i / L::NB;
-      if (!mbar_wait(&afull[b], ua & 1)) break;
+      const int h0 = L::SPLIT ? 2 * b : b;  // barrier of the buffer's first half (or of the buffer)
+      if (!mbar_wait(&afull[h0], ua & 1)) break;
       if (cu >= 1 && !mbar_wait(&accfree[c], (cu - 1) & 1)) break;
       __syncwarp();  // elect.sync needs the whole warp converged
       tc_fence_after();
       const uint32_t dacc = acc_col(c);
       const uint32_t abuf = a_col(b);
       const uint64_t dc = smem_desc(simg + L::IMG_C, 256, 128);
+      const uint64_t ds = smem_desc(simg + L::IMG_S, 256, 128);
+      // K step u of plane P = u / 4: 8 A columns (32 bytes), 512 bytes of image
+      auto plane_mmas = [&](int P) {
+        if (P < L::NT) {
 #pragma unroll
-      for (int u = 0; u < L::CSTEPS; ++u)  // K step u: 8 A columns (32 bytes), 512 bytes of image
-        umma_i8_ts_elect(dacc, abuf + 8u * u, dc + (uint64_t)(32 * u), idesc, u > 0 ? 1u : 0u);
-      if constexpr (SI) {
-        const uint64_t ds = smem_desc(simg + L::IMG_S, 256, 128);
+          for (int ks = 0; ks < 4; ++ks)
+            umma_i8_ts_elect(dacc, abuf + 32u * P + 8u * ks, dc + (uint64_t)(32 * (4 * P + ks)), idesc,
+                             (P > 0 || ks > 0) ? 1u : 0u);
+        } else {
 #pragma unroll
-        for (int u = 0; u < L::SSTEPS; ++u)
-          umma_i8_ts_elect(dacc + 16u, abuf + 32u * L::NT + 8u * u, ds + (uint64_t)(32 * u), idesc, u > 0 ? 1u : 0u);
+          for (int ks = 0; ks < 4; ++ks)
+            umma_i8_ts_elect(dacc + 16u, abuf + 32u * P + 8u * ks, ds + (uint64_t)(32 * ks), idesc, ks > 0 ? 1u : 0u);
+        }
+      };
+#pragma unroll
+      for (int P = 0; P < L::NL; ++P) plane_mmas(P);
+      if constexpr (L::SPLIT) {
+        umma_commit_elect(&mdone[h0]);
+        if (!mbar_wait(&afull[h0 + 1], ua & 1)) break;
+        __syncwarp();
+        tc_fence_after();
+#pragma unroll
+        for (int P = L::NL; P < L::NP; ++P) plane_mmas(P);
+        umma_commit_elect(&mdone[h0 + 1]);
+      } else {
+        umma_commit_elect(&mdone[b]);
       }
-      umma_commit_elect(&mdone[b]);
       umma_commit_elect(&cfull[c]);
     }
     __syncwarp();
@@ -547,8 +570,9 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
     }
     for (int i = par, s = 0, use = 0; i < n; i += 2) {  // item i sits in group i / 2: stage s, pass use
       const int b = i % L::NA, ua = i / L::NA;
+      const int h0 = L::SPLIT ? 2 * b : b;
       if (!mbar_wait(&full[s], use & 1)) break;
-      if (ua >= 1 && !mbar_wait(&mdone[b], (ua - 1) & 1)) break;  // MMAs of item i - NA have read A[b]
+      if (ua >= 1 && !mbar_wait(&mdone[h0], (ua - 1) & 1)) break;  // MMAs of item i - NA have read A[b] (half 0)
       const uint8_t* st = ring + s * L::STAGE + (i % GI) * 4 * L::TILEB + qd * L::TILEB + lane * 16;
       uint4 pw[KB + SI];
 #pragma unroll
@@ -563,8 +587,21 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
                            pw[0].w ^ pw[1].w ^ pw[2].w);
       if constexpr (SI) it[L::NT] = pw[KB];
       const uint32_t lanebase = a_col(b) + ((uint32_t)(32 * qd) << 16);
+      bool okh = true;
 #pragma unroll
       for (int P = 0; P < L::NP; ++P) {
+        if (L::SPLIT && P == L::NL) {  // first half done; the second half's previous MMAs must be done
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afull[h0]);
+          if (ua >= 1 && !mbar_wait(&mdone[h0 + 1], (ua - 1) & 1)) {
+            okh = false;
+            break;
+          }
+          __syncwarp();
+          tc_fence_after();
+        }
 #pragma unroll
         for (int cg = 0; cg < 2; ++cg) {
           uint32_t r[16];
@@ -579,10 +616,11 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
           tmem_st16(lanebase + 32 * P + 16 * cg, r);
         }
       }
+      if (!okh) break;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[b]);
+      if (lane == 0) mbar_arrive(&afull[L::SPLIT ? h0 + 1 : b]);
     }
   } else {
     // ---------------- query preparation, then the epilogue ----------------
