@@ -88,9 +88,9 @@ __device__ __forceinline__ int cofs(int row, int k) { return (k >> 3) * SLAB + (
 template <bool PROD, bool GEMM>
 struct RL {
   static constexpr int NX = GEMM ? 1 : (PROD ? 2 : 4);  // input tiles (TMA source) / the projected tile
-  static constexpr int NG = GEMM ? (PROD ? 5 : 8) : 0;   // GEMM K-block stages
-  static constexpr int KBLK = 32;                        // GEMM K block (elements)
-  static constexpr int GSTAGE = 2 * (KBLK / 8) * SLAB;   // x block + weight block (16 KB)
+  static constexpr int NG = GEMM ? (PROD ? 2 : 4) : 0;   // GEMM K-block stages
+  static constexpr int KBLK = 64;                        // GEMM K block (elements): one 128-byte swizzled row
+  static constexpr int GSTAGE = 2 * (KBLK / 8) * SLAB;   // x block + weight block (16 KB each), 1 TMA copy each
   static constexpr int HD = 0;                           // H D, canonical (N = out coordinate, K = in)
   static constexpr int SS = HD + TILE_B;                 // S, canonical (N = projection, K = coordinate)
   static constexpr int XS = SS + (PROD ? TILE_B : 0);    // [NX] input tiles
@@ -183,8 +183,9 @@ struct CoderR {
 template <bool GEMM>
 __device__ __forceinline__ void row_vector(const RArgs& a, int64_t tile, int r, int64_t& vg, bool& valid, bool& own) {
   if constexpr (GEMM) {
-    const int64_t tph = (a.n_tok + TV - 1) / TV;
-    const int64_t h = tile / tph, t = (tile - h * tph) * TV + r;
+    // GEMM tiles are numbered head-fastest (tile = m-tile * n_heads + head), so the CTAs that run
+    // at the same time share their token rows and read them from HBM once
+    const int64_t h = tile % a.n_heads, t = (tile / a.n_heads) * TV + r;
     vg = h * a.n_tok + t;
     valid = t < a.n_tok;
     own = valid || (h == a.n_heads - 1 && vg < a.n_pad);  // the zero tail of the last code tile
@@ -333,18 +334,17 @@ __global__ void __launch_bounds__(RL<PROD, GEMM>::NTHREADS, 1)
   const int64_t t0 = blockIdx.x, ts = gridDim.x;
   const int nt = t0 < n_tiles ? (int)((n_tiles - 1 - t0) / ts) + 1 : 0;  // tiles of this CTA
   auto tile_of = [&](int i) { return t0 + (int64_t)i * ts; };
-  const int nkb = GEMM ? a.hidden / L::KBLK : 0;
+  const int nkb = GEMM ? (a.hidden + L::KBLK - 1) / L::KBLK : 0;  // a last half block reads zeros past hidden
 
   if (warp == 0) {
     // ---------------- producer: input tiles, or the GEMM's K blocks, by TMA ----------------
     if (lane == 0) {
       if constexpr (GEMM) {
-        const int64_t tph = (a.n_tok + TV - 1) / TV;
         int64_t g = 0;
         bool ok = true;
         for (int i = 0; i < nt && ok; ++i) {
-          const int64_t tile = tile_of(i), h = tile / tph;
-          const int y = (int)((tile - h * tph) * TV), yw = (int)(h * TV);
+          const int64_t tile = tile_of(i), h = tile % a.n_heads;
+          const int y = (int)((tile / a.n_heads) * TV), yw = (int)(h * TV);
           for (int kb = 0; kb < nkb; ++kb, ++g) {
             const int s = (int)(g % NG);
             if (g >= NG && !mbar_wait(&gempty[s], (uint32_t)(((g - NG) / NG) & 1))) {
@@ -353,11 +353,8 @@ __global__ void __launch_bounds__(RL<PROD, GEMM>::NTHREADS, 1)
             }
             uint8_t* dst = smem + L::GS + s * L::GSTAGE;
             mbar_expect_tx(&gfull[s], L::GSTAGE);
-#pragma unroll
-            for (int j = 0; j < L::KBLK / 8; ++j) {
-              tma_load_2d(dst + j * SLAB, &tmap, L::KBLK * kb + 8 * j, y, &gfull[s]);
-              tma_load_2d(dst + (L::KBLK / 8 + j) * SLAB, &tmap_w, L::KBLK * kb + 8 * j, yw, &gfull[s]);
-            }
+            tma_load_2d(dst, &tmap, L::KBLK * kb, y, &gfull[s]);  // 128 rows x 128 bytes, swizzled
+            tma_load_2d(dst + L::GSTAGE / 2, &tmap_w, L::KBLK * kb, yw, &gfull[s]);
           }
         }
         for (int64_t i = (g > NG ? g - NG : 0); i < g; ++i) mbar_wait(&gfull[i % NG], (uint32_t)((i / NG) & 1));
@@ -499,12 +496,11 @@ __global__ void __launch_bounds__(RL<PROD, GEMM>::NTHREADS, 1)
           __syncwarp();
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + L::GS + s * L::GSTAGE);
-          const uint64_t ad = smem_desc(sa, SLAB, 128);
-          const uint64_t bd = smem_desc(sa + (L::KBLK / 8) * SLAB, SLAB, 128);
+          const uint64_t ad = smem_desc_sw128(sa);
+          const uint64_t bd = smem_desc_sw128(sa + L::GSTAGE / 2);
 #pragma unroll
-          for (int ks = 0; ks < L::KBLK / 16; ++ks)
-            umma_16_ss_elect(ycol(b), ad + (uint64_t)(ks * (2 * SLAB >> 4)), bd + (uint64_t)(ks * (2 * SLAB >> 4)),
-                             idg, (kb | ks) ? 1u : 0u);
+          for (int ks = 0; ks < L::KBLK / 16; ++ks)  // K step: 32 bytes along the swizzled rows
+            umma_16_ss_elect(ycol(b), ad + (uint64_t)(2 * ks), bd + (uint64_t)(2 * ks), idg, (kb | ks) ? 1u : 0u);
           umma_commit_elect(&gempty[s]);
           try_small(i);
         }
@@ -654,8 +650,7 @@ __global__ void __launch_bounds__(RL<PROD, GEMM>::NTHREADS, 1)
       int64_t vg;
       bool valid, own;
       row_vector<GEMM>(a, tile_of(i), v, vg, valid, own);
-      const int64_t tph = (a.n_tok + TV - 1) / TV;
-      const int64_t hh = tile_of(i) / tph, tok = vg - hh * a.n_tok;
+      const int64_t hh = tile_of(i) % a.n_heads, tok = vg - hh * a.n_tok;
       uint8_t* xs = smem + L::XS;
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
@@ -895,9 +890,9 @@ extern "C" int tq_project_quantize(const tq_params* p, const void* x, int64_t n_
   if (!aligned(codes, 16) || !aligned(norms, 2) || (rnorms && !aligned(rnorms, 2)))
     return set_error(TQ_EINVAL, "tq_project_quantize: codes must be 16-byte aligned, norms 2-byte aligned");
   CUtensorMap mx, mw;
-  rc = make_tmap_2d_u16(&mx, x, (uint64_t)hidden, (uint64_t)n_tok, (uint64_t)ld_x * 2, 8, TV);
+  rc = make_tmap_2d_u16(&mx, x, (uint64_t)hidden, (uint64_t)n_tok, (uint64_t)ld_x * 2, 64, TV, true);
   if (rc) return rc;
-  rc = make_tmap_2d_u16(&mw, w, (uint64_t)hidden, (uint64_t)n_heads * 128, (uint64_t)ld_w * 2, 8, TV);
+  rc = make_tmap_2d_u16(&mw, w, (uint64_t)hidden, (uint64_t)n_heads * 128, (uint64_t)ld_w * 2, 64, TV, true);
   if (rc) return rc;
   RArgs a = {};
   a.n_vec = (int64_t)n_heads * n_tok;

@@ -103,6 +103,14 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
   return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46);  // version 1 (sm_100), base 0, no swizzle
 }
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 bytes (64 16-bit
+// elements) whose 16-byte chunks are XOR-ed by row % 8, 8-row groups 1024 bytes apart (what a
+// TMA copy with 128-byte swizzle writes).  The tile starts on a 1024-byte boundary; a K step
+// of 16 elements inside the row adds 32 bytes to the start address.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+         (2ull << 61);  // leading offset unused (16 B), stride 1024 B, version 1, 128-byte swizzle
+}
 // Instruction descriptor for kind::f16: f16 x f16 -> f32, both K-major, M x N.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4)                      // D format f32

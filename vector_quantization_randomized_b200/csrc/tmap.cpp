@@ -27,7 +27,7 @@ EncodeTiled encode_fn() {
 }  // namespace
 
 int make_tmap_2d_u16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
-                     uint32_t box_cols, uint32_t box_rows) {
+                     uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
   EncodeTiled fn = encode_fn();
   if (!fn) return set_error(TQ_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t dims[2] = {cols, rows};
@@ -35,7 +35,9 @@ int make_tmap_2d_u16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(TQ_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return TQ_OK;
