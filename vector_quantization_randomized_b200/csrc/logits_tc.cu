@@ -31,11 +31,13 @@
 //               and one lane, chosen by elect.sync, issues, with the
 //               descriptors of a whole item unrolled from two base values;
 //   warps 3-10  expansion: stage -> masked words -> tcgen05.st into one of two
-//               or four A buffers (warp = lane quadrant; 3-6 even items, 7-10 odd);
+//               or four A buffers (warp = lane quadrant; 3-6 even items, 7-10 odd;
+//               with two buffers each is written and read in two halves).  They
+//               first take a share of u = S q_rot for the CTA's first image;
 //   warps 11-18 query preparation into a ring of two B images, then the
-//               epilogue: tcgen05.ld of the partial accumulators, digit
+//               epilogue: tcgen05.ld of the item's accumulator set, digit
 //               combination, norms (plain loads issued two items ahead), logits
-//               (warp = lane quadrant).
+//               (warp = lane quadrant; 11-14 even items, 15-18 odd).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -203,9 +205,10 @@ __device__ __forceinline__ void sq_part(const float4* qT, const uint8_t* sS, flo
 }
 
 // B images of n_img (1 or 2) consecutive KV heads into img0 / img1, by the 256
-// threads of warps 13-20 (et = 0..255) from the loads in pr.  Steps:
+// threads of warps 11-18 (et = 0..255) from the loads in pr.  Steps:
 // q_rot = H D q / sqrt(128) (warp per query: image ew / 4, query ew % 4);
-// u = S q_rot (thread = row of S x half of the coordinates, both images);
+// u = S q_rot (sq_part: a half row of S per thread, or, WIDE, a quarter row with
+// the 8 expansion warps joining between two 512-thread named barriers);
 // per-query scales 2^F, 2^G putting the largest weight just below 2^23; digits.
 template <int KB, int SI, bool WIDE, class Sync>
 __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* img0, uint8_t* img1, float4* qT,
@@ -624,7 +627,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
     }
   } else {
     // ---------------- query preparation, then the epilogue ----------------
-    // warps 13-16 take the even items, 17-20 the odd ones; each covers one lane quadrant
+    // warps 11-14 take the even items, 15-18 the odd ones; each covers one lane quadrant
     // (32 keys) and all the query heads of the KV head
     const int et = threadIdx.x - 32 * W_EPI0;
     const int ew = warp - W_EPI0;
