@@ -62,9 +62,18 @@ def test_ragged_tokens_three_heads(bits, mode):
 
 
 def test_layer_width_hidden_4096():
-    # the Llama-3.1-8B layer width: 128 K blocks of 32 per tile
+    # the Llama-3.1-8B layer width: 64 K blocks of 64 per tile
     n_tok, n_heads = 256, 2
     r = _run(n_tok, 4096, n_heads, 3, tq.TQ_MODE_PROD, seed=32)
+    _check_projection(r, n_heads)
+    compare_codes(r["op"], r["k"], r["codes"], r["norms"], r["rn"])
+
+
+@pytest.mark.parametrize("mode", [tq.TQ_MODE_PROD, tq.TQ_MODE_MSE])
+def test_hidden_half_k_block(mode):
+    # hidden 160 = two and a half K blocks of 64: the last block's box reads zeros past the row end
+    n_tok, n_heads = 200, 2
+    r = _run(n_tok, 160, n_heads, 3, mode, seed=36)
     _check_projection(r, n_heads)
     compare_codes(r["op"], r["k"], r["codes"], r["norms"], r["rn"])
 
