@@ -414,6 +414,7 @@ __global__ void __launch_bounds__(TL<KB, SI>::NTHREADS, 1) logits_tc_kernel(cons
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.stages;
+  grid_dependents_launch();  // every global write below follows this grid's own dependency wait
   // this CTA's items [i0, i1) = [b n_items / G, (b + 1) n_items / G), in 32-bit arithmetic
   // (a 64-bit division costs hundreds of cycles on the start-up path)
   const uint32_t bx = blockIdx.x;

@@ -156,6 +156,10 @@ struct Scan {
 // Programmatic dependent launch: wait until the preceding grid (query prep)
 // has completed and its writes are visible.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+// Let the next grid in the stream (launched with programmatic stream serialization) be
+// scheduled now: its CTAs take each SM as this grid's CTAs leave it, and wait in their own
+// grid_dependency_wait for this grid to complete before they read its outputs.
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
 // Combine the digit rows of an accumulator pair: thread (g, t) holds rows g,
 // g+8 (digits g>>2 and 2+(g>>2) of query g&3) for keys 2t, 2t+1.  Returns, in
