@@ -129,6 +129,13 @@ __device__ __forceinline__ float pow2(int k) {
   return (k >= -126 && k <= 127) ? __uint_as_float((uint32_t)(127 + k) << 23) : ldexpf(1.f, k);
 }
 
+// warp maximum of a float (redux.sync; finite, non-negative values here)
+__device__ __forceinline__ float warp_max_redux(float v) {
+  float r;
+  asm volatile("redux.sync.max.NaN.f32 %0, %1, 0xffffffff;\n" : "=f"(r) : "f"(v));
+  return r;
+}
+
 // Global loads of the query preparation, issued early so their latency overlaps
 // other work: warp ew's query (image ew / 4, query ew % 4), the sign flips and
 // 16-byte chunks et + 256 k of S (coalesced; make_images stores them to shared
@@ -249,7 +256,7 @@ __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* im
       mx = fmaxf(mx, fabsf(v));
     }
     sum = warp_sum(sum);
-    mx = warp_max(mx);
+    mx = warp_max_redux(mx);
     if (lane == 0) {
       rd[4 * jq] = sum;
       rd[4 * jq + 1] = mx;
@@ -295,14 +302,15 @@ __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* im
   }
   if (kq < n_img) {  // scales and per-query scalars: warp = (image kq, query jq)
     float su = 0.f, mu = 0.f;
-    if constexpr (SI) {
-      for (int i = lane; i < a.m; i += 32) {
-        const float v = uTf[512 * kq + 4 * i + jq];
+    if constexpr (SI) {  // m = 128 rows of S
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float v = uTf[512 * kq + 4 * (lane + 32 * k) + jq];
         su += v;
         mu = fmaxf(mu, fabsf(v));
       }
       su = warp_sum(su);
-      mu = warp_max(mu);
+      mu = warp_max_redux(mu);
     }
     float amax = 0.f;
 #pragma unroll
@@ -325,8 +333,9 @@ __device__ void make_images(const TArgs& a, PrepRegs& pr, int n_img, uint8_t* im
   constexpr int PER = 4 * L::NP * 32;
   for (int e = et; e < n_img * PER; e += 256) {
     const int im = e / PER, e2 = e - im * PER;
-    const int w = e2 & 3, c = (e2 >> 2) & 7, pq = e2 >> 5;
-    const int q = pq / L::NP, P = pq - q * L::NP;
+    // lanes run over (w, bit 0 of q, 4 bit classes): their word stores fall in 8 banks
+    const int w = e2 & 3, c = (e2 >> 3) & 7, pq = e2 >> 6;
+    const int qh = pq / L::NP, P = pq - qh * L::NP, q = 2 * qh + ((e2 >> 2) & 1);
     const bool cen = P < L::NT;
     const float* r2 = red + 16 * im;
     const float scale = cen ? 2.f * alpha[P] * r2[4 * q + 2] : 2.f * r2[4 * q + 3];
