@@ -15,8 +15,10 @@
 //    - TMA: warp 0 loads the tile as 16 boxes of 8 elements x 128 rows, which
 //      land as the K-major canonical layout of an MMA operand (K chunk k8 of
 //      every row in one 2 KB slab); rows past the end and columns past d read 0;
-//    - projection: warp 0 streams K blocks of 32 of the layer input x (128
-//      tokens) and of the head's weight rows by TMA into a ring, warp 1 runs the
+//    - projection: warp 0 streams K blocks of 64 of the layer input x (128
+//      tokens) and of the head's weight rows into a ring, one TMA box with
+//      128-byte swizzle per operand and block (tiles numbered head-fastest, so
+//      the CTAs running together share their token rows); warp 1 runs the
 //      bf16 GEMM x W_h^T into tensor memory (M = 128 tokens, N = 128, fp32), and
 //      warps 10-13 read the accumulator back, round it to bf16 and write the
 //      tile in the canonical layout (optionally also to memory);
