@@ -124,6 +124,40 @@ def test_validation_rejects_null_and_misaligned():
     assert lib.tq_code_bytes(-1, 1, 1, 1) == -1
 
 
+def test_project_quantize_validation():
+    """tq_project_quantize rejects bad shapes, NULL and misaligned buffers on the host, before
+    any tensor map or launch; n_tok == 0 is a no-op."""
+    st, keep = _fake_params()  # d = d_pad = 128, product mode, m = 128
+    f = tq._lib.tq_project_quantize
+    buf = np.zeros(4096, np.uint8)
+    b = (buf.ctypes.data + 15) // 16 * 16
+    ok = dict(x=b, n_tok=4, ld_x=64, hidden=64, w=b, n_heads=1, ld_w=64, codes=b, norms=b, rnorms=b, k_out=None,
+              ld_k=0)
+
+    def call(params=st, **kw):
+        a = dict(ok, **kw)
+        return f(ctypes.byref(params), a["x"], a["n_tok"], a["ld_x"], a["hidden"], a["w"], a["n_heads"], a["ld_w"],
+                 a["codes"], a["norms"], a["rnorms"], a["k_out"], a["ld_k"], None)
+
+    assert call(hidden=48, ld_x=48, ld_w=48) == tq.TQ_EINVAL          # hidden not a multiple of 32
+    assert call(hidden=0) == tq.TQ_EINVAL
+    assert call(n_heads=0) == tq.TQ_EINVAL
+    assert call(n_tok=-1) == tq.TQ_EINVAL
+    assert call(n_tok=0, x=None, w=None, codes=None, norms=None, rnorms=None) == tq.TQ_OK
+    assert call(x=None) == tq.TQ_EINVAL
+    assert call(rnorms=None) == tq.TQ_EINVAL                           # product mode needs residual norms
+    assert call(x=b + 2) == tq.TQ_EINVAL                               # x not 16-byte aligned
+    assert call(ld_x=32) == tq.TQ_EINVAL                               # ld_x < hidden
+    assert call(ld_w=68) == tq.TQ_EINVAL                               # row stride not a multiple of 8
+    assert call(k_out=b, ld_k=64) == tq.TQ_EINVAL                      # ld_k < 128 * n_heads
+    assert call(codes=b + 8) == tq.TQ_EINVAL                           # codes not 16-byte aligned
+    st2, keep2 = _fake_params(d=200, d_pad=256, m=256)
+    assert call(params=st2) == tq.TQ_EUNSUPPORTED                      # d_pad 256
+    st3, keep3 = _fake_params(m=64)
+    assert call(params=st3) == tq.TQ_EUNSUPPORTED                      # product mode with m < 128
+    assert tq.tq_last_error()
+
+
 @pytest.mark.parametrize("d_pad", [128, 256, 1024, 4096])
 @pytest.mark.parametrize("w", [1, 2, 3])
 def test_polar_tables_match_oracle(d_pad, w):
