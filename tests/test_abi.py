@@ -158,6 +158,39 @@ def test_project_quantize_validation():
     assert tq.tq_last_error()
 
 
+def test_sliced_decode_validation():
+    """tq_decode_attn with token-sliced values (the tensor-memory decode) rejects the shapes it does not
+    serve and bad buffers on the host; batch == 0 is a no-op; the sparse and partial forms refuse it."""
+    kp, keep_k = _fake_params(bits=3)                                        # keys: product, m = 128
+    vp, keep_v = _fake_params(bits=3, mode=tq.TQ_MODE_MSE, m=0, layout=tq.TQ_LAYOUT_SLICED)
+    f = tq._lib.tq_decode_attn
+    buf = np.zeros(4096, np.uint8)
+    b = (buf.ctypes.data + 15) // 16 * 16
+    ok = dict(kp=kp, q=b, batch=1, hq=4, hkv=1, kc=b, kn=b, krn=b, vc=b, vn=b, sl=b, T=64, out=b, ws=b,
+              wsb=1 << 40)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(ctypes.byref(a["kp"]), ctypes.byref(vp), a["q"], a["batch"], a["hq"], a["hkv"], a["kc"], a["kn"],
+                 a["krn"], a["vc"], a["vn"], a["sl"], a["T"], 0.0, a["out"], a["ws"], a["wsb"], None)
+
+    assert call(hq=8) == tq.TQ_EUNSUPPORTED                  # 8 query heads per KV head
+    assert call(T=48) == tq.TQ_EUNSUPPORTED                  # max_tokens not a multiple of 32
+    k64, keep64 = _fake_params(bits=3, m=64)
+    assert call(kp=k64) == tq.TQ_EUNSUPPORTED                # keys with m < 128
+    k256, keep256 = _fake_params(d=200, d_pad=256, bits=3, m=256)
+    assert call(kp=k256) == tq.TQ_EUNSUPPORTED               # d_pad 256
+    assert call(batch=-1) == tq.TQ_EINVAL
+    assert call(batch=0, q=None, kc=None, out=None, ws=None) == tq.TQ_OK
+    assert call(q=None) == tq.TQ_EINVAL
+    assert call(vn=b + 2) == tq.TQ_EINVAL                    # norms not 16-byte aligned
+    assert call(wsb=16) == tq.TQ_EINVAL                      # workspace too small
+    g = tq._lib.tq_decode_attn_sparse
+    assert g(ctypes.byref(kp), ctypes.byref(vp), b, 1, 4, 1, b, b, b, b, b, b, 64, 0.0, 1e-3, b, b, 1 << 40,
+             None) == tq.TQ_EUNSUPPORTED                     # Sparse V reads plane-layout values
+    assert tq.tq_last_error()
+
+
 @pytest.mark.parametrize("d_pad", [128, 256, 1024, 4096])
 @pytest.mark.parametrize("w", [1, 2, 3])
 def test_polar_tables_match_oracle(d_pad, w):
