@@ -191,6 +191,21 @@ def test_sliced_decode_validation():
     assert tq.tq_last_error()
 
 
+def test_logits_d256_kb3_validation():
+    """tq_logits at d_pad 256 with 3 index bits (the search scan writing every score): a ragged key
+    count across several KV heads and a short workspace are refused on the host."""
+    st, keep = _fake_params(d=200, d_pad=256, bits=4, m=256)
+    f = tq._lib.tq_logits
+    buf = np.zeros(4096, np.uint8)
+    b = (buf.ctypes.data + 15) // 16 * 16
+    need = tq._lib.tq_logits_workspace(ctypes.byref(st), 8)
+    assert need > 0
+    # q, n_q, group, codes, norms, rnorms, n_keys, n_kv_heads, logits, workspace, bytes, stream
+    assert f(ctypes.byref(st), b, 8, 4, b, b, b, 100, 2, b, b, need, None) == tq.TQ_EUNSUPPORTED
+    assert f(ctypes.byref(st), b, 8, 4, b, b, b, 128, 2, b, b, need - 1, None) == tq.TQ_EINVAL
+    assert f(ctypes.byref(st), b, 8, 4, b, b, b, 0, 2, b, b, 0, None) == tq.TQ_OK   # no keys: nothing to do
+
+
 @pytest.mark.parametrize("d_pad", [128, 256, 1024, 4096])
 @pytest.mark.parametrize("w", [1, 2, 3])
 def test_polar_tables_match_oracle(d_pad, w):
