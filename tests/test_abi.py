@@ -206,6 +206,54 @@ def test_logits_d256_kb3_validation():
     assert f(ctypes.byref(st), b, 8, 4, b, b, b, 0, 2, b, b, 0, None) == tq.TQ_OK   # no keys: nothing to do
 
 
+def test_host_validation_of_the_other_entry_points():
+    """Dequantize, logits with a row stride, search, the sharded merges and the partial decode refuse
+    bad arguments on the host (and empty calls are no-ops), before anything reaches the GPU."""
+    lib = tq._lib
+    st, keep = _fake_params()                                              # d 128, product, b = 4, m = 128
+    sm, keep_m = _fake_params(mode=tq.TQ_MODE_MSE, m=0, bits=3)           # MSE values
+    sl, keep_s = _fake_params(mode=tq.TQ_MODE_MSE, m=0, bits=3, layout=tq.TQ_LAYOUT_SLICED)
+    s256, keep2 = _fake_params(d=200, d_pad=256, bits=4, m=256)
+    buf = np.zeros(4096, np.uint8)
+    b = (buf.ctypes.data + 15) // 16 * 16
+    R = ctypes.byref
+    # tq_dequantize(p, codes, norms, rnorms, n_vec, out, ld, stream)
+    assert lib.tq_dequantize(R(st), b, b, b, 0, None, 0, None) == tq.TQ_OK
+    assert lib.tq_dequantize(R(st), b, b, b, -1, b, 128, None) == tq.TQ_EINVAL
+    assert lib.tq_dequantize(R(st), b, b, None, 4, b, 128, None) == tq.TQ_EINVAL      # product mode, no rnorms
+    assert lib.tq_dequantize(R(st), b, b, b, 4, b, 64, None) == tq.TQ_EINVAL          # ld < d
+    assert lib.tq_dequantize(R(st), b + 4, b, b, 4, b, 128, None) == tq.TQ_EINVAL     # codes misaligned
+    # tq_logits_ld(p, q, n_q, group, codes, norms, rnorms, n_keys, n_kv_heads, logits, ld, ws, ws_bytes, stream)
+    assert lib.tq_logits_ld(R(st), b, 4, 4, b, b, b, 256, 1, b, 128, b, 1 << 30, None) == tq.TQ_EINVAL  # ld < n_keys
+    assert lib.tq_logits_ld(R(sl), b, 4, 4, b, b, None, 256, 1, b, 256, b, 1 << 30, None) == tq.TQ_EUNSUPPORTED
+    # tq_search_workspace / tq_search_topk(p, q, n_q, codes, norms, rnorms, n_db, k, ids, scores, ws, bytes, s)
+    assert lib.tq_search_workspace(R(s256), 16, 1000, 0) == -1                      # k < 1
+    need = lib.tq_search_workspace(R(s256), 16, 1000, 10)
+    assert need > 0
+    assert lib.tq_search_topk(R(s256), b, 0, None, None, None, 1000, 10, None, None, None, 0, None) == tq.TQ_OK
+    assert lib.tq_search_topk(R(s256), b, 16, b, b, b, 5, 10, b, b, b, need, None) == tq.TQ_EINVAL   # n_db < k
+    assert lib.tq_search_topk(R(s256), b, 16, b, b, b, 1000, 0, b, b, b, need, None) == tq.TQ_EUNSUPPORTED
+    assert lib.tq_search_topk(R(s256), b, 16, b, b, b, 1000, 10, b, b, b, need - 1, None) == tq.TQ_EINVAL
+    assert lib.tq_search_topk(R(s256), b, 16, b + 8, b, b, 1000, 10, b, b, b, need, None) == tq.TQ_EINVAL
+    assert lib.tq_search_topk(R(sl), b, 16, b, b, None, 1000, 10, b, b, b, need, None) == tq.TQ_EUNSUPPORTED
+    # tq_search_merge(ids, scores, n_parts, id_offsets, n_q, k, out_ids, out_scores, stream)
+    assert lib.tq_search_merge(b, b, 0, b, 4, 10, b, b, None) == tq.TQ_EINVAL        # no parts
+    assert lib.tq_search_merge(b, b, 2, b, 4, 0, b, b, None) == tq.TQ_EINVAL         # k < 1
+    assert lib.tq_search_merge(b, b, 2, b, 0, 10, None, None, None) == tq.TQ_OK      # no queries
+    assert lib.tq_search_merge(None, b, 2, b, 4, 10, b, b, None) == tq.TQ_EINVAL
+    assert lib.tq_search_merge(b + 2, b, 2, b, 4, 10, b, b, None) == tq.TQ_EINVAL    # ids misaligned
+    # tq_decode_attn_partial_bytes / tq_decode_attn_partial / tq_decode_attn_merge
+    assert lib.tq_decode_attn_partial_bytes(R(sm), 2, 8) == 2 * 8 * (128 + 2) * 4
+    assert lib.tq_decode_attn_partial_bytes(R(sm), -1, 8) == -1
+    assert lib.tq_decode_attn_partial(R(st), R(sm), b, 1, 4, 1, b, b, b, b, b, b, 64, 0.0, None, b, 1 << 30,
+                                      None) == tq.TQ_EINVAL                          # NULL partial
+    assert lib.tq_decode_attn_merge(R(st), b, 2, 1, 4, b, None) == tq.TQ_EUNSUPPORTED  # needs the value params
+    assert lib.tq_decode_attn_merge(R(sm), b, 0, 1, 4, b, None) == tq.TQ_EINVAL        # no parts
+    assert lib.tq_decode_attn_merge(R(sm), b, 2, 0, 4, None, None) == tq.TQ_OK         # empty batch
+    assert lib.tq_decode_attn_merge(R(sm), None, 2, 1, 4, b, None) == tq.TQ_EINVAL
+    assert tq.tq_last_error()
+
+
 @pytest.mark.parametrize("d_pad", [128, 256, 1024, 4096])
 @pytest.mark.parametrize("w", [1, 2, 3])
 def test_polar_tables_match_oracle(d_pad, w):
