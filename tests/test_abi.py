@@ -254,6 +254,35 @@ def test_host_validation_of_the_other_entry_points():
     assert tq.tq_last_error()
 
 
+def test_polar_qjl_validation():
+    """The polar code's QJL stage (tq_polar_qjl) and its logits (tq_polar_logits_prod) refuse bad
+    arguments on the host; an empty call is a no-op."""
+    lib = tq._lib
+    pp, keep = _fake_polar()
+    buf = np.zeros(4096, np.uint8)
+    b = (buf.ctypes.data + 15) // 16 * 16
+    R = ctypes.byref
+    # tq_polar_qjl(p, S, m, x, dtype, n_vec, ld, codes, signs, rnorms, stream)
+    q = lambda **kw: lib.tq_polar_qjl(R(pp), kw.get("S", b), kw.get("m", 128), kw.get("x", b),
+                                      kw.get("dtype", tq.TQ_BF16), kw.get("n_vec", 4), kw.get("ld", 128),
+                                      b, b, b, None)
+    assert q(m=48) == tq.TQ_EINVAL                                   # m not a multiple of 32
+    assert q(m=256) == tq.TQ_EINVAL                                  # m > d_pad
+    assert q(n_vec=-1) == tq.TQ_EINVAL
+    assert q(n_vec=0, x=None, S=None) == tq.TQ_OK
+    assert q(dtype=9) == tq.TQ_EINVAL
+    assert q(S=None) == tq.TQ_EINVAL
+    assert q(ld=64) == tq.TQ_EINVAL                                  # ld < d
+    assert q(x=b + 2) == tq.TQ_EINVAL                                # x not 16-byte aligned
+    # tq_polar_logits_prod(p, S, m, q, group, codes, norms, signs, rnorms, n_keys, n_kv_heads, logits, s)
+    lp = lambda p=R(pp), m=128, signs=b: lib.tq_polar_logits_prod(p, b, m, b, 4, b, b, signs, b, 64, 1, b, None)
+    assert lp(p=None) == tq.TQ_EINVAL
+    assert lp(m=0) == tq.TQ_EINVAL
+    assert lp(signs=None) == tq.TQ_EINVAL
+    assert lp(signs=b + 2) == tq.TQ_EINVAL                           # signs not 4-byte aligned
+    assert tq.tq_last_error()
+
+
 @pytest.mark.parametrize("d_pad", [128, 256, 1024, 4096])
 @pytest.mark.parametrize("w", [1, 2, 3])
 def test_polar_tables_match_oracle(d_pad, w):
